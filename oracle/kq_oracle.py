@@ -1,0 +1,281 @@
+"""CPU oracle for the KroQuant online activation quantizer (float64, numpy).
+
+TEST INFRASTRUCTURE ONLY.  This module is the checker the GPU path is compared
+against.  Only the test-suite, the package's smoke check and the CPU-baseline
+leg of the benchmark may import it; the product path never calls it and has
+no CPU fallback.  It shares no code with the CUDA library.
+
+It follows the method as the pages state it, one step at a time, with no
+blocking, fusion or reordering beyond the definitions:
+
+1. ``G_k = L_k U_k``, a 2x2 unit-determinant LU factor with three scalars,
+   ``L = [[1, 0], [a, 1]]`` and ``U = [[b, c], [0, 1/b]]``
+   (KroQuant review, "What carries the argument" and section 3.2 Eq. 6; the
+   sign convention of ``U`` is the one whose determinant is +1, see
+   ``lu_factor``).
+2. ``K^(j) = G1 (x) G2 (x) G3 (x) G4 (x) G5``, an explicit dense Kronecker
+   product, one 32x32 block per 32 channels (review, "What carries the
+   argument"; section 3.2 Eq. 4: ``T`` is block diagonal).
+3. The activation row is multiplied on the right, ``y = x T`` (review,
+   "Circularity check", Eq. 1: ``A T (W T^-T)^T = A W^T``).
+4. MXFP4 quantization of every 32-element block: one shared E8M0 power-of-two
+   scale and E2M1 elements (the OCP Microscaling formats the paper cites for
+   "MXFP4e2"; abstract and "Core claim").
+
+Readings where the pages are silent (each listed in the design doc):
+
+* the scale exponent is ``floor(log2(amax)) - 2`` (2 = the largest E2M1
+  exponent), clamped to ``[-127, 127]``; an all-zero block gets ``-127``;
+* elements round to the nearest E2M1 value, ties to the even code, and
+  saturate at +-6; the code keeps the sign bit of its input, so a negative
+  value that rounds to zero gives code ``0x8``;
+* the quantization decision is taken on the float32 value of the transformed
+  element (the kernel's precision; the pages fix none);
+* two codes per byte, the even element in the low nibble;
+* E8M0 byte ``0xFF`` decodes to NaN.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import scipy.linalg
+
+BLOCK = 32            # elements per MX block and per Kronecker block
+N_FACTORS = 5         # 32 = 2**5, one 2x2 factor per index bit
+E2M1_EMAX = 2         # exponent of the largest E2M1 value (6 = 1.5 * 2**2)
+E8M0_BIAS = 127
+
+# OCP E2M1 magnitudes, indexed by the 3-bit magnitude code.
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+# --------------------------------------------------------------------------
+# Step 1-2: the Kronecker-structured block transform
+# --------------------------------------------------------------------------
+def lu_factor(a: float, b: float, c: float) -> np.ndarray:
+    """2x2 factor ``G = L U`` with ``L = [[1,0],[a,1]]``, ``U = [[b,c],[0,1/b]]``.
+
+    Section 3.2 Eq. 6 of the KroQuant paper (as quoted by the review) writes
+    ``U = [[a, b], [0, -1/a]]``, whose determinant is -1, while the review's
+    summary and its axiom ledger call the factor "unit-determinant".  The form
+    used here keeps three scalars and has determinant +1 for every ``b != 0``.
+    """
+    a, b, c = float(a), float(b), float(c)
+    L = np.array([[1.0, 0.0], [a, 1.0]])
+    U = np.array([[b, c], [0.0, 1.0 / b]])
+    return L @ U
+
+
+def block_factors(p_j: np.ndarray) -> list:
+    """The five 2x2 factors of one block from its ``[5, 3]`` parameters."""
+    p_j = np.asarray(p_j, dtype=np.float64)
+    return [lu_factor(*p_j[k]) for k in range(N_FACTORS)]
+
+
+def kron_factors(factors) -> np.ndarray:
+    """``F1 (x) F2 (x) ... (x) F5`` as a dense matrix (numpy's Kronecker
+    convention: the first factor acts on the most significant index bit)."""
+    K = np.array([[1.0]])
+    for G in factors:
+        K = np.kron(K, G)
+    return K
+
+
+def kron_block(p_j: np.ndarray) -> np.ndarray:
+    """Dense 32x32 ``K^(j) = G1 (x) G2 (x) G3 (x) G4 (x) G5``."""
+    return kron_factors(block_factors(p_j))
+
+
+def inverse_block(p_j: np.ndarray) -> np.ndarray:
+    """``K^-1 = G1^-1 (x) ... (x) G5^-1`` (review, axiom ledger: the inverse of
+    a Kronecker product factorizes); ``G^-1 = U^-1 L^-1`` in closed form."""
+    inv = []
+    for a, b, c in np.asarray(p_j, dtype=np.float64):
+        U_inv = np.array([[1.0 / b, -c], [0.0, b]])
+        L_inv = np.array([[1.0, 0.0], [-a, 1.0]])
+        inv.append(U_inv @ L_inv)
+    return kron_factors(inv)
+
+
+def hadamard_block() -> np.ndarray:
+    """Fixed orthonormal block Hadamard ``H_32 / sqrt(32)`` (Sylvester order),
+    the comparator the paper initialises from (review, "Core claim")."""
+    return scipy.linalg.hadamard(BLOCK).astype(np.float64) / math.sqrt(BLOCK)
+
+
+def _apply_blocks(x64: np.ndarray, blocks) -> np.ndarray:
+    x64 = np.asarray(x64, dtype=np.float64)
+    M, d = x64.shape
+    y = np.empty_like(x64)
+    for j in range(d // BLOCK):
+        sl = slice(BLOCK * j, BLOCK * (j + 1))
+        y[:, sl] = x64[:, sl] @ blocks(j)
+    return y
+
+
+def transform(x64: np.ndarray, params: np.ndarray) -> np.ndarray:
+    """``y = x T`` with ``T = diag(K^(1), ..., K^(d/32))``, float64."""
+    params = np.asarray(params)
+    return _apply_blocks(x64, lambda j: kron_block(params[j]))
+
+
+def inverse_transform(y64: np.ndarray, params: np.ndarray) -> np.ndarray:
+    """``x = y T^-1``, float64."""
+    params = np.asarray(params)
+    return _apply_blocks(y64, lambda j: inverse_block(params[j]))
+
+
+def transform_hadamard(x64: np.ndarray) -> np.ndarray:
+    H = hadamard_block()
+    return _apply_blocks(x64, lambda j: H)
+
+
+def transform_smooth(x64: np.ndarray, inv_s: np.ndarray) -> np.ndarray:
+    """Per-channel scaling ``x diag(s)^-1`` (SmoothQuant, as in the handbook
+    page "Quantization: where diffusion differs from an LLM", section
+    "SmoothQuant"), with the caller's float32 reciprocal scale."""
+    inv = np.asarray(inv_s, dtype=np.float32).astype(np.float64)
+    return np.asarray(x64, dtype=np.float64) * inv[None, :]
+
+
+# --------------------------------------------------------------------------
+# bfloat16 input
+# --------------------------------------------------------------------------
+def bf16_bits_to_float64(bits: np.ndarray) -> np.ndarray:
+    """Exact value of bfloat16 bit patterns (the top half of a float32)."""
+    bits = np.asarray(bits, dtype=np.uint16)
+    f32 = (bits.astype(np.uint32) << 16).view(np.float32)
+    return f32.astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# Step 4: MXFP4 (E8M0 scale + E2M1 elements)
+# --------------------------------------------------------------------------
+def decision_values(y64: np.ndarray) -> np.ndarray:
+    """The transformed values as the quantizer sees them: rounded once to
+    float32 (round to nearest even), held exactly in float64."""
+    return np.asarray(y64, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def e8m0_exponent(amax):
+    """Shared exponent of a block: ``floor(log2(amax)) - emax(E2M1)``, clamped
+    to the E8M0 range; ``-127`` for an all-zero block.  Works elementwise."""
+    amax = np.asarray(amax, dtype=np.float64)
+    _, p = np.frexp(amax)            # amax = f * 2**p with 0.5 <= f < 1 (exact)
+    e = (p.astype(np.int64) - 1) - E2M1_EMAX
+    e = np.where(amax == 0.0, -E8M0_BIAS, e)
+    return np.clip(e, -E8M0_BIAS, E8M0_BIAS)
+
+
+def e2m1_encode(v: np.ndarray) -> np.ndarray:
+    """Nearest E2M1 code (4 bits: sign, 3-bit magnitude), ties to the even
+    magnitude code, saturating at 6.  ``v`` is already divided by the scale."""
+    v = np.asarray(v, dtype=np.float64)
+    m = np.abs(v)
+    code = np.zeros(v.shape, dtype=np.uint8)
+    for k in range(len(E2M1_GRID) - 1):
+        mid = 0.5 * (E2M1_GRID[k] + E2M1_GRID[k + 1])
+        # past the midpoint -> at least k+1; on it -> the even one of k, k+1
+        up = (m > mid) | ((m == mid) & (k % 2 == 1))
+        code += up.astype(np.uint8)
+    code |= (np.signbit(v).astype(np.uint8) << 3)
+    return code
+
+
+def e2m1_decode(code: np.ndarray) -> np.ndarray:
+    """Value of an E2M1 code from its bit fields: sign, 2-bit exponent (bias
+    1), 1-bit mantissa; exponent field 0 is subnormal (0 or 0.5)."""
+    code = np.asarray(code, dtype=np.uint8)
+    s = (code >> 3) & 1
+    e = (code >> 1) & 3
+    m = (code & 1).astype(np.float64)
+    mag = np.where(e == 0, 0.5 * m, np.ldexp(1.0 + 0.5 * m, e.astype(np.int64) - 1))
+    return np.where(s == 1, -mag, mag)
+
+
+def mxfp4_quantize(y64: np.ndarray):
+    """Quantize ``[M, d]`` values block by block.
+
+    Returns ``(codes [M, d] uint8 (unpacked), scale bytes [M, d/32] uint8)``.
+    """
+    yq = decision_values(y64)
+    M, d = yq.shape
+    nb = d // BLOCK
+    blocks = yq.reshape(M, nb, BLOCK)
+    amax = np.abs(blocks).max(axis=2)
+    e = e8m0_exponent(amax)
+    v = blocks * np.ldexp(1.0, -e)[:, :, None]        # exact: power-of-two scaling
+    codes = e2m1_encode(v).reshape(M, d)
+    return codes, (e + E8M0_BIAS).astype(np.uint8)
+
+
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    """Two codes per byte: element ``2i`` in the low nibble, ``2i+1`` high."""
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray) -> np.ndarray:
+    packed = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(packed.shape[:-1] + (packed.shape[-1] * 2,), dtype=np.uint8)
+    out[..., 0::2] = packed & 0xF
+    out[..., 1::2] = packed >> 4
+    return out
+
+
+def e8m0_decode(scale: np.ndarray) -> np.ndarray:
+    """``2**(s - 127)``; the byte 0xFF is NaN."""
+    s = np.asarray(scale, dtype=np.int64)
+    val = np.ldexp(1.0, s - E8M0_BIAS)
+    return np.where(s == 255, np.nan, val)
+
+
+def dequantize(q_packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """Exact float64 value of packed codes times their block scales."""
+    codes = unpack_codes(q_packed)
+    M, d = codes.shape
+    vals = e2m1_decode(codes).reshape(M, d // BLOCK, BLOCK)
+    return (vals * e8m0_decode(scales)[:, :, None]).reshape(M, d)
+
+
+# --------------------------------------------------------------------------
+# The entry points the library exposes, end to end
+# --------------------------------------------------------------------------
+def quantize(x_bits: np.ndarray, params: np.ndarray):
+    """KroQuant quantizer: bf16 bits ``[M, d]`` -> (packed codes, scales)."""
+    codes, scales = mxfp4_quantize(transform(bf16_bits_to_float64(x_bits), params))
+    return pack_codes(codes), scales
+
+
+def quantize_hadamard(x_bits: np.ndarray):
+    codes, scales = mxfp4_quantize(transform_hadamard(bf16_bits_to_float64(x_bits)))
+    return pack_codes(codes), scales
+
+
+def quantize_smooth(x_bits: np.ndarray, inv_s: np.ndarray):
+    codes, scales = mxfp4_quantize(transform_smooth(bf16_bits_to_float64(x_bits), inv_s))
+    return pack_codes(codes), scales
+
+
+# --------------------------------------------------------------------------
+# Magnitudes the tolerance rule is stated against
+# --------------------------------------------------------------------------
+def abs_transform(x64: np.ndarray, params: np.ndarray) -> np.ndarray:
+    """``|x| |T|`` elementwise (``|K| = |G1| (x) ... (x) |G5|``): the size of
+    the sum each transformed element is, used to state rounding tolerances."""
+    params = np.asarray(params)
+    return _apply_blocks(np.abs(x64), lambda j: np.abs(kron_block(params[j])))
+
+
+def abs_transform_hadamard(x64: np.ndarray) -> np.ndarray:
+    H = np.abs(hadamard_block())
+    return _apply_blocks(np.abs(x64), lambda j: H)
+
+
+def abs_inverse_transform(y64: np.ndarray, params: np.ndarray) -> np.ndarray:
+    params = np.asarray(params)
+    return _apply_blocks(np.abs(y64), lambda j: np.abs(inverse_block(params[j])))
+
+
+PARAMS_PER_BLOCK = 3 * N_FACTORS          # three scalars per 2x2 factor
