@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Throughput of the KroQuant online activation quantizer (kq_quantize) on B200.
+
+One step = one kq_quantize call over the whole bandwidth-stress activation
+(16384 x 12288 bf16, Student-t(3), 0.5% outlier channels x100): Kronecker
+block transform, E8M0 scale and E2M1 codes for every 32-element block.
+Reported as algorithmic GB/s (2 B read + 0.5 B + 1/32 B written per element)
+and as a fraction of the measured HBM bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With N > 1 it runs under torch.distributed.run, one rank per GPU; every rank
+quantizes its own 16384-row shard of one larger batch (weak scaling, no
+collective on the data path); the time is the maximum over ranks.
+``--impl reference`` times the float64 CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import multiprocessing as mp
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "kq_quantize GB/s (bf16 in→MXFP4 out) and % of B200 HBM peak"
+UNIT = "GB/s"
+WORKLOAD = "stress"
+FALLBACK_HBM_GBS = 6650.0
+CPU_SAMPLE_ROWS = 4096
+REFERENCE_BUDGET_S = 60.0
+
+
+# ------------------------------------------------------------------ helpers
+def dist_env():
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def shard_row0(rank: int, rows_per_rank: int) -> int:
+    """First row of this rank's shard in the global batch (weak scaling)."""
+    return rank * rows_per_rank
+
+
+def aggregate_gbs(bytes_per_rank_step: float, world: int, steps: int, max_ms: float) -> float:
+    """Whole-job GB/s: bytes every rank moved over the slowest rank's time."""
+    return bytes_per_rank_step * world * steps / (max_ms * 1e-3) / 1e9
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    src = os.path.join(ROOT, "w4a4_post_quantization_b200", "csrc")
+    for f in sorted(glob.glob(os.path.join(src, "*.cu")) + glob.glob(os.path.join(src, "*.cuh"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel_hash: str, name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", name)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    kv = {}
+    for line in text.splitlines():
+        if ":" in line and line.startswith("- "):
+            k, v = line[2:].split(":", 1)
+            kv[k.strip()] = v.strip().strip("`")
+    if kv.get("kernel_source_hash") != kernel_hash:
+        return None
+    try:
+        return float(kv["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, local_rank: int, period_s: float = 0.002):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ids = [v for v in vis.split(",") if v.strip()] if vis else []
+            ident = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+            if ident.startswith("GPU-") or ident.startswith("MIG-"):
+                self.h = pynvml.nvmlDeviceGetHandleByUUID(ident)
+            else:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(int(ident))
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:            # no NVML on this host
+            self.nvml, self.error = None, repr(e)
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(k)
+            except Exception as e:
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        return {
+            "sm_mhz": statistics.median(self.samples) if self.samples else None,
+            "sm_max_mhz": self.max_mhz,
+            "reasons": sorted(self.reasons),
+            "samples": len(self.samples),
+            "source": "nvml" if self.nvml is not None else f"unavailable: {self.error}",
+        }
+
+
+# -------------------------------------------------------- oracle (CPU) leg
+def _oracle_chunk(args):
+    """Runs in a spawned worker with one BLAS thread: oracle on a row chunk."""
+    bits, params = args
+    from oracle import kq_oracle as o
+    t0 = time.perf_counter()
+    o.quantize(bits, params)
+    return time.perf_counter() - t0
+
+
+def _cpu_workers() -> int:
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(32, n))
+
+
+def oracle_pool(workers: int):
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[var] = "1"
+    return mp.get_context("spawn").Pool(workers)
+
+
+def time_oracle(pool, case, rows: int, chunk: int = 128):
+    """Wall time of the oracle over the first ``rows`` rows, split in chunks
+    over the pool's workers."""
+    bits = case.x_bits()[:rows]
+    jobs = [(bits[r:r + chunk], case.params) for r in range(0, rows, chunk)]
+    t0 = time.perf_counter()
+    pool.map(_oracle_chunk, jobs)
+    return time.perf_counter() - t0
+
+
+def run_reference(args):
+    import workloads as w
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    workers = _cpu_workers()
+    pool = oracle_pool(workers)
+    M_full = w.CONFIGS[WORKLOAD]["M"]
+    probe = w.make_case(WORKLOAD, M=min(M_full, 64 * workers))
+    d = probe.d
+    # Oracle rate on this host, then rows per step so that all K + W steps
+    # take about REFERENCE_BUDGET_S.
+    sec = time_oracle(pool, probe, probe.M, chunk=64)
+    rate_rows = probe.M / sec
+    per_step = REFERENCE_BUDGET_S / (args.steps + args.warmup)
+    rows = int(max(workers, min(M_full, rate_rows * per_step)))
+    case = w.make_case(WORKLOAD, M=rows)
+    chunk = max(1, -(-rows // workers))
+    for _ in range(args.warmup):
+        time_oracle(pool, case, rows, chunk)
+    elapsed = [time_oracle(pool, case, rows, chunk) for _ in range(args.steps)]
+    pool.close()
+    total = sum(elapsed)
+    gbs = w.algorithmic_bytes(rows, d) * args.steps / total / 1e9
+    sample = (f"rows 0-{rows - 1} of the {M_full}x{d} stress input per step, "
+              f"float64 numpy oracle in {workers} spawned processes, 1 BLAS thread each")
+    line = {
+        "metric": METRIC, "value": gbs, "unit": UNIT, "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(_config(d, M_full, "oracle"), sample_rows_per_step=rows),
+        "cpu_baseline": {"value": gbs, "unit": UNIT, "cores": workers, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(d, M, impl):
+    return {
+        "workload": f"bandwidth stress: M={M} tokens x d={d} bf16, Student-t(3), "
+                    "0.5% outlier channels x100, learned Kronecker-LU block params",
+        "M": M, "d": d, "block": 32, "format": "MXFP4 (E2M1 codes + E8M0 scale per 32)",
+        "impl": impl,
+        "l2": "inputs larger than L2 (403 MB x vs 126 MB L2); no flush",
+    }
+
+
+# --------------------------------------------------------------- GPU leg
+def time_steps(fn, steps: int, warmup: int, stream, sampler=None):
+    """Average ms per step over exactly ``steps`` calls, CUDA events on
+    ``stream``, barrier + synchronize on both sides."""
+    import torch
+    import torch.distributed as dist
+    for _ in range(warmup):
+        fn()
+    sync = (lambda: dist.barrier()) if dist.is_initialized() else (lambda: None)
+    torch.cuda.synchronize()
+    sync()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if sampler is not None:
+        sampler.start()
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler is not None else None
+    sync()
+    return start.elapsed_time(end) / steps, clocks
+
+
+def run_gpu(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import w4a4_post_quantization_b200 as kq
+    import workloads as w
+
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+
+    # CPU baseline pool first (spawned, rank 0 at N=1 only).
+    pool = None
+    if world == 1 and not args.no_cpu_baseline:
+        pool = oracle_pool(_cpu_workers())
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    M = w.CONFIGS[WORKLOAD]["M"]
+    case = w.make_case(WORKLOAD, row0=shard_row0(rank, M))
+    d = case.d
+    x = case.x.to(dev)
+    params = torch.from_numpy(case.params).to(dev)
+    inv_s = torch.from_numpy(case.inv_s).to(dev)
+    q = torch.empty((M, d // 2), dtype=torch.uint8, device=dev)
+    s = torch.empty((M, d // 32), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    alg_bytes = w.algorithmic_bytes(M, d)
+
+    def step():
+        kq.quantize(x, params, q, s)
+
+    # Clock ramp: untimed launches for ~0.3 s so the timed region starts warm.
+    t_end = time.perf_counter() + 0.3
+    while time.perf_counter() < t_end:
+        step()
+        torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    ms, clocks = time_steps(step, args.steps, args.warmup, stream, sampler)
+    ms_max = max_over_ranks(ms, dev)
+    value = aggregate_gbs(alg_bytes, world, args.steps, ms_max * args.steps)
+
+    # Comparators and the copy ceiling on the same input (context, same GPU).
+    variants = {}
+    if not args.quick:
+        ms_h, _ = time_steps(lambda: kq.quantize_hadamard(x, q, s), args.steps, args.warmup, stream)
+        ms_s, _ = time_steps(lambda: kq.quantize_smooth(x, inv_s, q, s), args.steps, args.warmup,
+                             stream)
+        ms_max_h = max_over_ranks(ms_h, dev)
+        ms_max_s = max_over_ranks(ms_s, dev)
+        buf = torch.empty_like(x)
+        ms_c, _ = time_steps(lambda: buf.copy_(x), args.steps, args.warmup, stream)
+        ms_max_c = max_over_ranks(ms_c, dev)
+        variants = {
+            "hadamard": {"gbs": alg_bytes / (ms_max_h * 1e-3) / 1e9, "ms": ms_max_h},
+            "smooth": {"gbs": alg_bytes / (ms_max_s * 1e-3) / 1e9, "ms": ms_max_s},
+            "kronecker_over_smooth_speed": ms_max_s / ms_max,
+            "d2d_copy_gbs": 2 * x.numel() * 2 / (ms_max_c * 1e-3) / 1e9,
+        }
+        del buf
+
+    # End to end through the public API: pinned host in, pinned host out.
+    e2e = None
+    if not args.no_e2e:
+        x_host = case.x.pin_memory()
+        p_host = torch.from_numpy(case.params).pin_memory()
+        q_host = torch.empty((M, d // 2), dtype=torch.uint8).pin_memory()
+        s_host = torch.empty((M, d // 32), dtype=torch.uint8).pin_memory()
+        x_dev = torch.empty_like(x)
+        p_dev = torch.empty_like(params)
+
+        def e2e_step():
+            x_dev.copy_(x_host, non_blocking=True)
+            p_dev.copy_(p_host, non_blocking=True)
+            kq.quantize(x_dev, p_dev, q, s)
+            q_host.copy_(q, non_blocking=True)
+            s_host.copy_(s, non_blocking=True)
+
+        e2e_steps = min(args.steps, 20)
+        ms_e, _ = time_steps(e2e_step, e2e_steps, min(args.warmup, 3), stream)
+        ms_max_e = max_over_ranks(ms_e, dev)
+        h2d = x_host.numel() * 2 + p_host.numel() * 4
+        d2h = q_host.numel() + s_host.numel()
+        e2e = {"value": aggregate_gbs(alg_bytes, world, 1, ms_max_e), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+               "ms_per_step": ms_max_e}
+        assert torch.equal(q_host, q.cpu()) and torch.equal(s_host, s.cpu())
+
+    peak, peak_src = measured_peak()
+    per_launch_gbs = alg_bytes / (ms * 1e-3) / 1e9
+    khash = kernel_source_hash()
+    roof = {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
+            "frac": per_launch_gbs / peak, "peak_source": peak_src,
+            "traffic": profiled_traffic(khash, "kq_quantize_stress_traffic.md"),
+            "algorithmic_bytes_per_launch": alg_bytes, "kernel": "tma_kernel<kron, mx4>",
+            "kernel_source_hash": khash}
+
+    cpu = None
+    if pool is not None and rank == 0:
+        rows = CPU_SAMPLE_ROWS
+        sec = time_oracle(pool, case, rows)
+        pool.close()
+        cpu = {"value": w.algorithmic_bytes(rows, d) / sec / 1e9, "unit": UNIT,
+               "cores": _cpu_workers(), "kind": "oracle",
+               "sample": f"rows 0-{rows - 1} of the {M}x{d} stress input, float64 numpy "
+                         f"oracle in {_cpu_workers()} spawned processes, 1 BLAS thread each, "
+                         f"{sec:.2f} s wall"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": dict(_config(d, M, "tma"), global_batch_rows=M * world,
+                           parallelism=f"row shards x{world}", clock_ramp_s=0.3),
+            "hbm_frac": value / world / peak,
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+            "gpu_launches": args.steps, "variants": variants,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="skip the comparator timings")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

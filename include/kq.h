@@ -1,0 +1,127 @@
+/*
+ * kq.h -- C ABI of the B200 (sm_100a) KroQuant online activation quantizer.
+ *
+ * What it computes (KroQuant review on pith.science, "What carries the
+ * argument" and section 3.2 Eq. 4 / Eq. 6; abstract): every 32-channel block j
+ * of a bf16 activation row x is multiplied on the right by a learned
+ * invertible 32x32 block
+ *
+ *     K^(j) = G1 (x) G2 (x) G3 (x) G4 (x) G5,
+ *     G_k   = [[1, 0], [a_k, 1]] . [[b_k, c_k], [0, 1/b_k]]   (det G_k = 1),
+ *
+ * (y = x T with T = diag(K^(1), ..., K^(d/32)); Eq. 1 of the paper folds T^-1
+ * into the weights offline), and the transformed block is quantized to MXFP4:
+ * one E8M0 scale byte per 32 elements and one E2M1 code per element, two codes
+ * per byte.  G1 acts on the most significant bit of the 5-bit in-block index.
+ *
+ * Quantization rule (OCP Microscaling MXFP4, which the paper's "MXFP4e2"
+ * names):  e = clamp(floor(log2(max_c |y_c|)) - 2, -127, 127)  (e = -127 for
+ * an all-zero block), scale byte = e + 127, code = nearest E2M1 value of
+ * y_c / 2^e in {0, .5, 1, 1.5, 2, 3, 4, 6} with ties to the even code,
+ * saturating at 6, sign bit 0x8 set for negative values (also when they round
+ * to zero).  Element 2i goes to the low nibble of byte i, element 2i+1 to the
+ * high nibble.  The transform runs in float32; the decision is taken on the
+ * float32 value.
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers that the caller allocates and
+ *     owns; nothing is allocated, freed or retained by the library.
+ *   - Arrays are dense and row-major: x and y are [M][d], q_packed is
+ *     [M][d/2] bytes, scales is [M][d/32] bytes, params is [d/32][5][3]
+ *     float32 holding (a, b, c) for factors k = 1..5, inv_s is [d] float32.
+ *   - d must be a positive multiple of 32.  M == 0 is a no-op returning
+ *     KQ_OK; M < 0 is KQ_ERR_INVALID.  M * d must not exceed 2^40.
+ *   - x, q_packed, y (float32 in or out) must be 16-byte aligned; params and
+ *     inv_s 4-byte aligned; scales has no alignment requirement.
+ *   - stream is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *     asynchronous: they enqueue kernels and return without synchronising.
+ *   - Results for non-finite inputs or parameters (b_k == 0, NaN, Inf, or a
+ *     transform that overflows float32) are unspecified.
+ *   - Return value: KQ_OK, KQ_ERR_INVALID (argument check failed, nothing
+ *     enqueued), KQ_ERR_CUDA (a CUDA call or launch failed; see
+ *     kq_last_cuda_error) or KQ_ERR_DEVICE (current device is not sm_100).
+ */
+#ifndef KQ_H_
+#define KQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    KQ_OK = 0,
+    KQ_ERR_INVALID = 1,
+    KQ_ERR_CUDA = 2,
+    KQ_ERR_DEVICE = 3,
+    KQ_ERR_TIMEOUT = 4
+};
+
+/* Implementation selector for kq_quantize_ex (for measurements). */
+enum {
+    KQ_IMPL_AUTO = 0,       /* what kq_quantize uses */
+    KQ_IMPL_TMA = 1,        /* TMA-staged, persistent, thread per 32-block */
+    KQ_IMPL_DIRECT = 2,     /* direct 32-byte global loads, thread per 32-block */
+    KQ_IMPL_WARP = 3        /* one 32-block per warp, shuffle butterfly */
+};
+
+/* KroQuant quantizer, the hot path: q_packed/scales = MXFP4(x T).
+ * KroQuant review, "What carries the argument"; section 3.2 Eq. 4 and 6. */
+int kq_quantize(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                uint8_t* q_packed, uint8_t* scales, void* stream);
+
+/* Same computation with an explicit implementation choice (KQ_IMPL_*).
+ * KQ_ERR_INVALID if the implementation cannot take this shape. */
+int kq_quantize_ex(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                   uint8_t* q_packed, uint8_t* scales, int impl, void* stream);
+
+/* Comparator: fixed orthonormal block Hadamard H_32/sqrt(32) (Sylvester
+ * order) in place of K^(j), then the same MXFP4 quantizer.  KroQuant review,
+ * "Core claim" (the Hadamard initialisation) and abstract. */
+int kq_quantize_hadamard(const uint16_t* x, int64_t M, int64_t d,
+                         uint8_t* q_packed, uint8_t* scales, void* stream);
+
+/* Comparator: per-channel scaling y[c] = x[c] * inv_s[c] (SmoothQuant's
+ * X diag(s)^-1 with the caller's float32 reciprocal scale), then the same
+ * MXFP4 quantizer.  Handbook page "Quantization: where diffusion differs from
+ * an LLM", section "SmoothQuant"; KroQuant abstract. */
+int kq_quantize_smooth(const uint16_t* x, int64_t M, int64_t d, const float* inv_s,
+                       uint8_t* q_packed, uint8_t* scales, void* stream);
+
+/* y = x T in float32 (the kq_quantize transform without quantization), for
+ * parity checks. */
+int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                 float* y, void* stream);
+
+/* x = y T^-1 in float32 with T^-1 = diag(G1^-1 (x) ... (x) G5^-1) (review,
+ * axiom ledger: the inverse of a Kronecker product factorizes). */
+int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,
+                         float* x, void* stream);
+
+/* y = E2M1(code) * 2^(scale - 127) in float32 (exact; scale byte 0xFF gives
+ * NaN, results beyond the float32 range give +-Inf). */
+int kq_dequantize(const uint8_t* q_packed, const uint8_t* scales, int64_t M, int64_t d,
+                  float* y, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* kq_status_string(int status);
+
+/* The cudaError_t of the last KQ_ERR_CUDA on this thread (0 if none). */
+int kq_last_cuda_error(void);
+
+/* Synchronises the current device, then reads and clears the library's
+ * device-side error word: 0 if every bounded in-kernel wait finished,
+ * otherwise a bit mask of the waits that gave up (kernels that give up stop
+ * early and leave their outputs incomplete).  Returns KQ_OK or KQ_ERR_CUDA. */
+int kq_device_status(int* flags);
+
+/* ABI version, (major << 16) | minor. */
+int kq_version(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* KQ_H_ */

@@ -1,0 +1,90 @@
+"""The C-ABI library loads without a GPU, exports every entry point the
+header declares, and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kq.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from w4a4_post_quantization_b200 import build
+    build.build()
+    from w4a4_post_quantization_b200 import _lib
+    return _lib.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_covers_the_header():
+    from w4a4_post_quantization_b200 import _lib
+    assert sorted(_lib.SIGNATURES) == _declared()
+
+
+def test_status_strings_and_version(lib):
+    assert lib.kq_status_string(0) == b"ok"
+    assert lib.kq_status_string(1) == b"invalid argument"
+    assert lib.kq_status_string(123) == b"unknown status"
+    assert lib.kq_version() >> 16 == 1
+
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: checks fail first
+
+
+@pytest.mark.parametrize("M,d", [(-1, 64), (4, 0), (4, 48), (4, 16), (1 << 30, 1 << 20)])
+def test_bad_shapes(lib, M, d):
+    assert lib.kq_quantize(FAKE, M, d, FAKE, FAKE, FAKE, None) == 1
+    assert lib.kq_quantize_hadamard(FAKE, M, d, FAKE, FAKE, None) == 1
+    assert lib.kq_quantize_smooth(FAKE, M, d, FAKE, FAKE, FAKE, None) == 1
+    assert lib.kq_transform(FAKE, M, d, FAKE, FAKE, None) == 1
+    assert lib.kq_inverse_transform(FAKE, M, d, FAKE, FAKE, None) == 1
+    assert lib.kq_dequantize(FAKE, FAKE, M, d, FAKE, None) == 1
+
+
+def test_null_and_misaligned_pointers(lib):
+    assert lib.kq_quantize(None, 4, 64, FAKE, FAKE, FAKE, None) == 1
+    assert lib.kq_quantize(FAKE, 4, 64, None, FAKE, FAKE, None) == 1
+    assert lib.kq_quantize(FAKE, 4, 64, FAKE, None, FAKE, None) == 1
+    assert lib.kq_quantize(FAKE, 4, 64, FAKE, FAKE, None, None) == 1
+    assert lib.kq_quantize(FAKE + 8, 4, 64, FAKE, FAKE, FAKE, None) == 1      # x not 16-B aligned
+    assert lib.kq_quantize(FAKE, 4, 64, FAKE + 2, FAKE, FAKE, None) == 1      # params not 4-B
+    assert lib.kq_quantize(FAKE, 4, 64, FAKE, FAKE + 4, FAKE, None) == 1      # q not 16-B
+    assert lib.kq_quantize_smooth(FAKE, 4, 64, FAKE + 4, FAKE, FAKE, None) == 1
+    assert lib.kq_quantize_ex(FAKE, 4, 64, FAKE, FAKE, FAKE, 7, None) == 1
+    assert lib.kq_dequantize(FAKE, FAKE, 4, 64, FAKE + 4, None) == 1
+    assert lib.kq_device_status(None) == 1
+
+
+def test_empty_input_needs_no_device(lib):
+    assert lib.kq_quantize(None, 0, 64, None, None, None, None) == 0
+    assert lib.kq_dequantize(None, None, 0, 64, None, None) == 0
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    import w4a4_post_quantization_b200 as kq
+    x = torch.zeros((2, 64), dtype=torch.bfloat16)
+    p = torch.zeros((2, 5, 3), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        kq.quantize(x, p)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    from w4a4_post_quantization_b200 import _lib
+    with pytest.raises(ImportError):
+        _lib.load_library(str(tmp_path / "libkq.so"))

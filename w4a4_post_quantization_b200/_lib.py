@@ -1,0 +1,205 @@
+"""ctypes binding of ``libkq.so`` (the C ABI declared in ``include/kq.h``).
+
+Argument marshalling only: tensors are checked for device, dtype, shape and
+contiguity, their device pointers and the current CUDA stream are passed to
+the library, and a non-zero status raises.  Every step of the computation runs
+in the library's kernels; there is no CPU fallback, and a missing library
+raises ImportError.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkq.so")
+
+KQ_OK, KQ_ERR_INVALID, KQ_ERR_CUDA, KQ_ERR_DEVICE, KQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
+KQ_IMPL_AUTO, KQ_IMPL_TMA, KQ_IMPL_DIRECT, KQ_IMPL_WARP = 0, 1, 2, 3
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+
+# name -> (argtypes); every entry point returns int unless listed in _RESTYPE.
+SIGNATURES = {
+    "kq_quantize": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_quantize_ex": [_p, _i64, _i64, _p, _p, _p, _int, _p],
+    "kq_quantize_hadamard": [_p, _i64, _i64, _p, _p, _p],
+    "kq_quantize_smooth": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_transform": [_p, _i64, _i64, _p, _p, _p],
+    "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
+    "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
+    "kq_status_string": [_int],
+    "kq_last_cuda_error": [],
+    "kq_device_status": [ctypes.POINTER(_int)],
+    "kq_version": [],
+}
+_RESTYPE = {"kq_status_string": ctypes.c_char_p}
+
+
+class KQError(RuntimeError):
+    def __init__(self, fn: str, status: int, lib):
+        msg = lib.kq_status_string(status).decode()
+        if status == KQ_ERR_CUDA:
+            msg += f" (cudaError {lib.kq_last_cuda_error()})"
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+def load_library(path: str = LIB_PATH):
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it first (python -c 'import __graft_entry__ as g; g.build()')")
+    lib = ctypes.CDLL(path)
+    for name, args in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = _RESTYPE.get(name, ctypes.c_int)
+    return lib
+
+
+_LIB = None
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        _LIB = load_library()
+    return _LIB
+
+
+def _check(name: str, status: int) -> None:
+    if status != KQ_OK:
+        raise KQError(name, status, lib())
+
+
+def _stream(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _dev_tensor(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _shape(x: torch.Tensor):
+    if x.dim() != 2:
+        raise ValueError("x must be 2-D [M, d]")
+    M, d = x.shape
+    if d % 32 != 0 or d == 0:
+        raise ValueError("d must be a positive multiple of 32")
+    return M, d
+
+
+def _out_codes(x, q, scales):
+    M, d = _shape(x)
+    if q is None:
+        q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((M, d // 32), dtype=torch.uint8, device=x.device)
+    _dev_tensor(q, torch.uint8, "q")
+    _dev_tensor(scales, torch.uint8, "scales")
+    if tuple(q.shape) != (M, d // 2) or tuple(scales.shape) != (M, d // 32):
+        raise ValueError("output shapes must be [M, d/2] and [M, d/32]")
+    return M, d, q, scales
+
+
+def _params(params: torch.Tensor, d: int) -> torch.Tensor:
+    _dev_tensor(params, torch.float32, "params")
+    if params.numel() != (d // 32) * 15:
+        raise ValueError("params must hold [d/32, 5, 3] float32 values")
+    return params
+
+
+def quantize(x: torch.Tensor, params: torch.Tensor, q=None, scales=None, impl: int = KQ_IMPL_AUTO):
+    """MXFP4(x T): returns (packed codes uint8 [M, d/2], scale bytes uint8 [M, d/32])."""
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d, q, scales = _out_codes(x, q, scales)
+    _params(params, d)
+    if impl == KQ_IMPL_AUTO:
+        st = lib().kq_quantize(x.data_ptr(), M, d, params.data_ptr(), q.data_ptr(),
+                               scales.data_ptr(), _stream(x.device))
+    else:
+        st = lib().kq_quantize_ex(x.data_ptr(), M, d, params.data_ptr(), q.data_ptr(),
+                                  scales.data_ptr(), impl, _stream(x.device))
+    _check("kq_quantize", st)
+    return q, scales
+
+
+def quantize_hadamard(x: torch.Tensor, q=None, scales=None):
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d, q, scales = _out_codes(x, q, scales)
+    st = lib().kq_quantize_hadamard(x.data_ptr(), M, d, q.data_ptr(), scales.data_ptr(),
+                                    _stream(x.device))
+    _check("kq_quantize_hadamard", st)
+    return q, scales
+
+
+def quantize_smooth(x: torch.Tensor, inv_s: torch.Tensor, q=None, scales=None):
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d, q, scales = _out_codes(x, q, scales)
+    _dev_tensor(inv_s, torch.float32, "inv_s")
+    if inv_s.numel() != d:
+        raise ValueError("inv_s must hold d float32 values")
+    st = lib().kq_quantize_smooth(x.data_ptr(), M, d, inv_s.data_ptr(), q.data_ptr(),
+                                  scales.data_ptr(), _stream(x.device))
+    _check("kq_quantize_smooth", st)
+    return q, scales
+
+
+def transform(x: torch.Tensor, params: torch.Tensor, y=None):
+    """y = x T in float32."""
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    _params(params, d)
+    if y is None:
+        y = torch.empty((M, d), dtype=torch.float32, device=x.device)
+    _dev_tensor(y, torch.float32, "y")
+    st = lib().kq_transform(x.data_ptr(), M, d, params.data_ptr(), y.data_ptr(), _stream(x.device))
+    _check("kq_transform", st)
+    return y
+
+
+def inverse_transform(y: torch.Tensor, params: torch.Tensor, x=None):
+    """x = y T^-1 in float32."""
+    _dev_tensor(y, torch.float32, "y")
+    M, d = _shape(y)
+    _params(params, d)
+    if x is None:
+        x = torch.empty((M, d), dtype=torch.float32, device=y.device)
+    _dev_tensor(x, torch.float32, "x")
+    st = lib().kq_inverse_transform(y.data_ptr(), M, d, params.data_ptr(), x.data_ptr(),
+                                    _stream(y.device))
+    _check("kq_inverse_transform", st)
+    return x
+
+
+def dequantize(q: torch.Tensor, scales: torch.Tensor, y=None):
+    """float32 [M, d] = E2M1(code) * 2^(scale - 127)."""
+    _dev_tensor(q, torch.uint8, "q")
+    _dev_tensor(scales, torch.uint8, "scales")
+    M, half = q.shape
+    d = 2 * half
+    if tuple(scales.shape) != (M, d // 32):
+        raise ValueError("scales must be [M, d/32]")
+    if y is None:
+        y = torch.empty((M, d), dtype=torch.float32, device=q.device)
+    _dev_tensor(y, torch.float32, "y")
+    st = lib().kq_dequantize(q.data_ptr(), scales.data_ptr(), M, d, y.data_ptr(), _stream(q.device))
+    _check("kq_dequantize", st)
+    return y
+
+
+def device_status() -> int:
+    """Synchronise and return (and clear) the device-side wait-timeout flags."""
+    flags = _int(0)
+    _check("kq_device_status", lib().kq_device_status(ctypes.byref(flags)))
+    return flags.value

@@ -1,0 +1,288 @@
+// Device-side building blocks of the quantizer kernels (sm_100a only):
+// PTX wrappers for mbarriers, TMA, packed float32x2 arithmetic and the E2M1
+// conversion, the three block transforms and the shared MXFP4 epilogue.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library targets sm_100a (B200) only"
+#endif
+
+namespace kq {
+
+constexpr int kBlock = 32;           // elements per MX block and per Kronecker block
+constexpr int kFactors = 5;          // 32 = 2^5: one 2x2 factor per index bit
+constexpr int kTabStride = 44;       // floats per block in a Kronecker coefficient table
+
+// Bits of the device error word (kq_device_status).
+constexpr int kErrConsumerWait = 1;
+constexpr int kErrProducerWait = 2;
+
+// A bounded mbarrier wait polls at most kWaitPolls times, each poll suspending
+// for at most kWaitHintNs: about four seconds in all, far above any real wait.
+constexpr int kWaitPolls = 4000;
+constexpr uint32_t kWaitHintNs = 1000000;
+
+// --------------------------------------------------------------- addresses
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(
+                   smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// Waits for the phase of the given parity to complete; gives up (returns
+// false) after kWaitPolls suspended polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_addr(bar);
+  for (int poll = 0; poll < kWaitPolls; ++poll) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(addr), "r"(parity), "r"(kWaitHintNs)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+// ------------------------------------------------------------------- TMA
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 2-D tiled bulk tensor load into this CTA's shared memory (no multicast).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// ----------------------------------------------------- packed float32 x 2
+// A pair of floats in one 64-bit register pair; the first float is the low
+// half.  Blackwell executes add/mul/fma on both halves with one instruction.
+typedef unsigned long long f2;
+
+__device__ __forceinline__ f2 pack2(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 fma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 add2(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 sub2(f2 a, f2 b) {
+  f2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// Two bf16 values (element 2m in the low half-word) widened exactly to f32.
+__device__ __forceinline__ f2 bf16x2_to_f2(uint32_t w) {
+  return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// ----------------------------------------------------------- E2M1 convert
+// Eight floats (already divided by the block scale) to eight E2M1 codes,
+// element 0 in the low nibble of the low byte.  Round to nearest even,
+// saturating to +-6.
+__device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v3, float v4,
+                                           float v5, float v6, float v7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+  return r;
+}
+
+// ------------------------------------------------------ block transforms
+// A 32-element block lives in u[16]; u[m] holds elements 2m (low) and 2m+1.
+//
+// One butterfly stage applies a 2x2 factor G to every index pair that differs
+// only in bit p, as a row vector times G:
+//     y_lo = x_lo G00 + x_hi G10,   y_hi = x_lo G01 + x_hi G11.
+// For p >= 1 the two members of a pair sit in different registers and two
+// neighbouring pairs share a packed register, so one packed instruction does
+// two pairs; for p = 0 the pair shares one register and runs scalar.
+
+// Coefficients of stage s (bit 4 - s) in a table entry, as float4s:
+//   e[2s]   = (G00, G00, G10, G10)
+//   e[2s+1] = (G01, G01, G11, G11)
+template <int kHalfDist>
+__device__ __forceinline__ void stage_packed(f2 (&u)[16], float4 c0, float4 c1) {
+  const f2 g00 = pack2(c0.x, c0.y), g10 = pack2(c0.z, c0.w);
+  const f2 g01 = pack2(c1.x, c1.y), g11 = pack2(c1.z, c1.w);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    if (m & kHalfDist) continue;
+    const f2 lo = u[m], hi = u[m + kHalfDist];
+    u[m] = fma2(g10, hi, mul2(g00, lo));
+    u[m + kHalfDist] = fma2(g11, hi, mul2(g01, lo));
+  }
+}
+
+__device__ __forceinline__ void stage_bit0(f2 (&u)[16], float4 c0, float4 c1) {
+  const float g00 = c0.x, g10 = c0.z, g01 = c1.x, g11 = c1.z;
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    float lo, hi;
+    unpack2(u[m], lo, hi);
+    const float ylo = __fmaf_rn(g10, hi, __fmul_rn(g00, lo));
+    const float yhi = __fmaf_rn(g11, hi, __fmul_rn(g01, lo));
+    u[m] = pack2(ylo, yhi);
+  }
+}
+
+// y = x K with K = G1 (x) ... (x) G5, from a table entry of kTabStride floats.
+__device__ __forceinline__ void kron_apply(f2 (&u)[16], const float* entry) {
+  const float4* e = reinterpret_cast<const float4*>(entry);
+  stage_packed<8>(u, e[0], e[1]);   // G1, index bit 4
+  stage_packed<4>(u, e[2], e[3]);   // G2, bit 3
+  stage_packed<2>(u, e[4], e[5]);   // G3, bit 2
+  stage_packed<1>(u, e[6], e[7]);   // G4, bit 1
+  stage_bit0(u, e[8], e[9]);        // G5, bit 0
+}
+
+// Fills one table entry from the (a, b, c) parameters of a block; the four
+// entries of each G_k (or of G_k^-1 = [[G11, -G01], [-G10, G00]], det 1) are
+// formed in double and rounded once to float.
+__device__ __forceinline__ void kron_entry(float* entry, const float* p, bool inverse) {
+#pragma unroll
+  for (int k = 0; k < kFactors; ++k) {
+    const double a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
+    double g00 = b, g01 = c, g10 = a * b, g11 = __fma_rn(a, c, 1.0 / b);
+    if (inverse) {
+      const double t00 = g11, t01 = -g01, t10 = -g10, t11 = g00;
+      g00 = t00; g01 = t01; g10 = t10; g11 = t11;
+    }
+    const float f00 = (float)g00, f01 = (float)g01, f10 = (float)g10, f11 = (float)g11;
+    float4* e = reinterpret_cast<float4*>(entry + 8 * k);
+    e[0] = make_float4(f00, f00, f10, f10);
+    e[1] = make_float4(f01, f01, f11, f11);
+  }
+}
+
+// Fixed block Hadamard H_32 (Sylvester order: H2 = [[1,1],[1,-1]] on every
+// bit), then the orthonormal factor 1/sqrt(32) as one float32 multiply.
+__device__ __forceinline__ void hadamard_apply(f2 (&u)[16]) {
+#pragma unroll
+  for (int hd = 8; hd >= 1; hd >>= 1) {
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      if (m & hd) continue;
+      const f2 lo = u[m], hi = u[m + hd];
+      u[m] = add2(lo, hi);
+      u[m + hd] = sub2(lo, hi);
+    }
+  }
+  const float s = 0.17677669529663688f;   // 1/sqrt(32) rounded to float32
+  const f2 s2 = pack2(s, s);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    float lo, hi;
+    unpack2(u[m], lo, hi);
+    u[m] = mul2(pack2(lo + hi, lo - hi), s2);
+  }
+}
+
+// Per-channel scaling y[c] = x[c] * inv_s[c]; ``inv`` points at the block's
+// 32 reciprocal scales (16-byte aligned).
+__device__ __forceinline__ void smooth_apply(f2 (&u)[16], const float* inv) {
+  const float4* v = reinterpret_cast<const float4*>(inv);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 s = v[i];
+    u[2 * i] = mul2(u[2 * i], pack2(s.x, s.y));
+    u[2 * i + 1] = mul2(u[2 * i + 1], pack2(s.z, s.w));
+  }
+}
+
+// ------------------------------------------------------------ MXFP4 epilogue
+// Shared E8M0 scale of the block and the 16 bytes of packed codes.
+struct Mx4Block {
+  uint4 codes;
+  uint32_t scale;
+};
+
+__device__ __forceinline__ Mx4Block mxfp4_block(const f2 (&u)[16]) {
+  float m[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float lo, hi;
+    unpack2(u[i], lo, hi);
+    m[i] = fmaxf(fabsf(lo), fabsf(hi));
+  }
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  // floor(log2(amax)) is the biased exponent field minus 127, so the scale
+  // byte e + 127 = field - 2, clamped at 0 (zero and subnormal maxima too).
+  const int field = static_cast<int>(__float_as_uint(m[0]) >> 23);
+  const int sbyte = field > 2 ? field - 2 : 0;
+  // 2^-e as a normal float32: biased exponent 127 - e = 254 - sbyte.
+  const float inv_x = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);
+  const f2 s2 = pack2(inv_x, inv_x);
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) unpack2(mul2(u[4 * k + i], s2), v[2 * i], v[2 * i + 1]);
+    w[k] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+  }
+  Mx4Block r;
+  r.codes = make_uint4(w[0], w[1], w[2], w[3]);
+  r.scale = static_cast<uint32_t>(sbyte);
+  return r;
+}
+
+}  // namespace kq

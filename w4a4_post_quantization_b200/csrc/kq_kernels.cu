@@ -1,0 +1,532 @@
+// Kernels of the KroQuant quantizer library and their launchers.
+//
+// Hot path (kq_quantize): one thread owns one 32-element block.  x is staged
+// into shared memory by TMA tile loads (64-byte swizzle, so that the
+// thread-per-block reads are bank-conflict free) through a ring of stages
+// guarded by mbarriers; a producer warp issues the loads and eight consumer
+// warps run the butterfly, the block maximum, the E8M0 scale and the E2M1
+// conversion, and store 16 bytes of codes and one scale byte per block.
+// CTAs are persistent (one per SM) and walk the flat list of blocks
+// (row-major, so block g is row g / nb, column block g % nb).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "kq.h"
+#include "kq_device.cuh"
+
+namespace kq {
+
+__device__ int g_device_error = 0;
+
+enum Xform { kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2 };
+enum Out { kOutMx4 = 0, kOutF32 = 1 };
+
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumers = 32 * kConsumerWarps;       // threads = blocks per tile
+constexpr int kTmaThreads = kConsumers + 32;          // + one producer warp
+constexpr int kTile = kConsumers;                     // 32-blocks per TMA tile
+constexpr int kTileBytes = kTile * kBlock * 2;        // bf16 tile, 16 KiB
+constexpr int kMaxStages = 8;
+constexpr int kTmaMaxNb = 512;                        // blocks per row the TMA kernel tables
+constexpr int kDirectThreads = 256;                   // = column blocks per direct-kernel panel
+
+struct LaunchArgs {
+  int64_t G;            // 32-blocks in this launch (rows * nb)
+  int32_t nb;           // 32-blocks per row
+  int32_t n_tiles;      // ceil(G / kTile)
+  int32_t stages;       // TMA ring depth
+  int32_t inverse;      // table from G_k^-1 instead of G_k
+  const float* aux;     // params [nb][5][3] (Kronecker) or inv_s [nb*32] (smooth)
+  uint8_t* q;           // [G][16] packed codes
+  uint8_t* scales;      // [G] scale bytes
+  float* y;             // [G][32] float32 output (kOutF32)
+};
+
+// ------------------------------------------------------------ table build
+// Per-CTA shared table: for the Kronecker transform kTabStride floats per
+// column block (the G_k entries), for smooth the 32 reciprocal scales.
+template <int kXf>
+__device__ __forceinline__ void build_table(float* tab, const LaunchArgs& a, int j0, int jn,
+                                            int t, int nt) {
+  if (kXf == kXfKron) {
+    for (int j = t; j < jn; j += nt) kron_entry(tab + j * kTabStride, a.aux + (j0 + j) * 15, a.inverse);
+  } else if (kXf == kXfSmooth) {
+    const float4* src = reinterpret_cast<const float4*>(a.aux + (int64_t)j0 * kBlock);
+    float4* dst = reinterpret_cast<float4*>(tab);
+    for (int i = t; i < jn * (kBlock / 4); i += nt) dst[i] = src[i];
+  }
+}
+
+template <int kXf>
+__device__ __forceinline__ void apply_xform(f2 (&u)[16], const float* tab, int j) {
+  if (kXf == kXfKron) kron_apply(u, tab + j * kTabStride);
+  else if (kXf == kXfHadamard) hadamard_apply(u);
+  else smooth_apply(u, tab + j * kBlock);
+}
+
+template <int kOut>
+__device__ __forceinline__ void store_block(const f2 (&u)[16], const LaunchArgs& a, int64_t g) {
+  if (kOut == kOutMx4) {
+    const Mx4Block r = mxfp4_block(u);
+    __stcs(reinterpret_cast<uint4*>(a.q + g * 16), r.codes);
+    a.scales[g] = static_cast<uint8_t>(r.scale);
+  } else {
+    float4* dst = reinterpret_cast<float4*>(a.y + g * kBlock);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float x0, x1, x2, x3;
+      unpack2(u[2 * i], x0, x1);
+      unpack2(u[2 * i + 1], x2, x3);
+      __stcs(dst + i, make_float4(x0, x1, x2, x3));
+    }
+  }
+}
+
+__host__ __device__ constexpr int table_floats(int xf, int nb) {
+  return xf == kXfKron ? nb * kTabStride : (xf == kXfSmooth ? nb * kBlock : 0);
+}
+
+// ------------------------------------------------------------ TMA kernel
+template <int kXf, int kOut>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    tma_kernel(const __grid_constant__ CUtensorMap xmap, const LaunchArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  // Stage buffers first, 1 KiB aligned: the 64-byte swizzle pattern repeats
+  // every 512 bytes and is a function of the shared-memory address.
+  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = base;
+  float* tab = reinterpret_cast<float*>(base + a.stages * kTileBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(tab + table_floats(kXf, a.nb));
+  uint64_t* empty = full + a.stages;
+
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    for (int s = 0; s < a.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumers);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int S = a.stages;
+  const int n_local =
+      blockIdx.x < a.n_tiles ? (a.n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+
+  if (tid >= kConsumers) {
+    // Producer warp: one lane streams the CTA's tiles through the ring.
+    if (tid == kConsumers) {
+      tma_prefetch_map(&xmap);
+      int issued = 0;
+      bool ok = true;
+      for (int i = 0; i < n_local; ++i) {
+        const int s = i % S;
+        if (i >= S && !mbar_wait(&empty[s], ((i / S) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], kTileBytes);
+        tma_load_2d(stages + s * kTileBytes, &xmap, 0, (blockIdx.x + i * gridDim.x) * kTile,
+                    &full[s]);
+        issued = i + 1;
+      }
+      if (!ok) {
+        atomicOr(&g_device_error, kErrProducerWait);
+        // Let the copies still in flight land before the CTA exits.
+        for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+          mbar_wait(&full[i % S], (i / S) & 1);
+      }
+    }
+    return;
+  }
+
+  // Consumers: build the coefficient table, then one 32-block per tile each.
+  build_table<kXf>(tab, a, 0, a.nb, tid, kConsumers);
+  asm volatile("bar.sync 1, %0;" ::"r"(kConsumers) : "memory");
+
+  const int64_t step = (int64_t)gridDim.x * kTile;
+  int64_t g = (int64_t)blockIdx.x * kTile + tid;
+  int j = static_cast<int>(g % a.nb);
+  const int jstep = static_cast<int>(step % a.nb);
+  // Row tid of a tile holds its 4 chunks of 16 bytes at chunk ^ ((tid >> 1) & 3).
+  const uint32_t swz = (tid >> 1) & 3;
+  for (int i = 0; i < n_local; ++i) {
+    const int s = i % S;
+    if (!mbar_wait(&full[s], (i / S) & 1)) {
+      atomicOr(&g_device_error, kErrConsumerWait);
+      break;
+    }
+    const uint8_t* row = stages + s * kTileBytes + tid * (kBlock * 2);
+    uint4 c[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) c[q] = *reinterpret_cast<const uint4*>(row + 16 * (q ^ swz));
+    mbar_arrive(&empty[s]);
+    if (g < a.G) {
+      f2 u[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        u[4 * q + 0] = bf16x2_to_f2(c[q].x);
+        u[4 * q + 1] = bf16x2_to_f2(c[q].y);
+        u[4 * q + 2] = bf16x2_to_f2(c[q].z);
+        u[4 * q + 3] = bf16x2_to_f2(c[q].w);
+      }
+      apply_xform<kXf>(u, tab, j);
+      store_block<kOut>(u, a, g);
+    }
+    g += step;
+    j += jstep;
+    if (j >= a.nb) j -= a.nb;
+  }
+}
+
+// ---------------------------------------------------------- direct kernel
+// Grid (row groups, column panels of kDirectThreads blocks); thread t of
+// panel p handles column block 256 p + t of rows blockIdx.x, +gridDim.x, ...
+// Input is bf16 (four 16-byte loads per block) or float32 (eight).
+template <int kXf, int kOut, bool kF32In>
+__global__ void __launch_bounds__(kDirectThreads)
+    direct_kernel(const void* __restrict__ xin, int64_t M, const LaunchArgs a) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  float* tab = reinterpret_cast<float*>(smem_raw);
+  const int j0 = blockIdx.y * kDirectThreads;
+  const int jn = min(kDirectThreads, a.nb - j0);
+  build_table<kXf>(tab, a, j0, jn, threadIdx.x, blockDim.x);
+  __syncthreads();
+  const int t = threadIdx.x;
+  if (t >= jn) return;
+  for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
+    const int64_t g = r * a.nb + j0 + t;
+    f2 u[16];
+    if (!kF32In) {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(xin) + g * kBlock);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 c = __ldg(src + q);
+        u[4 * q + 0] = bf16x2_to_f2(c.x);
+        u[4 * q + 1] = bf16x2_to_f2(c.y);
+        u[4 * q + 2] = bf16x2_to_f2(c.z);
+        u[4 * q + 3] = bf16x2_to_f2(c.w);
+      }
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(xin) + g * kBlock);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 v = __ldcs(src + i);
+        u[2 * i] = pack2(v.x, v.y);
+        u[2 * i + 1] = pack2(v.z, v.w);
+      }
+    }
+    apply_xform<kXf>(u, tab, t);
+    store_block<kOut>(u, a, g);
+  }
+}
+
+// ------------------------------------------------------- dequantize kernel
+__global__ void __launch_bounds__(256)
+    dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, int64_t G,
+                   float* __restrict__ y) {
+  __shared__ float lut[16];
+  if (threadIdx.x < 16) {
+    const int c = threadIdx.x, e = (c >> 1) & 3, m = c & 1;
+    const float mag = e == 0 ? 0.5f * m : ldexpf(1.0f + 0.5f * m, e - 1);
+    lut[c] = (c & 8) ? -mag : mag;
+  }
+  __syncthreads();
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < G;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 c = __ldcs(reinterpret_cast<const uint4*>(q + g * 16));
+    const uint32_t s = scales[g];
+    const float x = s == 255 ? __uint_as_float(0x7FC00000u)
+                             : (s == 0 ? __uint_as_float(0x00400000u) : __uint_as_float(s << 23));
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    float4* dst = reinterpret_cast<float4*>(y + g * kBlock);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = lut[(w[k] >> (4 * i)) & 15] * x;
+      __stcs(dst + 2 * k, make_float4(v[0], v[1], v[2], v[3]));
+      __stcs(dst + 2 * k + 1, make_float4(v[4], v[5], v[6], v[7]));
+    }
+  }
+}
+
+// =================================================================== host
+namespace {
+
+thread_local int t_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return KQ_ERR_CUDA;
+}
+
+struct DeviceInfo {
+  bool ready = false;
+  int status = KQ_OK;
+  int sms = 0;
+  int smem_optin = 0;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceInfo g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int device_info(const DeviceInfo** out, int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return KQ_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    cudaDeviceProp prop;
+    e = cudaGetDeviceProperties(&prop, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    di.status = prop.major == 10 ? KQ_OK : KQ_ERR_DEVICE;
+    di.sms = prop.multiProcessorCount;
+    di.smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+    if (!g_encode) {
+      cudaDriverEntryPointQueryResult qr;
+      void* fn = nullptr;
+      e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                           &qr);
+      if (e != cudaSuccess || qr != cudaDriverEntryPointSuccess || !fn)
+        return cuda_fail(e != cudaSuccess ? e : cudaErrorNotSupported);
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    di.ready = true;
+  }
+  *out = &di;
+  *dev_out = dev;
+  return di.status;
+}
+
+bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+int check_shape(int64_t M, int64_t d) {
+  if (M < 0 || d < kBlock || d % kBlock != 0) return KQ_ERR_INVALID;
+  if (M > 0 && d > (int64_t(1) << 40) / M) return KQ_ERR_INVALID;
+  return KQ_OK;
+}
+
+// Sets the dynamic shared-memory limit of one kernel once per device.
+template <auto kKernel>
+int allow_smem(int bytes, int dev) {
+  static std::mutex mu;
+  static int done[kMaxDevices] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev] < bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    done[dev] = bytes;
+  }
+  return KQ_OK;
+}
+
+template <int kXf, int kOut>
+int launch_tma(const uint16_t* x, int64_t M, int64_t d, LaunchArgs a, cudaStream_t st,
+               const DeviceInfo& di, int dev) {
+  const int nb = static_cast<int>(d / kBlock);
+  if (nb > kTmaMaxNb) return KQ_ERR_INVALID;
+  const int tab_bytes = table_floats(kXf, nb) * 4;
+  const int fixed = 1024 + tab_bytes + 2 * kMaxStages * 8;
+  const int stages = std::min(kMaxStages, (di.smem_optin - fixed) / kTileBytes);
+  if (stages < 2) return KQ_ERR_INVALID;
+  const int smem = 1024 + stages * kTileBytes + tab_bytes + 2 * stages * 8;
+  int rc = allow_smem<tma_kernel<kXf, kOut>>(smem, dev);
+  if (rc != KQ_OK) return rc;
+  // Rows per launch keep the tile coordinate (an int32) in range.
+  const int64_t rows_per_launch = ((int64_t(1) << 30) / nb);
+  for (int64_t r0 = 0; r0 < M; r0 += rows_per_launch) {
+    const int64_t rows = std::min(rows_per_launch, M - r0);
+    LaunchArgs la = a;
+    la.G = rows * nb;
+    la.nb = nb;
+    la.n_tiles = static_cast<int32_t>((la.G + kTile - 1) / kTile);
+    la.stages = stages;
+    const int64_t off = r0 * nb;          // in 32-blocks
+    if (la.q) la.q += off * 16;
+    if (la.scales) la.scales += off;
+    if (la.y) la.y += off * kBlock;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kBlock), static_cast<cuuint64_t>(la.G)};
+    const cuuint64_t strides[1] = {kBlock * 2};
+    const cuuint32_t box[2] = {kBlock, kTile};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult cr = g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                           const_cast<uint16_t*>(x + off * kBlock), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+    const int grid = std::min(la.n_tiles, di.sms);
+    tma_kernel<kXf, kOut><<<grid, kTmaThreads, smem, st>>>(map, la);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return KQ_OK;
+}
+
+template <int kXf, int kOut, bool kF32In>
+int launch_direct(const void* x, int64_t M, int64_t d, LaunchArgs a, cudaStream_t st,
+                  const DeviceInfo& di, int dev) {
+  const int nb = static_cast<int>(d / kBlock);
+  const int panels = (nb + kDirectThreads - 1) / kDirectThreads;
+  const int smem = table_floats(kXf, std::min(nb, kDirectThreads)) * 4;
+  int rc = allow_smem<direct_kernel<kXf, kOut, kF32In>>(std::max(smem, 1), dev);
+  if (rc != KQ_OK) return rc;
+  a.nb = nb;
+  a.G = M * nb;
+  const int64_t want = std::max<int64_t>(1, (int64_t)di.sms * 8 / panels);
+  const int rows = static_cast<int>(std::min<int64_t>(M, std::min<int64_t>(want, 65535)));
+  dim3 grid(rows, panels);
+  direct_kernel<kXf, kOut, kF32In><<<grid, kDirectThreads, smem, st>>>(x, M, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KQ_OK;
+}
+
+template <int kXf, int kOut>
+int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, uint8_t* scales,
+        float* y, int impl, void* stream) {
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  LaunchArgs a{};
+  a.aux = aux;
+  a.q = q;
+  a.scales = scales;
+  a.y = y;
+  a.inverse = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t nb = d / kBlock;
+  if (impl == KQ_IMPL_AUTO) impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
+  if (impl == KQ_IMPL_TMA) return launch_tma<kXf, kOut>(x, M, d, a, st, *di, dev);
+  if (impl == KQ_IMPL_DIRECT) return launch_direct<kXf, kOut, false>(x, M, d, a, st, *di, dev);
+  return KQ_ERR_INVALID;
+}
+
+int check_quant_args(const uint16_t* x, int64_t M, int64_t d, const void* aux, bool need_aux,
+                     const uint8_t* q, const uint8_t* scales) {
+  int rc = check_shape(M, d);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!x || !q || !scales || (need_aux && !aux)) return KQ_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(q, 16) || (need_aux && !aligned(aux, 4))) return KQ_ERR_INVALID;
+  return KQ_OK;
+}
+
+}  // namespace
+}  // namespace kq
+
+// ================================================================= C ABI
+using namespace kq;
+
+extern "C" int kq_quantize_ex(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                              uint8_t* q_packed, uint8_t* scales, int impl, void* stream) {
+  int rc = check_quant_args(x, M, d, params, true, q_packed, scales);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (impl < KQ_IMPL_AUTO || impl > KQ_IMPL_WARP) return KQ_ERR_INVALID;
+  return run<kXfKron, kOutMx4>(x, M, d, params, q_packed, scales, nullptr, impl, stream);
+}
+
+extern "C" int kq_quantize(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                           uint8_t* q_packed, uint8_t* scales, void* stream) {
+  return kq_quantize_ex(x, M, d, params, q_packed, scales, KQ_IMPL_AUTO, stream);
+}
+
+extern "C" int kq_quantize_hadamard(const uint16_t* x, int64_t M, int64_t d, uint8_t* q_packed,
+                                    uint8_t* scales, void* stream) {
+  int rc = check_quant_args(x, M, d, nullptr, false, q_packed, scales);
+  if (rc != KQ_OK || M == 0) return rc;
+  return run<kXfHadamard, kOutMx4>(x, M, d, nullptr, q_packed, scales, nullptr, KQ_IMPL_AUTO,
+                                   stream);
+}
+
+extern "C" int kq_quantize_smooth(const uint16_t* x, int64_t M, int64_t d, const float* inv_s,
+                                  uint8_t* q_packed, uint8_t* scales, void* stream) {
+  int rc = check_quant_args(x, M, d, inv_s, true, q_packed, scales);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!aligned(inv_s, 16)) return KQ_ERR_INVALID;
+  return run<kXfSmooth, kOutMx4>(x, M, d, inv_s, q_packed, scales, nullptr, KQ_IMPL_AUTO, stream);
+}
+
+extern "C" int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                            float* y, void* stream) {
+  int rc = check_shape(M, d);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!x || !params || !y || !aligned(x, 16) || !aligned(y, 16) || !aligned(params, 4))
+    return KQ_ERR_INVALID;
+  return run<kXfKron, kOutF32>(x, M, d, params, nullptr, nullptr, y, KQ_IMPL_AUTO, stream);
+}
+
+extern "C" int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,
+                                    float* x, void* stream) {
+  int rc = check_shape(M, d);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!y || !params || !x || !aligned(y, 16) || !aligned(x, 16) || !aligned(params, 4))
+    return KQ_ERR_INVALID;
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  LaunchArgs a{};
+  a.aux = params;
+  a.y = x;
+  a.inverse = 1;
+  return launch_direct<kXfKron, kOutF32, true>(y, M, d, a, static_cast<cudaStream_t>(stream), *di,
+                                               dev);
+}
+
+extern "C" int kq_dequantize(const uint8_t* q_packed, const uint8_t* scales, int64_t M, int64_t d,
+                             float* y, void* stream) {
+  int rc = check_shape(M, d);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!q_packed || !scales || !y || !aligned(q_packed, 16) || !aligned(y, 16)) return KQ_ERR_INVALID;
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  const int64_t G = M * (d / kBlock);
+  const int64_t want = (G + 255) / 256;
+  const int grid = static_cast<int>(std::min<int64_t>(want, (int64_t)di->sms * 8));
+  dequant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(q_packed, scales, G, y);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KQ_OK;
+}
+
+extern "C" const char* kq_status_string(int status) {
+  switch (status) {
+    case KQ_OK: return "ok";
+    case KQ_ERR_INVALID: return "invalid argument";
+    case KQ_ERR_CUDA: return "CUDA error";
+    case KQ_ERR_DEVICE: return "unsupported device (needs sm_100)";
+    case KQ_ERR_TIMEOUT: return "a bounded device wait gave up";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int kq_last_cuda_error(void) { return t_last_cuda_error; }
+
+extern "C" int kq_device_status(int* flags) {
+  if (!flags) return KQ_ERR_INVALID;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int zero = 0;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e);
+  *flags = v;
+  return KQ_OK;
+}
+
+extern "C" int kq_version(void) { return (1 << 16) | 0; }

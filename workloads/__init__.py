@@ -128,9 +128,13 @@ def synth_inv_s(x: torch.Tensor) -> np.ndarray:
 
 
 def make_case(name: str, d_idx: int = 0, gain_idx: int = 0, M: Optional[int] = None,
-              threads: Optional[int] = None) -> Case:
+              threads: Optional[int] = None, row0: int = 0) -> Case:
     """Build a seeded case; ``M`` (default: the config's token count) keeps a
-    row prefix of the full-size case."""
+    row prefix of the full-size case.  ``row0`` (a multiple of ``ROW_CHUNK``)
+    starts the rows further down the same stream, so that several shards of
+    one larger batch can be drawn independently."""
+    if row0 % ROW_CHUNK:
+        raise ValueError("row0 must be a multiple of ROW_CHUNK")
     cfg = CONFIGS[name]
     d = cfg["d"][d_idx]
     gain = cfg["gains"][gain_idx]
@@ -142,7 +146,7 @@ def make_case(name: str, d_idx: int = 0, gain_idx: int = 0, M: Optional[int] = N
     def fill(chunk: int) -> None:
         r0 = chunk * ROW_CHUNK
         rows = min(ROW_CHUNK, M - r0)
-        v = _draw_rows(cfg["dist"], seed, chunk, ROW_CHUNK, d)[:rows] * g
+        v = _draw_rows(cfg["dist"], seed, chunk + row0 // ROW_CHUNK, ROW_CHUNK, d)[:rows] * g
         x[r0:r0 + rows] = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
 
     n_chunks = (M + ROW_CHUNK - 1) // ROW_CHUNK
@@ -175,6 +179,19 @@ def random_bf16(shape, seed: int, scale: float = 1.0) -> torch.Tensor:
     return torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
 
 
+def device_randn_bf16(shape, seed: int, device) -> torch.Tensor:
+    """N(0, 1) bf16 drawn on the device by torch's seeded generator, for
+    inputs too large to draw on the host (large-offset tests)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(int(seed))
+    out = torch.empty(shape, dtype=torch.bfloat16, device=device)
+    rows = max(1, (1 << 26) // max(1, shape[1]))
+    for r0 in range(0, shape[0], rows):
+        blk = torch.randn((min(rows, shape[0] - r0), shape[1]), generator=gen, device=device)
+        out[r0:r0 + blk.shape[0]] = blk.to(torch.bfloat16)
+    return out
+
+
 def bf16_from_float(values) -> torch.Tensor:
     """bf16 tensor from values that are exactly representable in bf16."""
     t = torch.as_tensor(np.asarray(values, dtype=np.float32))
@@ -191,5 +208,5 @@ def algorithmic_bytes(M: int, d: int) -> float:
 
 
 __all__ = ["CONFIGS", "Case", "make_case", "case_seed", "all_case_keys", "random_bf16",
-           "bf16_from_float", "draw_params", "channel_gain", "synth_inv_s", "algorithmic_bytes",
+           "bf16_from_float", "device_randn_bf16", "draw_params", "channel_gain", "synth_inv_s", "algorithmic_bytes",
            "ROW_CHUNK", "BLOCK"]
