@@ -299,8 +299,8 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    M = w.CONFIGS[WORKLOAD]["M"]
-    case = w.make_case(WORKLOAD, row0=shard_row0(rank, M))
+    M = args.rows or w.CONFIGS[WORKLOAD]["M"]
+    case = w.make_case(WORKLOAD, M=M, row0=shard_row0(rank, -(-M // w.ROW_CHUNK) * w.ROW_CHUNK))
     d = case.d
     x = case.x.to(dev)
     params = torch.from_numpy(case.params).to(dev)
@@ -310,8 +310,15 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
     alg_bytes = w.algorithmic_bytes(M, d)
 
-    def step():
-        kq.quantize(x, params, q, s)
+    if args.op == "kron":
+        def step():
+            kq.quantize(x, params, q, s)
+    elif args.op == "hadamard":
+        def step():
+            kq.quantize_hadamard(x, q, s)
+    else:
+        def step():
+            kq.quantize_smooth(x, inv_s, q, s)
 
     # Clock ramp: untimed launches for ~0.3 s so the timed region starts warm.
     t_end = time.perf_counter() + 0.3
@@ -334,7 +341,14 @@ def run_gpu(args):
         buf = torch.empty_like(x)
         ms_c, _ = time_steps(lambda: buf.copy_(x), args.steps, args.warmup, stream)
         ms_max_c = max_over_ranks(ms_c, dev)
+        impls = {}
+        for name, code in (("panel", kq.KQ_IMPL_PANEL), ("tma_flat", kq.KQ_IMPL_TMA),
+                           ("direct", kq.KQ_IMPL_DIRECT)):
+            ms_i, _ = time_steps(lambda: kq.quantize(x, params, q, s, impl=code), args.steps,
+                                 args.warmup, stream)
+            impls[name] = alg_bytes / (max_over_ranks(ms_i, dev) * 1e-3) / 1e9
         variants = {
+            "kq_quantize_impl_gbs": impls,
             "hadamard": {"gbs": alg_bytes / (ms_max_h * 1e-3) / 1e9, "ms": ms_max_h},
             "smooth": {"gbs": alg_bytes / (ms_max_s * 1e-3) / 1e9, "ms": ms_max_s},
             "kronecker_over_smooth_speed": ms_max_s / ms_max,
@@ -375,7 +389,7 @@ def run_gpu(args):
     roof = {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
             "frac": per_launch_gbs / peak, "peak_source": peak_src,
             "traffic": profiled_traffic(khash, "kq_quantize_stress_traffic.md"),
-            "algorithmic_bytes_per_launch": alg_bytes, "kernel": "tma_kernel<kron, mx4>",
+            "algorithmic_bytes_per_launch": alg_bytes, "kernel": "panel_kernel<kron, mx4, 2>",
             "kernel_source_hash": khash}
 
     cpu = None
@@ -397,7 +411,7 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": dict(_config(d, M, "tma"), global_batch_rows=M * world,
+            "config": dict(_config(d, M, "panel"), op=args.op, global_batch_rows=M * world,
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3),
             "hbm_frac": value / world / peak,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
@@ -418,6 +432,12 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the comparator timings")
+    ap.add_argument("--op", default="kron", choices=["kron", "hadamard", "smooth"],
+                    help="quantizer timed as the step (kron = kq_quantize, the metric; "
+                         "the comparators are for profiling)")
+    ap.add_argument("--rows", type=int, default=0,
+                    help="rows of the stress input per GPU (default: its 16384); "
+                         "smaller values are for profiling captures only")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

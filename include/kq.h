@@ -35,8 +35,9 @@
  *     inv_s 4-byte aligned; scales has no alignment requirement.
  *   - stream is a cudaStream_t (NULL = the legacy default stream).  Calls are
  *     asynchronous: they enqueue kernels and return without synchronising.
- *   - Results for non-finite inputs or parameters (b_k == 0, NaN, Inf, or a
- *     transform that overflows float32) are unspecified.
+ *   - Results for non-finite inputs or parameters (b_k == 0, NaN, Inf), for a
+ *     transform that overflows float32, or for |x| >= 2^100 (intermediate
+ *     butterfly values may overflow) are unspecified.
  *   - Return value: KQ_OK, KQ_ERR_INVALID (argument check failed, nothing
  *     enqueued), KQ_ERR_CUDA (a CUDA call or launch failed; see
  *     kq_last_cuda_error) or KQ_ERR_DEVICE (current device is not sm_100).
@@ -64,7 +65,8 @@ enum {
     KQ_IMPL_AUTO = 0,       /* what kq_quantize uses */
     KQ_IMPL_TMA = 1,        /* TMA-staged, persistent, thread per 32-block */
     KQ_IMPL_DIRECT = 2,     /* direct 32-byte global loads, thread per 32-block */
-    KQ_IMPL_WARP = 3        /* one 32-block per warp, shuffle butterfly */
+    KQ_IMPL_WARP = 3,       /* one 32-block per warp, shuffle butterfly */
+    KQ_IMPL_PANEL = 4       /* TMA-staged column panels, factors in registers */
 };
 
 /* KroQuant quantizer, the hot path: q_packed/scales = MXFP4(x T).

@@ -103,9 +103,12 @@ def check_mx4(q_gpu, s_gpu, y64, cond, tol: float = TOL, strict_zero_sign: bool 
             f"{int((~ok).sum())} codes outside the allowed set: " + str(
                 [(tuple(i), int(c_gpu[tuple(i)]), int(codes_ref[tuple(i)]), float(v[tuple(i)]),
                   float(vb[tuple(i)])) for i in idx]))
+    differ = c_gpu != codes_ref
+    zero_sign = differ & ((c_gpu & 7) == 0) & ((codes_ref & 7) == 0)
     return {
         "scale_exempt": int((s_int != s_ref).sum()),
-        "code_exempt": int((c_gpu != codes_ref).sum()),
+        "code_exempt": int((differ & ~zero_sign).sum()),
+        "zero_sign_exempt": int(zero_sign.sum()),
         "blocks": int(M * nb),
         "elements": int(M * d),
     }

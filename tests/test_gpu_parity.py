@@ -42,7 +42,7 @@ def _run_all_variants(x_bits, x_t, params, inv_s):
             dict(q=q, s=s, qh=qh, sh=sh, qs=qs, ss=ss, y=y).items()}
 
 
-def _check_rows(out, x_bits, params, inv_s, rows=None):
+def _check_rows(out, x_bits, params, inv_s, rows=None, bound_exemptions=True):
     """Oracle comparison on all rows, or on the given row indices."""
     if rows is not None:
         x_bits = x_bits[rows]
@@ -58,9 +58,12 @@ def _check_rows(out, x_bits, params, inv_s, rows=None):
     # A single float32 product is exact on both sides: no tolerance band.
     sts = check_mx4(out["qs"], out["ss"], ys, np.zeros_like(ys), strict_zero_sign=True)
     assert sts["scale_exempt"] == 0 and sts["code_exempt"] == 0
-    for stats in (st, sth):
-        assert stats["scale_exempt"] <= max(2, stats["blocks"] // 1000)
-        assert stats["code_exempt"] <= max(4, stats["elements"] // 10000)
+    if bound_exemptions:
+        # Boundary cases are rare on these inputs: far more would point at a
+        # kernel that is right only to within the band everywhere.
+        for stats in (st, sth):
+            assert stats["scale_exempt"] <= max(2, stats["blocks"] // 1000)
+            assert stats["code_exempt"] <= max(4, stats["elements"] // 10000)
     return worst, st, sth
 
 
@@ -106,7 +109,23 @@ def test_full_size_sampled_rows(key):
     _requantize_is_identity(out["q"], out["s"], c.M, c.d)
 
 
-def test_impls_agree_bitwise():
+IMPLS = {"panel": kq.KQ_IMPL_PANEL, "tma": kq.KQ_IMPL_TMA, "direct": kq.KQ_IMPL_DIRECT}
+
+
+@pytest.mark.parametrize("impl", sorted(IMPLS))
+@pytest.mark.parametrize("key", [("sana", 1, 0), ("flux_schnell", 1, 2), ("tiny", 0, 0)],
+                         ids=lambda k: f"{k[0]}-d{k[1]}-g{k[2]}")
+def test_each_implementation_against_oracle(impl, key):
+    name, di, gi = key
+    c = w.make_case(name, di, gi, M=301 if name != "tiny" else 256)
+    q, s = kq.quantize(_gpu(c.x), _params_dev(c.params), impl=IMPLS[impl])
+    x64 = o.bf16_bits_to_float64(c.x_bits())
+    check_mx4(q.cpu().numpy(), s.cpu().numpy(), o.transform(x64, c.params),
+              o.abs_transform(x64, c.params))
+
+
+def test_table_implementations_agree_bitwise():
+    """The flat TMA and the direct kernel run the same four-term stages."""
     c = w.make_case("sana", 1, M=301)
     xd, pd = _gpu(c.x), _params_dev(c.params)
     q1, s1 = kq.quantize(xd, pd, impl=kq.KQ_IMPL_TMA)
@@ -114,13 +133,32 @@ def test_impls_agree_bitwise():
     assert torch.equal(q1, q2) and torch.equal(s1, s2)
 
 
+def test_singular_shear_factor_takes_the_plain_form():
+    """(a, b, c) = (-1, 1, 1) gives G = [[1, 1], [-1, 0]] (det 1, g11 = 0):
+    the scaled-shear form cannot hold it, so its panel runs the plain
+    four-term stages; the other panels keep the shear form."""
+    c = w.make_case("flux_schnell", 0, 0, M=150)
+    p = c.params.copy()
+    p[5, 2] = [-1.0, 1.0, 1.0]                 # block 5, factor G3
+    p[90, 0] = [-1.0, 1.0, 1.0]                # a block in another panel
+    pd = _params_dev(p)
+    xd = _gpu(c.x)
+    q, s = kq.quantize(xd, pd)
+    y = kq.transform(xd, pd)
+    x64 = o.bf16_bits_to_float64(c.x_bits())
+    y64 = o.transform(x64, p)
+    cond = o.abs_transform(x64, p)
+    check_transform(y.cpu().numpy(), y64, cond)
+    check_mx4(q.cpu().numpy(), s.cpu().numpy(), y64, cond)
+
+
 # ------------------------------------------------------------- edge cases
-def _edge(x_t, params, inv_s=None):
+def _edge(x_t, params, inv_s=None, bound=True):
     if inv_s is None:
         inv_s = np.ones(x_t.shape[1], dtype=np.float32)
     out = _run_all_variants(None, x_t, params, inv_s)
     bits = x_t.view(torch.int16).numpy().view(np.uint16)
-    _check_rows(out, bits, params, inv_s)
+    _check_rows(out, bits, params, inv_s, bound_exemptions=bound)
     return out
 
 
@@ -129,9 +167,12 @@ def test_single_block():
     _edge(x, w.draw_params(32, 1))
 
 
-def test_wide_rows_use_the_panel_kernel():
-    for d in (512 * 32, 513 * 32):          # last TMA width and first fallback width
-        x = w.random_bf16((3, d), seed=d)
+def test_wide_and_prime_width_rows():
+    """512 blocks (one 256-wide panel pair), 513 = 27 * 19 (57-wide panels)
+    and 521 blocks (prime: no useful panel, the flat TMA/direct path)."""
+    for nb in (512, 513, 521):
+        d = nb * 32
+        x = w.random_bf16((5, d), seed=d)
         _edge(x, w.draw_params(d, 2))
 
 
@@ -144,7 +185,7 @@ def test_zero_subnormal_and_huge_blocks():
     x[3, 0:32] = -0.0
     x[3, 32] = 1e-38
     t = torch.from_numpy(x).to(torch.bfloat16)
-    out = _edge(t, w.draw_params(d, 3))
+    out = _edge(t, w.draw_params(d, 3), bound=False)
     assert (out["s"][0] == 0).all() and (out["q"][0] & 0x77 == 0).all()
 
 

@@ -48,6 +48,13 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// Orders this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy (TMA) accesses: needed before a stage that was read with
+// ordinary loads is handed back to be overwritten by a TMA load.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar))
                : "memory");
@@ -83,6 +90,16 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_addr(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// 3-D tiled bulk tensor load into this CTA's shared memory (no multicast).
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
       : "memory");
 }
 
@@ -210,6 +227,158 @@ __device__ __forceinline__ void kron_entry(float* entry, const float* p, bool in
   }
 }
 
+// --------------------------------------------- register-resident factors
+// The factors of one column block, held in registers by a thread that keeps
+// the same block for the whole kernel.
+//
+// Scaled-shear form: with row-vector factors G = [[g00, g01], [g10, g11]],
+//     G = S D,   S = [[1, r01], [r10, 1]],   D = diag(g00, g11),
+//     r10 = g10 / g00 = a,   r01 = g01 / g11 = c / (a c + 1/b),
+// and by the mixed-product rule K = (S1 (x) ... (x) S5)(D1 (x) ... (x) D5):
+// five stages of one multiply-add per output, then one multiply by the
+// diagonal delta_i = prod_k (bit_k(i) ? g11_k : g00_k).  Since |S||D| = |G|
+// entrywise, the rounding error stays bounded by the same |x| |K| as the
+// plain four-term stage.  It needs every g11 != 0 and a bounded growth of
+// the intermediate values; blocks that miss that use the plain form.
+struct ShearDiag {
+  f2 r10[4], r01[4];     // stages on index bits 4..1, both halves equal
+  float r10b, r01b;      // stage on bit 0
+  f2 delta[16];          // (delta_2m, delta_2m+1)
+};
+
+struct PlainFactors {
+  f2 g00[4], g10[4], g01[4], g11[4];   // bits 4..1
+  float h00, h10, h01, h11;            // bit 0
+};
+
+// Bound on the growth of the shear form's intermediate values over the five
+// stages (prod_k max(1 + |r10|, 1 + |r01|)): with inputs below 2^100 they
+// stay inside the float32 range.
+constexpr double kShearGrowthMax = 16777216.0;   // 2^24
+
+// The four entries of G_k (row-vector form) from (a, b, c), in double.
+__device__ __forceinline__ void factor_entries(const float* p, int k, double& g00, double& g01,
+                                               double& g10, double& g11) {
+  const double a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
+  g00 = b;
+  g01 = c;
+  g10 = a * b;
+  g11 = __fma_rn(a, c, 1.0 / b);
+}
+
+// Fills the shear form for the block with parameters p[15]; returns false if
+// the block must use the plain form instead.
+__device__ __forceinline__ bool load_shear_diag(ShearDiag& f, const float* p) {
+  double g00[kFactors], g11[kFactors];
+  double growth = 1.0;
+  bool ok = true;
+  float r10[kFactors], r01[kFactors];
+#pragma unroll
+  for (int k = 0; k < kFactors; ++k) {
+    double a00, a01, a10, a11;
+    factor_entries(p, k, a00, a01, a10, a11);
+    g00[k] = a00;
+    g11[k] = a11;
+    const double ra = p[3 * k + 0];
+    const double rb = a01 / a11;
+    ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
+    growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
+    r10[k] = (float)ra;
+    r01[k] = (float)rb;
+  }
+  ok = ok && (growth <= kShearGrowthMax);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f.r10[k] = pack2(r10[k], r10[k]);
+    f.r01[k] = pack2(r01[k], r01[k]);
+  }
+  f.r10b = r10[4];
+  f.r01b = r01[4];
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    double d0 = 1.0, d1;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) d0 *= ((2 * m) >> (4 - k)) & 1 ? g11[k] : g00[k];
+    d1 = d0 * g11[4];
+    d0 = d0 * g00[4];
+    f.delta[m] = pack2((float)d0, (float)d1);
+  }
+  return ok;
+}
+
+__device__ __forceinline__ void load_plain(PlainFactors& f, const float* p) {
+#pragma unroll
+  for (int k = 0; k < kFactors; ++k) {
+    double g00, g01, g10, g11;
+    factor_entries(p, k, g00, g01, g10, g11);
+    const float f00 = (float)g00, f01 = (float)g01, f10 = (float)g10, f11 = (float)g11;
+    if (k < 4) {
+      f.g00[k] = pack2(f00, f00);
+      f.g01[k] = pack2(f01, f01);
+      f.g10[k] = pack2(f10, f10);
+      f.g11[k] = pack2(f11, f11);
+    } else {
+      f.h00 = f00; f.h01 = f01; f.h10 = f10; f.h11 = f11;
+    }
+  }
+}
+
+template <int kHalfDist>
+__device__ __forceinline__ void shear_stage(f2 (&u)[16], f2 r10, f2 r01) {
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    if (m & kHalfDist) continue;
+    const f2 lo = u[m], hi = u[m + kHalfDist];
+    u[m] = fma2(r10, hi, lo);
+    u[m + kHalfDist] = fma2(r01, lo, hi);
+  }
+}
+
+// The shear stages; the diagonal is applied by the caller.
+__device__ __forceinline__ void shear_apply(f2 (&u)[16], const ShearDiag& f) {
+  shear_stage<8>(u, f.r10[0], f.r01[0]);
+  shear_stage<4>(u, f.r10[1], f.r01[1]);
+  shear_stage<2>(u, f.r10[2], f.r01[2]);
+  shear_stage<1>(u, f.r10[3], f.r01[3]);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    float lo, hi;
+    unpack2(u[m], lo, hi);
+    u[m] = pack2(__fmaf_rn(f.r10b, hi, lo), __fmaf_rn(f.r01b, lo, hi));
+  }
+}
+
+// Per-element diagonal multiply (the shear form's D, or SmoothQuant's 1/s).
+__device__ __forceinline__ void diag_mul(f2 (&u)[16], const f2 (&delta)[16]) {
+#pragma unroll
+  for (int m = 0; m < 16; ++m) u[m] = mul2(u[m], delta[m]);
+}
+
+template <int kHalfDist>
+__device__ __forceinline__ void plain_stage(f2 (&u)[16], f2 g00, f2 g10, f2 g01, f2 g11) {
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    if (m & kHalfDist) continue;
+    const f2 lo = u[m], hi = u[m + kHalfDist];
+    u[m] = fma2(g10, hi, mul2(g00, lo));
+    u[m + kHalfDist] = fma2(g11, hi, mul2(g01, lo));
+  }
+}
+
+__device__ __forceinline__ void plain_apply(f2 (&u)[16], const PlainFactors& f) {
+  plain_stage<8>(u, f.g00[0], f.g10[0], f.g01[0], f.g11[0]);
+  plain_stage<4>(u, f.g00[1], f.g10[1], f.g01[1], f.g11[1]);
+  plain_stage<2>(u, f.g00[2], f.g10[2], f.g01[2], f.g11[2]);
+  plain_stage<1>(u, f.g00[3], f.g10[3], f.g01[3], f.g11[3]);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    float lo, hi;
+    unpack2(u[m], lo, hi);
+    u[m] = pack2(__fmaf_rn(f.h10, hi, __fmul_rn(f.h00, lo)),
+                 __fmaf_rn(f.h11, hi, __fmul_rn(f.h01, lo)));
+  }
+}
+
 // Fixed block Hadamard H_32 (Sylvester order: H2 = [[1,1],[1,-1]] on every
 // bit), then the orthonormal factor 1/sqrt(32) as one float32 multiply.
 __device__ __forceinline__ void hadamard_apply(f2 (&u)[16]) {
@@ -234,12 +403,14 @@ __device__ __forceinline__ void hadamard_apply(f2 (&u)[16]) {
 }
 
 // Per-channel scaling y[c] = x[c] * inv_s[c]; ``inv`` points at the block's
-// 32 reciprocal scales (16-byte aligned).
-__device__ __forceinline__ void smooth_apply(f2 (&u)[16], const float* inv) {
+// 32 reciprocal scales in shared memory, stored as 8 chunks of 4 with chunk i
+// at position i ^ (j & 7), so that eight threads with consecutive blocks j
+// read eight different bank groups.
+__device__ __forceinline__ void smooth_apply(f2 (&u)[16], const float* inv, int j) {
   const float4* v = reinterpret_cast<const float4*>(inv);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float4 s = v[i];
+    const float4 s = v[i ^ (j & 7)];
     u[2 * i] = mul2(u[2 * i], pack2(s.x, s.y));
     u[2 * i + 1] = mul2(u[2 * i + 1], pack2(s.z, s.w));
   }
@@ -252,18 +423,34 @@ struct Mx4Block {
   uint32_t scale;
 };
 
-__device__ __forceinline__ Mx4Block mxfp4_block(const f2 (&u)[16]) {
-  float m[16];
+// Three-input maximum (sm_100).
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Largest magnitude of the 32 values: a tree of three-input maxima.
+__device__ __forceinline__ float block_amax(const f2 (&u)[16]) {
+  float a[32];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    float lo, hi;
-    unpack2(u[i], lo, hi);
-    m[i] = fmaxf(fabsf(lo), fabsf(hi));
+    unpack2(u[i], a[2 * i], a[2 * i + 1]);
+    a[2 * i] = fabsf(a[2 * i]);
+    a[2 * i + 1] = fabsf(a[2 * i + 1]);
   }
+  float b[11];
 #pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
+  for (int i = 0; i < 10; ++i) b[i] = max3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[10] = fmaxf(a[30], a[31]);
+  const float c0 = max3(b[0], b[1], b[2]), c1 = max3(b[3], b[4], b[5]);
+  const float c2 = max3(b[6], b[7], b[8]), c3 = fmaxf(b[9], b[10]);
+  return fmaxf(max3(c0, c1, c2), c3);
+}
+
+__device__ __forceinline__ Mx4Block mxfp4_block(const f2 (&u)[16]) {
+  float m[1];
+  m[0] = block_amax(u);
   // floor(log2(amax)) is the biased exponent field minus 127, so the scale
   // byte e + 127 = field - 2, clamped at 0 (zero and subnormal maxima too).
   const int field = static_cast<int>(__float_as_uint(m[0]) >> 23);

@@ -14,6 +14,7 @@
 
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "kq.h"
@@ -58,7 +59,10 @@ __device__ __forceinline__ void build_table(float* tab, const LaunchArgs& a, int
   } else if (kXf == kXfSmooth) {
     const float4* src = reinterpret_cast<const float4*>(a.aux + (int64_t)j0 * kBlock);
     float4* dst = reinterpret_cast<float4*>(tab);
-    for (int i = t; i < jn * (kBlock / 4); i += nt) dst[i] = src[i];
+    for (int i = t; i < jn * (kBlock / 4); i += nt) {
+      const int j = i >> 3, c = i & 7;           // block j's chunk c -> position c ^ (j & 7)
+      dst[8 * j + (c ^ (j & 7))] = src[i];
+    }
   }
 }
 
@@ -66,7 +70,7 @@ template <int kXf>
 __device__ __forceinline__ void apply_xform(f2 (&u)[16], const float* tab, int j) {
   if (kXf == kXfKron) kron_apply(u, tab + j * kTabStride);
   else if (kXf == kXfHadamard) hadamard_apply(u);
-  else smooth_apply(u, tab + j * kBlock);
+  else smooth_apply(u, tab + j * kBlock, j);
 }
 
 template <int kOut>
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < a.stages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumers);
+      mbar_init(&empty[s], kConsumerWarps);
     }
     fence_mbar_init();
   }
@@ -157,15 +161,20 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   const uint32_t swz = (tid >> 1) & 3;
   for (int i = 0; i < n_local; ++i) {
     const int s = i % S;
-    if (!mbar_wait(&full[s], (i / S) & 1)) {
-      atomicOr(&g_device_error, kErrConsumerWait);
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], (i / S) & 1))) {
+      if ((tid & 31) == 0) atomicOr(&g_device_error, kErrConsumerWait);
       break;
     }
     const uint8_t* row = stages + s * kTileBytes + tid * (kBlock * 2);
     uint4 c[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) c[q] = *reinterpret_cast<const uint4*>(row + 16 * (q ^ swz));
-    mbar_arrive(&empty[s]);
+    // Hand the stage back: the reads above must be ordered before the TMA
+    // load that will overwrite it (generic -> async proxy), then one arrival
+    // per warp.
+    fence_proxy_async_smem();
+    __syncwarp();
+    if ((tid & 31) == 0) mbar_arrive(&empty[s]);
     if (g < a.G) {
       f2 u[16];
 #pragma unroll
@@ -182,6 +191,227 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     j += jstep;
     if (j >= a.nb) j -= a.nb;
   }
+}
+
+// ------------------------------------------------------------ panel kernel
+// CTA c owns the column panel c % panels (W consecutive 32-blocks of every
+// row) and walks its row tiles; consumer thread t < W*R keeps column block
+// j = panel*W + t % W for the whole kernel (its factors stay in registers)
+// and handles rows t / W + r*R, r < kRpt, of every tile.  A tile is the TMA
+// box {32 elements, W blocks, kRpt*R rows} of the 3-D view x[M][nb][32].
+struct PanelArgs {
+  int64_t M;            // rows
+  int32_t nb;           // 32-blocks per row
+  int32_t W;            // panel width in 32-blocks (divides nb)
+  int32_t R;            // thread rows per tile (a tile holds kRpt * R rows)
+  int32_t panels;       // nb / W
+  int32_t row_tiles;    // ceil(M / (kRpt * R))
+  int32_t stages;       // TMA ring depth
+  int32_t tile_bytes;   // W * kRpt * R * 64 (one TMA box)
+  int32_t stage_bytes;  // tile_bytes rounded up to 1 KiB: every stage starts on
+                        // a multiple of the 512-byte 64B-swizzle period
+  const float* aux;     // params [nb][5][3] (Kronecker) or inv_s [nb*32] (smooth)
+  uint8_t* q;
+  uint8_t* scales;
+  float* y;
+};
+
+// Launch shape of the panel kernel: consumer warps, rows per consumer thread
+// per tile, and CTAs per SM it is compiled for.
+template <int kCW_, int kRpt_, int kMinBlocks_>
+struct PanelCfg {
+  static constexpr int kCW = kCW_;
+  static constexpr int kRpt = kRpt_;
+  static constexpr int kMinBlocks = kMinBlocks_;
+  static constexpr int kCons = 32 * kCW_;
+  static constexpr int kThreads = kCons + 32;
+};
+
+// Hands a stage back to the producer: the generic->async proxy fence orders
+// this thread's shared-memory reads of the stage before the TMA load that
+// will overwrite it (without it, lanes were seen reading the next tile's
+// data); then one arrival per warp.
+__device__ __forceinline__ void release_stage(uint64_t* bar, int lane) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar);
+}
+
+template <int kXf, int kOut, class Cfg, int kForm>
+__device__ __forceinline__ void panel_consume(const PanelArgs& a, const uint8_t* stages,
+                                              uint64_t* full, uint64_t* empty, int n_local,
+                                              int k0, int cpp, int tid, bool active, int rho,
+                                              int j, const ShearDiag& sd, const PlainFactors& pf) {
+  constexpr int kRpt = Cfg::kRpt;
+  const int S = a.stages;
+  const int lane = tid & 31;
+  // Byte offsets of this thread's 16-byte chunks inside a stage: row
+  // ridx = (rho + r R) W + (t mod W) holds chunk q at q ^ ((ridx >> 1) & 3).
+  uint32_t off[kRpt][4];
+#pragma unroll
+  for (int r = 0; r < kRpt; ++r) {
+    const int ridx = (rho + r * a.R) * a.W + (tid % a.W);
+    const uint32_t swz = (ridx >> 1) & 3;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) off[r][q] = ridx * (kBlock * 2) + 16 * (q ^ swz);
+  }
+  const int64_t tile_rows = (int64_t)kRpt * a.R;
+  int64_t row = k0 * tile_rows + rho;
+  const int64_t row_step = (int64_t)cpp * tile_rows;
+  int s = 0;
+  uint32_t phase = 0;
+  for (int i = 0; i < n_local; ++i) {
+    // Every lane waits; the warp gives up only as a whole, so that no lane
+    // leaves while the others sit in a warp-wide operation.
+    if (!__all_sync(0xFFFFFFFFu, mbar_wait(&full[s], phase))) {
+      if (lane == 0) atomicOr(&g_device_error, kErrConsumerWait);
+      return;
+    }
+    const uint8_t* st = stages + s * a.stage_bytes;
+    uint4 c[kRpt][4];
+#pragma unroll
+    for (int r = 0; r < kRpt; ++r)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        c[r][q] = active ? *reinterpret_cast<const uint4*>(st + off[r][q]) : make_uint4(0, 0, 0, 0);
+    release_stage(&empty[s], lane);
+    if (++s == S) {
+      s = 0;
+      phase ^= 1;
+    }
+    const int64_t row_i = row;
+    row += row_step;
+    if (!active) continue;
+#pragma unroll
+    for (int r = 0; r < kRpt; ++r) {
+      const int64_t rr = row_i + (int64_t)r * a.R;
+      if (rr >= a.M) break;
+      f2 u[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        u[4 * q + 0] = bf16x2_to_f2(c[r][q].x);
+        u[4 * q + 1] = bf16x2_to_f2(c[r][q].y);
+        u[4 * q + 2] = bf16x2_to_f2(c[r][q].z);
+        u[4 * q + 3] = bf16x2_to_f2(c[r][q].w);
+      }
+      if (kXf == kXfKron && kForm == 1) {
+        plain_apply(u, pf);
+      } else if (kXf == kXfHadamard) {
+        hadamard_apply(u);
+      } else {
+        if (kXf == kXfKron) shear_apply(u, sd);
+        diag_mul(u, sd.delta);
+      }
+      const int64_t g = rr * a.nb + j;
+      if (kOut == kOutMx4) {
+        const Mx4Block b = mxfp4_block(u);
+        __stcs(reinterpret_cast<uint4*>(a.q + g * 16), b.codes);
+        a.scales[g] = static_cast<uint8_t>(b.scale);
+      } else {
+        float4* dst = reinterpret_cast<float4*>(a.y + g * kBlock);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          float x0, x1, x2, x3;
+          unpack2(u[2 * t], x0, x1);
+          unpack2(u[2 * t + 1], x2, x3);
+          __stcs(dst + t, make_float4(x0, x1, x2, x3));
+        }
+      }
+    }
+  }
+}
+
+template <int kXf, int kOut, class Cfg>
+__global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
+    panel_kernel(const __grid_constant__ CUtensorMap xmap, const PanelArgs a) {
+  constexpr int kRpt = Cfg::kRpt;
+  constexpr int kCons = Cfg::kCons;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = base;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + a.stages * a.stage_bytes);
+  uint64_t* empty = full + a.stages;
+  const int tid = threadIdx.x;
+  const int S = a.stages;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], Cfg::kCW);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  const int panel = blockIdx.x % a.panels;
+  const int cpp = gridDim.x / a.panels;           // CTAs per panel
+  const int k0 = blockIdx.x / a.panels;           // first row tile of this CTA
+  const int n_local = k0 < a.row_tiles ? (a.row_tiles - k0 + cpp - 1) / cpp : 0;
+
+  if (tid >= kCons) {
+    if (tid == kCons) {
+      tma_prefetch_map(&xmap);
+      int issued = 0;
+      bool ok = true;
+      int s = 0;
+      uint32_t phase = 0;                 // parity of the empty-barrier phase to wait for
+      int row0 = k0 * (kRpt * a.R);
+      const int row_step = cpp * (kRpt * a.R);
+      for (int i = 0; i < n_local; ++i) {
+        if (i >= S && !mbar_wait(&empty[s], phase)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], a.tile_bytes);
+        tma_load_3d(stages + s * a.stage_bytes, &xmap, 0, panel * a.W, row0, &full[s]);
+        row0 += row_step;
+        issued = i + 1;
+        if (++s == S) {
+          s = 0;
+          if (i >= S) phase ^= 1;
+        }
+      }
+      if (!ok) {
+        atomicOr(&g_device_error, kErrProducerWait);
+        for (int i = issued > S ? issued - S : 0; i < issued; ++i)
+          mbar_wait(&full[i % S], (i / S) & 1);
+      }
+    }
+    return;
+  }
+
+  const bool active = tid < a.W * a.R;
+  const int rho = tid / a.W;
+  const int j = panel * a.W + (tid % a.W);
+  ShearDiag sd;
+  PlainFactors pf;
+  int plain = 0;
+  if (kXf == kXfKron) {
+    if (active) plain = load_shear_diag(sd, a.aux + (int64_t)j * 15) ? 0 : 1;
+    // One form for the whole CTA: the plain one if any of its blocks needs it.
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+        : "=r"(plain)
+        : "r"(plain), "r"(kCons)
+        : "memory");
+    if (plain && active) load_plain(pf, a.aux + (int64_t)j * 15);
+  } else if (kXf == kXfSmooth) {
+    if (active) {
+      const float4* v = reinterpret_cast<const float4*>(a.aux + (int64_t)j * kBlock);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const float4 x = v[t];
+        sd.delta[2 * t] = pack2(x.x, x.y);
+        sd.delta[2 * t + 1] = pack2(x.z, x.w);
+      }
+    }
+  }
+  if (plain)
+    panel_consume<kXf, kOut, Cfg, 1>(a, stages, full, empty, n_local, k0, cpp, tid, active, rho,
+                                      j, sd, pf);
+  else
+    panel_consume<kXf, kOut, Cfg, 0>(a, stages, full, empty, n_local, k0, cpp, tid, active, rho,
+                                      j, sd, pf);
 }
 
 // ---------------------------------------------------------- direct kernel
@@ -271,6 +501,7 @@ struct DeviceInfo {
   int status = KQ_OK;
   int sms = 0;
   int smem_optin = 0;
+  int smem_per_sm = 0;
 };
 
 constexpr int kMaxDevices = 64;
@@ -292,6 +523,7 @@ int device_info(const DeviceInfo** out, int* dev_out) {
     di.status = prop.major == 10 ? KQ_OK : KQ_ERR_DEVICE;
     di.sms = prop.multiProcessorCount;
     di.smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
+    di.smem_per_sm = static_cast<int>(prop.sharedMemPerMultiprocessor);
     if (!g_encode) {
       cudaDriverEntryPointQueryResult qr;
       void* fn = nullptr;
@@ -373,6 +605,118 @@ int launch_tma(const uint16_t* x, int64_t M, int64_t d, LaunchArgs a, cudaStream
   return KQ_OK;
 }
 
+// Panel shape for nb blocks per row: W divides nb, R = thread rows per tile,
+// W * R <= cons, and W <= 256 and rpt * R <= 256 (TMA box dimension limit); the best thread use wins,
+// then the wider panel.  Returns the fraction of busy consumer threads.
+double panel_shape(int nb, int cons, int rpt, int* W_out, int* R_out) {
+  double best = 0.0;
+  for (int W = std::min(std::min(nb, cons), 256); W >= 1; --W) {
+    if (nb % W) continue;
+    const int R = std::min(cons / W, 256 / rpt);
+    const double use = double(W * R) / cons;
+    if (use > best + 1e-9) {
+      best = use;
+      *W_out = W;
+      *R_out = R;
+    }
+  }
+  return best;
+}
+
+// Panel-kernel shapes measured on B200 (interleaved medians on the
+// 16384 x 12288 stress input, GB/s): 12 consumer warps x 2 rows 5526,
+// 15 x 2 5405, 14 x 2 4971, 8 x 2 4972, 15 x 1 5441, 16 x 1 with the diagonal
+// in shared memory 4978.  More warps hide latency until the register budget
+// (ceil(warps / 4) warps share one scheduler's 16K registers) forces spills.
+using PanelV0 = PanelCfg<12, 2, 1>;
+using PanelV1 = PanelCfg<8, 2, 1>;
+using PanelV2 = PanelCfg<15, 1, 1>;
+constexpr int kDefaultPanel = 0;
+constexpr int kPanelMaxStages = 6;
+
+// KQ_PANEL_VARIANT selects another compiled shape (read at every call; for
+// tuning measurements only).
+int panel_variant() {
+  const char* e = getenv("KQ_PANEL_VARIANT");
+  return e ? atoi(e) : kDefaultPanel;
+}
+
+template <class Cfg>
+double panel_use(int nb, int* W, int* R) {
+  return panel_shape(nb, Cfg::kCons, Cfg::kRpt, W, R);
+}
+
+template <int kXf, int kOut, class Cfg>
+int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q,
+                     uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev) {
+  constexpr int kRpt = Cfg::kRpt;
+  const int nb = static_cast<int>(d / kBlock);
+  PanelArgs a{};
+  if (panel_use<Cfg>(nb, &a.W, &a.R) < 0.5) return KQ_ERR_INVALID;
+  a.M = M;
+  a.nb = nb;
+  a.panels = nb / a.W;
+  a.tile_bytes = a.W * kRpt * a.R * kBlock * 2;
+  a.stage_bytes = (a.tile_bytes + 1023) / 1024 * 1024;
+  // Shared memory per CTA: the opt-in limit, or an equal share of the SM.
+  const int budget = Cfg::kMinBlocks == 1 ? di.smem_optin
+                                          : di.smem_per_sm / Cfg::kMinBlocks - 1024;
+  a.stages = std::min(kPanelMaxStages,
+                      (budget - 1024 - 2 * kPanelMaxStages * 8) / a.stage_bytes);
+  if (a.stages < 2) return KQ_ERR_INVALID;
+  const int64_t tile_rows = (int64_t)kRpt * a.R;
+  const int64_t row_tiles = (M + tile_rows - 1) / tile_rows;
+  if (M > (int64_t(1) << 31) - 1 - tile_rows || row_tiles > (int64_t(1) << 30))
+    return KQ_ERR_INVALID;
+  a.row_tiles = static_cast<int32_t>(row_tiles);
+  a.aux = aux;
+  a.q = q;
+  a.scales = scales;
+  a.y = y;
+  const int smem = 1024 + a.stages * a.stage_bytes + 2 * a.stages * 8;
+  int rc = allow_smem<panel_kernel<kXf, kOut, Cfg>>(smem, dev);
+  if (rc != KQ_OK) return rc;
+  CUtensorMap map;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBlock), static_cast<cuuint64_t>(nb),
+                              static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[2] = {kBlock * 2, static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[3] = {kBlock, static_cast<cuuint32_t>(a.W),
+                             static_cast<cuuint32_t>(tile_rows)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult cr = g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  // A multiple of the panel count, up to the resident CTAs of the device.
+  const int64_t resident = (int64_t)di.sms * Cfg::kMinBlocks;
+  const int64_t per_panel = std::max<int64_t>(1, std::min<int64_t>(resident / a.panels, row_tiles));
+  const int grid = static_cast<int>(per_panel * a.panels);
+  panel_kernel<kXf, kOut, Cfg><<<grid, Cfg::kThreads, smem, st>>>(map, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KQ_OK;
+}
+
+template <int kXf, int kOut>
+int launch_panel(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q,
+                 uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev) {
+  switch (panel_variant()) {
+    case 1: return launch_panel_cfg<kXf, kOut, PanelV1>(x, M, d, aux, q, scales, y, st, di, dev);
+    case 2: return launch_panel_cfg<kXf, kOut, PanelV2>(x, M, d, aux, q, scales, y, st, di, dev);
+    default: return launch_panel_cfg<kXf, kOut, PanelV0>(x, M, d, aux, q, scales, y, st, di, dev);
+  }
+}
+
+bool panel_fits(int nb) {
+  int W = 0, R = 0;
+  switch (panel_variant()) {
+    case 1: return panel_use<PanelV1>(nb, &W, &R) >= 0.75;
+    case 2: return panel_use<PanelV2>(nb, &W, &R) >= 0.75;
+    default: return panel_use<PanelV0>(nb, &W, &R) >= 0.75;
+  }
+}
+
 template <int kXf, int kOut, bool kF32In>
 int launch_direct(const void* x, int64_t M, int64_t d, LaunchArgs a, cudaStream_t st,
                   const DeviceInfo& di, int dev) {
@@ -407,7 +751,16 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
   a.inverse = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nb = d / kBlock;
-  if (impl == KQ_IMPL_AUTO) impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
+  if (impl == KQ_IMPL_AUTO) {
+    if (nb <= 65535 && panel_fits(static_cast<int>(nb)) && M < (int64_t(1) << 30))
+      impl = KQ_IMPL_PANEL;
+    else
+      impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
+  }
+  if (impl == KQ_IMPL_PANEL) {
+    if (nb > 65535) return KQ_ERR_INVALID;
+    return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
+  }
   if (impl == KQ_IMPL_TMA) return launch_tma<kXf, kOut>(x, M, d, a, st, *di, dev);
   if (impl == KQ_IMPL_DIRECT) return launch_direct<kXf, kOut, false>(x, M, d, a, st, *di, dev);
   return KQ_ERR_INVALID;
@@ -432,7 +785,7 @@ extern "C" int kq_quantize_ex(const uint16_t* x, int64_t M, int64_t d, const flo
                               uint8_t* q_packed, uint8_t* scales, int impl, void* stream) {
   int rc = check_quant_args(x, M, d, params, true, q_packed, scales);
   if (rc != KQ_OK || M == 0) return rc;
-  if (impl < KQ_IMPL_AUTO || impl > KQ_IMPL_WARP) return KQ_ERR_INVALID;
+  if (impl < KQ_IMPL_AUTO || impl > KQ_IMPL_PANEL) return KQ_ERR_INVALID;
   return run<kXfKron, kOutMx4>(x, M, d, params, q_packed, scales, nullptr, impl, stream);
 }
 
