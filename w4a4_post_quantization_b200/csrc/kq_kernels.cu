@@ -606,21 +606,27 @@ int launch_tma(const uint16_t* x, int64_t M, int64_t d, LaunchArgs a, cudaStream
 }
 
 // Panel shape for nb blocks per row: W divides nb, R = thread rows per tile,
-// W * R <= cons, and W <= 256 and rpt * R <= 256 (TMA box dimension limit); the best thread use wins,
-// then the wider panel.  Returns the fraction of busy consumer threads.
-double panel_shape(int nb, int cons, int rpt, int* W_out, int* R_out) {
-  double best = 0.0;
+// W * R <= cons, and W <= 256 and rpt * R <= 256 (TMA box dimension limit).
+// Score: the share of busy consumer threads times the share of SMs that a
+// grid made of whole panels (nb / W CTAs each) keeps busy; the best score
+// wins, then the wider panel.  Returns the busy-thread share of the winner.
+double panel_shape(int nb, int cons, int rpt, int sms, int* W_out, int* R_out) {
+  double best = -1.0, best_use = 0.0;
   for (int W = std::min(std::min(nb, cons), 256); W >= 1; --W) {
     if (nb % W) continue;
     const int R = std::min(cons / W, 256 / rpt);
     const double use = double(W * R) / cons;
-    if (use > best + 1e-9) {
-      best = use;
+    const int panels = nb / W;
+    const double sm_use = panels >= sms ? 1.0 : double(sms / panels * panels) / sms;
+    const double score = use * sm_use;
+    if (score > best + 1e-9) {
+      best = score;
+      best_use = use;
       *W_out = W;
       *R_out = R;
     }
   }
-  return best;
+  return best_use;
 }
 
 // Panel-kernel shapes measured on B200 (interleaved medians on the
@@ -642,8 +648,8 @@ int panel_variant() {
 }
 
 template <class Cfg>
-double panel_use(int nb, int* W, int* R) {
-  return panel_shape(nb, Cfg::kCons, Cfg::kRpt, W, R);
+double panel_use(int nb, int sms, int* W, int* R) {
+  return panel_shape(nb, Cfg::kCons, Cfg::kRpt, sms * Cfg::kMinBlocks, W, R);
 }
 
 template <int kXf, int kOut, class Cfg>
@@ -652,7 +658,7 @@ int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, 
   constexpr int kRpt = Cfg::kRpt;
   const int nb = static_cast<int>(d / kBlock);
   PanelArgs a{};
-  if (panel_use<Cfg>(nb, &a.W, &a.R) < 0.5) return KQ_ERR_INVALID;
+  if (panel_use<Cfg>(nb, di.sms, &a.W, &a.R) < 0.5) return KQ_ERR_INVALID;
   a.M = M;
   a.nb = nb;
   a.panels = nb / a.W;
@@ -708,12 +714,12 @@ int launch_panel(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint
   }
 }
 
-bool panel_fits(int nb) {
+bool panel_fits(int nb, int sms) {
   int W = 0, R = 0;
   switch (panel_variant()) {
-    case 1: return panel_use<PanelV1>(nb, &W, &R) >= 0.75;
-    case 2: return panel_use<PanelV2>(nb, &W, &R) >= 0.75;
-    default: return panel_use<PanelV0>(nb, &W, &R) >= 0.75;
+    case 1: return panel_use<PanelV1>(nb, sms, &W, &R) >= 0.75;
+    case 2: return panel_use<PanelV2>(nb, sms, &W, &R) >= 0.75;
+    default: return panel_use<PanelV0>(nb, sms, &W, &R) >= 0.75;
   }
 }
 
@@ -752,7 +758,7 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nb = d / kBlock;
   if (impl == KQ_IMPL_AUTO) {
-    if (nb <= 65535 && panel_fits(static_cast<int>(nb)) && M < (int64_t(1) << 30))
+    if (nb <= 65535 && panel_fits(static_cast<int>(nb), di->sms) && M < (int64_t(1) << 30))
       impl = KQ_IMPL_PANEL;
     else
       impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
