@@ -107,6 +107,28 @@ int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* para
 int kq_dequantize(const uint8_t* q_packed, const uint8_t* scales, int64_t M, int64_t d,
                   float* y, void* stream);
 
+/* End-to-end quantization of activations in HOST memory: the same result as
+ * kq_quantize, with x_host [M][d] bf16 read from host memory and q_host
+ * [M][d/2] and scales_host [M][d/32] written to host memory.  Rows move in
+ * chunks through `workspace` (device memory the caller allocates, 256-byte
+ * aligned; two chunks live in it at a time), so that the host-to-device copy
+ * of one chunk, the quantizer on the previous one and the device-to-host copy
+ * of the one before overlap.  The host buffers should be page-locked (pinned)
+ * for the copies to overlap.  params is a device pointer.  The call is
+ * asynchronous: it returns once the work is queued, and `stream` completes
+ * when the last outputs have reached host memory; the host buffers must stay
+ * valid until then.  The library keeps two copy streams and a few events per
+ * device, created on the first call; calls for the same device are queued
+ * one at a time.  KQ_ERR_INVALID if the workspace cannot hold two chunks of
+ * one row (kq_quantize_host_workspace_bytes(d, 1)). */
+int kq_quantize_host(const uint16_t* x_host, int64_t M, int64_t d, const float* params,
+                     uint8_t* q_host, uint8_t* scales_host, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* Workspace bytes kq_quantize_host needs for chunks of rows_per_chunk rows
+ * of width d (0 for an invalid d or rows_per_chunk < 1). */
+size_t kq_quantize_host_workspace_bytes(int64_t d, int64_t rows_per_chunk);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* kq_status_string(int status);
 

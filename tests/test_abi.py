@@ -88,3 +88,16 @@ def test_missing_library_fails_loudly(tmp_path):
     from w4a4_post_quantization_b200 import _lib
     with pytest.raises(ImportError):
         _lib.load_library(str(tmp_path / "libkq.so"))
+
+
+def test_host_pipeline_argument_checks(lib):
+    need = lib.kq_quantize_host_workspace_bytes(64, 1)
+    assert need >= 2 * (64 * 2 + 32 + 2)
+    assert lib.kq_quantize_host_workspace_bytes(48, 1) == 0
+    assert lib.kq_quantize_host_workspace_bytes(64, 0) == 0
+    # too small a workspace, misaligned workspace, bad shape, null pointers
+    assert lib.kq_quantize_host(FAKE, 4, 64, FAKE, FAKE, FAKE, FAKE, need - 1, None) == 1
+    assert lib.kq_quantize_host(FAKE, 4, 64, FAKE, FAKE, FAKE, FAKE + 16, need, None) == 1
+    assert lib.kq_quantize_host(FAKE, 4, 48, FAKE, FAKE, FAKE, FAKE, need, None) == 1
+    assert lib.kq_quantize_host(None, 4, 64, FAKE, FAKE, FAKE, FAKE, need, None) == 1
+    assert lib.kq_quantize_host(FAKE, 0, 64, FAKE, FAKE, FAKE, FAKE, need, None) == 0

@@ -32,12 +32,15 @@ SIGNATURES = {
     "kq_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
+    "kq_quantize_host": [_p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p],
+    "kq_quantize_host_workspace_bytes": [_i64, _i64],
     "kq_status_string": [_int],
     "kq_last_cuda_error": [],
     "kq_device_status": [ctypes.POINTER(_int)],
     "kq_version": [],
 }
-_RESTYPE = {"kq_status_string": ctypes.c_char_p}
+_RESTYPE = {"kq_status_string": ctypes.c_char_p,
+            "kq_quantize_host_workspace_bytes": ctypes.c_size_t}
 
 
 class KQError(RuntimeError):
@@ -196,6 +199,40 @@ def dequantize(q: torch.Tensor, scales: torch.Tensor, y=None):
     st = lib().kq_dequantize(q.data_ptr(), scales.data_ptr(), M, d, y.data_ptr(), _stream(q.device))
     _check("kq_dequantize", st)
     return y
+
+
+def host_workspace_bytes(d: int, rows_per_chunk: int) -> int:
+    """Device workspace bytes quantize_host needs for chunks of that many rows."""
+    return int(lib().kq_quantize_host_workspace_bytes(d, rows_per_chunk))
+
+
+def _host_tensor(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor")
+    return t
+
+
+def quantize_host(x: torch.Tensor, params: torch.Tensor, q: torch.Tensor, scales: torch.Tensor,
+                  workspace: torch.Tensor, stream=None):
+    """MXFP4(x T) for host-resident x (pinned bf16 [M, d]) into host q / scales
+    (pinned uint8), streamed through a device ``workspace`` (uint8 CUDA
+    tensor).  Asynchronous on ``stream`` (default: the current stream of the
+    workspace's device)."""
+    _host_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    _host_tensor(q, torch.uint8, "q")
+    _host_tensor(scales, torch.uint8, "scales")
+    if tuple(q.shape) != (M, d // 2) or tuple(scales.shape) != (M, d // 32):
+        raise ValueError("output shapes must be [M, d/2] and [M, d/32]")
+    _dev_tensor(workspace, torch.uint8, "workspace")
+    _params(params, d)
+    st = stream if stream is not None else _stream(workspace.device)
+    rc = lib().kq_quantize_host(x.data_ptr(), M, d, params.data_ptr(), q.data_ptr(),
+                                scales.data_ptr(), workspace.data_ptr(), workspace.numel(), st)
+    _check("kq_quantize_host", rc)
+    return q, scales
 
 
 def device_status() -> int:

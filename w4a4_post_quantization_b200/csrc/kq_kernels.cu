@@ -24,6 +24,14 @@ namespace kq {
 
 __device__ int g_device_error = 0;
 
+thread_local int t_last_cuda_error = 0;
+
+// Remembers a failed CUDA call for kq_last_cuda_error; returns KQ_ERR_CUDA.
+int record_cuda_error(cudaError_t e) {
+  t_last_cuda_error = static_cast<int>(e);
+  return KQ_ERR_CUDA;
+}
+
 enum Xform { kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2 };
 enum Out { kOutMx4 = 0, kOutF32 = 1 };
 
@@ -489,12 +497,7 @@ __global__ void __launch_bounds__(256)
 // =================================================================== host
 namespace {
 
-thread_local int t_last_cuda_error = 0;
-
-int cuda_fail(cudaError_t e) {
-  t_last_cuda_error = static_cast<int>(e);
-  return KQ_ERR_CUDA;
-}
+int cuda_fail(cudaError_t e) { return record_cuda_error(e); }
 
 struct DeviceInfo {
   bool ready = false;
