@@ -129,6 +129,29 @@ int kq_quantize_host(const uint16_t* x_host, int64_t M, int64_t d, const float* 
  * of width d (0 for an invalid d or rows_per_chunk < 1). */
 size_t kq_quantize_host_workspace_bytes(int64_t d, int64_t rows_per_chunk);
 
+/* Size of the staging area built into the library for
+ * kq_quantize_host_static: 16 MiB of device memory. */
+#define KQ_STATIC_STAGING_BYTES (16u << 20)
+
+/* The same result as kq_quantize_host, for callers that cannot allocate
+ * device memory: a serving process whose memory pool already holds nearly
+ * all of the GPU can see cudaMalloc fail, and cudaMalloc / cudaFree may
+ * synchronise the whole device.  This call takes no workspace and allocates
+ * nothing (no cudaMalloc, no streams, no events): rows are copied in,
+ * quantized and copied out chunk by chunk, in order on `stream` alone,
+ * through a KQ_STATIC_STAGING_BYTES staging area that is part of the library
+ * itself.  Each GPU on which that area is loaded keeps it until the process
+ * exits.  The first call on a device looks up the area's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls share the one area and the last call's data stays in it: calls
+ * that overlap on the GPU (on different streams, or from several host
+ * threads) race and must be serialised by the caller.  KQ_ERR_INVALID for
+ * rows too wide for the area: 2 d + d/2 + d/32 bytes plus rounding must fit
+ * in KQ_STATIC_STAGING_BYTES (d up to about 6.6 million).  The pages have no
+ * counterpart of this entry point. */
+int kq_quantize_host_static(const uint16_t* x_host, int64_t M, int64_t d, const float* params,
+                            uint8_t* q_host, uint8_t* scales_host, void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* kq_status_string(int status);
 

@@ -34,6 +34,7 @@ SIGNATURES = {
     "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
     "kq_quantize_host": [_p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p],
     "kq_quantize_host_workspace_bytes": [_i64, _i64],
+    "kq_quantize_host_static": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_status_string": [_int],
     "kq_last_cuda_error": [],
     "kq_device_status": [ctypes.POINTER(_int)],
@@ -232,6 +233,26 @@ def quantize_host(x: torch.Tensor, params: torch.Tensor, q: torch.Tensor, scales
     rc = lib().kq_quantize_host(x.data_ptr(), M, d, params.data_ptr(), q.data_ptr(),
                                 scales.data_ptr(), workspace.data_ptr(), workspace.numel(), st)
     _check("kq_quantize_host", rc)
+    return q, scales
+
+
+def quantize_host_static(x: torch.Tensor, params: torch.Tensor, q: torch.Tensor,
+                         scales: torch.Tensor, stream=None):
+    """quantize_host without a workspace, for callers that cannot allocate
+    device memory: the rows pass through a 16 MiB staging area built into the
+    library.  Calls that overlap on the GPU share that area and must be
+    serialised.  Runs on ``stream`` (default: the current CUDA stream)."""
+    _host_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    _host_tensor(q, torch.uint8, "q")
+    _host_tensor(scales, torch.uint8, "scales")
+    if tuple(q.shape) != (M, d // 2) or tuple(scales.shape) != (M, d // 32):
+        raise ValueError("output shapes must be [M, d/2] and [M, d/32]")
+    _params(params, d)
+    st = stream if stream is not None else _stream(params.device)
+    rc = lib().kq_quantize_host_static(x.data_ptr(), M, d, params.data_ptr(), q.data_ptr(),
+                                       scales.data_ptr(), st)
+    _check("kq_quantize_host_static", rc)
     return q, scales
 
 
