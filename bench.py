@@ -21,6 +21,7 @@ import hashlib
 import json
 import multiprocessing as mp
 import os
+import re
 import statistics
 import sys
 import threading
@@ -76,14 +77,21 @@ def measured_peak():
 KERNEL_SOURCES = ("kq_kernels.cu", "kq_device.cuh")
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and whitespace."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return re.sub(r"\s+", "", text)
+
+
 def kernel_source_hash() -> str:
-    """Hash of the sources that define the timed kernel (a committed ncu
-    traffic figure is reported only while they are unchanged)."""
+    """Hash of the code (comments and whitespace aside) that defines the timed
+    kernel: a committed ncu traffic figure is reported only while it holds."""
     h = hashlib.sha256()
     src = os.path.join(ROOT, "w4a4_post_quantization_b200", "csrc")
     for f in KERNEL_SOURCES:
-        with open(os.path.join(src, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(src, f)) as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

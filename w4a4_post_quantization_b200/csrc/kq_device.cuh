@@ -430,7 +430,8 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// Largest magnitude of the 32 values: a tree of three-input maxima.
+// Largest magnitude of the 32 values: a tree of three-input maxima (fewer
+// instructions on B200 than two-input maxima with folded |.|, measured).
 __device__ __forceinline__ float block_amax(const f2 (&u)[16]) {
   float a[32];
 #pragma unroll

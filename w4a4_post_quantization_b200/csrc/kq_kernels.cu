@@ -635,7 +635,7 @@ double panel_shape(int nb, int cons, int rpt, int sms, int* W_out, int* R_out) {
 // Panel-kernel shapes measured on B200 (interleaved medians on the
 // 16384 x 12288 stress input, GB/s): 12 consumer warps x 2 rows 5526,
 // 15 x 2 5405, 14 x 2 4971, 8 x 2 4972, 15 x 1 5441, 16 x 1 with the diagonal
-// in shared memory 4978.  More warps hide latency until the register budget
+// in shared memory 4978, 8 x 3 4740, 10 x 3 4601.  More warps hide latency until the register budget
 // (ceil(warps / 4) warps share one scheduler's 16K registers) forces spills.
 using PanelV0 = PanelCfg<12, 2, 1>;
 using PanelV1 = PanelCfg<8, 2, 1>;
