@@ -109,7 +109,8 @@ def test_full_size_sampled_rows(key):
     _requantize_is_identity(out["q"], out["s"], c.M, c.d)
 
 
-IMPLS = {"panel": kq.KQ_IMPL_PANEL, "tma": kq.KQ_IMPL_TMA, "direct": kq.KQ_IMPL_DIRECT}
+IMPLS = {"panel": kq.KQ_IMPL_PANEL, "tma": kq.KQ_IMPL_TMA, "direct": kq.KQ_IMPL_DIRECT,
+         "mma": kq.KQ_IMPL_MMA}
 
 
 @pytest.mark.parametrize("impl", sorted(IMPLS))
@@ -122,6 +123,20 @@ def test_each_implementation_against_oracle(impl, key):
     x64 = o.bf16_bits_to_float64(c.x_bits())
     check_mx4(q.cpu().numpy(), s.cpu().numpy(), o.transform(x64, c.params),
               o.abs_transform(x64, c.params))
+
+
+@pytest.mark.parametrize("key", w.all_case_keys(), ids=lambda k: f"{k[0]}-d{k[1]}-g{k[2]}")
+def test_tensor_core_transform_all_configs(key):
+    """The tcgen05 path (dense K as three bf16 terms) on every config, with a
+    ragged last 128-row tile."""
+    name, di, gi = key
+    c = w.make_case(name, di, gi, M=200 if name != "tiny" else 256)
+    q, s = kq.quantize(_gpu(c.x), _params_dev(c.params), impl=kq.KQ_IMPL_MMA)
+    x64 = o.bf16_bits_to_float64(c.x_bits())
+    st = check_mx4(q.cpu().numpy(), s.cpu().numpy(), o.transform(x64, c.params),
+                   o.abs_transform(x64, c.params))
+    assert st["scale_exempt"] <= max(2, st["blocks"] // 1000)
+    assert st["code_exempt"] <= max(4, st["elements"] // 10000)
 
 
 def test_table_implementations_agree_bitwise():

@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkq.so")
 
 KQ_OK, KQ_ERR_INVALID, KQ_ERR_CUDA, KQ_ERR_DEVICE, KQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
-KQ_IMPL_AUTO, KQ_IMPL_TMA, KQ_IMPL_DIRECT, KQ_IMPL_WARP, KQ_IMPL_PANEL = 0, 1, 2, 3, 4
+KQ_IMPL_AUTO, KQ_IMPL_TMA, KQ_IMPL_DIRECT, KQ_IMPL_WARP, KQ_IMPL_PANEL, KQ_IMPL_MMA = 0, 1, 2, 3, 4, 5
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64

@@ -1,0 +1,56 @@
+// Host-side helpers shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "kq.h"
+
+namespace kq {
+
+constexpr int kMaxDevices = 64;
+
+// Remembers a failed CUDA call for kq_last_cuda_error; returns KQ_ERR_CUDA.
+int record_cuda_error(cudaError_t e);
+
+struct DeviceInfo {
+  bool ready = false;
+  int status = KQ_OK;
+  int sms = 0;
+  int smem_optin = 0;
+  int smem_per_sm = 0;
+};
+
+// Properties of the current device (cached) and its index; KQ_ERR_DEVICE if
+// it is not an sm_100 part.
+int device_info(const DeviceInfo** out, int* dev_out);
+
+// The driver's cuTensorMapEncodeTiled (valid after a successful device_info).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// Device address of the library's device-side error word on device `dev`.
+int device_error_word(int dev, int** out);
+
+// Sets the dynamic shared-memory limit of one kernel once per device.
+template <auto kKernel>
+int allow_smem(int bytes, int dev) {
+  static std::mutex mu;
+  static int done[kMaxDevices] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (done[dev] < bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    done[dev] = bytes;
+  }
+  return KQ_OK;
+}
+
+// Launchers defined in other translation units.
+int launch_mma_kron(const uint16_t* x, int64_t M, int64_t d, const float* params, uint8_t* q,
+                    uint8_t* scales, float* y, cudaStream_t st);
+
+}  // namespace kq

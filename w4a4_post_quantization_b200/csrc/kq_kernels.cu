@@ -19,6 +19,7 @@
 
 #include "kq.h"
 #include "kq_device.cuh"
+#include "kq_internal.h"
 
 namespace kq {
 
@@ -495,34 +496,22 @@ __global__ void __launch_bounds__(256)
 }
 
 // =================================================================== host
-namespace {
-
-int cuda_fail(cudaError_t e) { return record_cuda_error(e); }
-
-struct DeviceInfo {
-  bool ready = false;
-  int status = KQ_OK;
-  int sms = 0;
-  int smem_optin = 0;
-  int smem_per_sm = 0;
-};
-
-constexpr int kMaxDevices = 64;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::mutex g_mu;
 DeviceInfo g_dev[kMaxDevices];
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+int* g_error_word[kMaxDevices] = {};
 
 int device_info(const DeviceInfo** out, int* dev_out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e);
+  if (e != cudaSuccess) return record_cuda_error(e);
   if (dev < 0 || dev >= kMaxDevices) return KQ_ERR_DEVICE;
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceInfo& di = g_dev[dev];
   if (!di.ready) {
     cudaDeviceProp prop;
     e = cudaGetDeviceProperties(&prop, dev);
-    if (e != cudaSuccess) return cuda_fail(e);
+    if (e != cudaSuccess) return record_cuda_error(e);
     di.status = prop.major == 10 ? KQ_OK : KQ_ERR_DEVICE;
     di.sms = prop.multiProcessorCount;
     di.smem_optin = static_cast<int>(prop.sharedMemPerBlockOptin);
@@ -533,7 +522,7 @@ int device_info(const DeviceInfo** out, int* dev_out) {
       e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
                                            &qr);
       if (e != cudaSuccess || qr != cudaDriverEntryPointSuccess || !fn)
-        return cuda_fail(e != cudaSuccess ? e : cudaErrorNotSupported);
+        return record_cuda_error(e != cudaSuccess ? e : cudaErrorNotSupported);
       g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
     di.ready = true;
@@ -543,25 +532,29 @@ int device_info(const DeviceInfo** out, int* dev_out) {
   return di.status;
 }
 
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() { return g_encode; }
+
+int device_error_word(int dev, int** out) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_error_word[dev]) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_device_error);
+    if (e != cudaSuccess) return record_cuda_error(e);
+    g_error_word[dev] = static_cast<int*>(p);
+  }
+  *out = g_error_word[dev];
+  return KQ_OK;
+}
+
+namespace {
+
+int cuda_fail(cudaError_t e) { return record_cuda_error(e); }
+
 bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
 
 int check_shape(int64_t M, int64_t d) {
   if (M < 0 || d < kBlock || d % kBlock != 0) return KQ_ERR_INVALID;
   if (M > 0 && d > (int64_t(1) << 40) / M) return KQ_ERR_INVALID;
-  return KQ_OK;
-}
-
-// Sets the dynamic shared-memory limit of one kernel once per device.
-template <auto kKernel>
-int allow_smem(int bytes, int dev) {
-  static std::mutex mu;
-  static int done[kMaxDevices] = {0};
-  std::lock_guard<std::mutex> lock(mu);
-  if (done[dev] < bytes) {
-    cudaError_t e = cudaFuncSetAttribute(kKernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return cuda_fail(e);
-    done[dev] = bytes;
-  }
   return KQ_OK;
 }
 
@@ -766,6 +759,11 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
     else
       impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
   }
+  if (impl == KQ_IMPL_MMA) {
+    if (kXf != kXfKron) return KQ_ERR_INVALID;
+    return launch_mma_kron(x, M, d, aux, kOut == kOutMx4 ? q : nullptr,
+                           kOut == kOutMx4 ? scales : nullptr, kOut == kOutF32 ? y : nullptr, st);
+  }
   if (impl == KQ_IMPL_PANEL) {
     if (nb > 65535) return KQ_ERR_INVALID;
     return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
@@ -794,7 +792,7 @@ extern "C" int kq_quantize_ex(const uint16_t* x, int64_t M, int64_t d, const flo
                               uint8_t* q_packed, uint8_t* scales, int impl, void* stream) {
   int rc = check_quant_args(x, M, d, params, true, q_packed, scales);
   if (rc != KQ_OK || M == 0) return rc;
-  if (impl < KQ_IMPL_AUTO || impl > KQ_IMPL_PANEL) return KQ_ERR_INVALID;
+  if (impl < KQ_IMPL_AUTO || impl > KQ_IMPL_MMA) return KQ_ERR_INVALID;
   return run<kXfKron, kOutMx4>(x, M, d, params, q_packed, scales, nullptr, impl, stream);
 }
 
