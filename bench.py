@@ -326,6 +326,9 @@ def run_gpu(args):
     if args.op == "kron":
         def step():
             kq.quantize(x, params, q, s)
+    elif args.op == "kron_mma":
+        def step():
+            kq.quantize(x, params, q, s, impl=kq.KQ_IMPL_MMA)
     elif args.op == "hadamard":
         def step():
             kq.quantize_hadamard(x, q, s)
@@ -339,8 +342,23 @@ def run_gpu(args):
         step()
         torch.cuda.synchronize()
     sampler = ClockSampler(local)
-    ms, clocks = time_steps(step, args.steps, args.warmup, stream, sampler)
+    eager_ms, eager_clocks = time_steps(step, args.steps, args.warmup, stream,
+                                        None if args.launch == "graph" else sampler)
+    if args.launch == "graph":
+        # The K timed steps captured once into a CUDA graph and replayed once:
+        # the same K kernel launches without the host's per-launch cost.
+        graph, gstream = torch.cuda.CUDAGraph(), torch.cuda.Stream(dev)
+        gstream.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=gstream):
+            for _ in range(args.steps):
+                step()
+        torch.cuda.synchronize()
+        ms, clocks = time_steps(graph.replay, 1, max(args.warmup // args.steps, 3), stream, sampler)
+        ms /= args.steps
+    else:
+        ms, clocks = eager_ms, eager_clocks
     ms_max = max_over_ranks(ms, dev)
+    eager_max = max_over_ranks(eager_ms, dev)
     value = aggregate_gbs(alg_bytes, world, args.steps, ms_max * args.steps)
 
     # Comparators and the copy ceiling on the same input (context, same GPU).
@@ -356,11 +374,12 @@ def run_gpu(args):
         ms_max_c = max_over_ranks(ms_c, dev)
         impls = {}
         for name, code in (("panel", kq.KQ_IMPL_PANEL), ("tma_flat", kq.KQ_IMPL_TMA),
-                           ("direct", kq.KQ_IMPL_DIRECT)):
+                           ("direct", kq.KQ_IMPL_DIRECT), ("tcgen05_dense_k", kq.KQ_IMPL_MMA)):
             ms_i, _ = time_steps(lambda: kq.quantize(x, params, q, s, impl=code), args.steps,
                                  args.warmup, stream)
             impls[name] = alg_bytes / (max_over_ranks(ms_i, dev) * 1e-3) / 1e9
         variants = {
+            "eager_gbs": aggregate_gbs(alg_bytes, world, 1, eager_max),
             "kq_quantize_impl_gbs": impls,
             "hadamard": {"gbs": alg_bytes / (ms_max_h * 1e-3) / 1e9, "ms": ms_max_h},
             "smooth": {"gbs": alg_bytes / (ms_max_s * 1e-3) / 1e9, "ms": ms_max_s},
@@ -426,7 +445,9 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": dict(_config(d, M, "panel"), op=args.op, global_batch_rows=M * world,
+            "config": dict(_config(d, M, "panel"), op=args.op,
+                           launch=("cuda_graph: the K steps captured once, replayed once"
+                                   if args.launch == "graph" else "eager: one call per step"), global_batch_rows=M * world,
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3),
             "hbm_frac": value / world / peak,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
@@ -447,7 +468,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the comparator timings")
-    ap.add_argument("--op", default="kron", choices=["kron", "hadamard", "smooth"],
+    ap.add_argument("--launch", default="eager", choices=["graph", "eager"],
+                    help="time the K steps as K calls (default) or as one CUDA graph replay")
+    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "hadamard", "smooth"],
                     help="quantizer timed as the step (kron = kq_quantize, the metric; "
                          "the comparators are for profiling)")
     ap.add_argument("--rows", type=int, default=0,
