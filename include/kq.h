@@ -165,6 +165,17 @@ int kq_last_cuda_error(void);
  * early and leave their outputs incomplete).  Returns KQ_OK or KQ_ERR_CUDA. */
 int kq_device_status(int* flags);
 
+/* Device-side error word bits (kq_device_status). */
+#define KQ_DEVERR_CONSUMER_WAIT 1  /* a consumer gave up waiting for its data */
+#define KQ_DEVERR_PRODUCER_WAIT 2  /* a producer gave up waiting for a free stage */
+#define KQ_DEVERR_SELFTEST 4       /* set by kq_selftest_wait_timeout */
+
+/* Self-test of the bounded waits: launches one tiny kernel that waits (at
+ * most 64 polls of about 1 us) on a barrier nothing completes, gives up and
+ * sets KQ_DEVERR_SELFTEST in the device error word, which kq_device_status
+ * then reports and clears.  The device stays usable afterwards. */
+int kq_selftest_wait_timeout(void* stream);
+
 /* ABI version, (major << 16) | minor. */
 int kq_version(void);
 

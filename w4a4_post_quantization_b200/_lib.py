@@ -39,6 +39,7 @@ SIGNATURES = {
     "kq_last_cuda_error": [],
     "kq_device_status": [ctypes.POINTER(_int)],
     "kq_version": [],
+    "kq_selftest_wait_timeout": [_p],
 }
 _RESTYPE = {"kq_status_string": ctypes.c_char_p,
             "kq_quantize_host_workspace_bytes": ctypes.c_size_t}

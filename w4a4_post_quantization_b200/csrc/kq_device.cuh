@@ -20,6 +20,7 @@ constexpr int kTabStride = 44;       // floats per block in a Kronecker coeffici
 // Bits of the device error word (kq_device_status).
 constexpr int kErrConsumerWait = 1;
 constexpr int kErrProducerWait = 2;
+constexpr int kErrSelfTest = 4;
 
 // A bounded mbarrier wait polls at most kWaitPolls times, each poll suspending
 // for at most kWaitHintNs: about four seconds in all, far above any real wait.

@@ -465,6 +465,35 @@ __global__ void __launch_bounds__(kDirectThreads)
   }
 }
 
+// ------------------------------------------------------ wait self-test
+// Waits on an mbarrier that nothing ever completes, with a short bound, and
+// reports the expiry through the device error word: the same give-up path
+// every pipeline wait takes, exercised without any fault.
+__global__ void wait_selftest_kernel(int polls) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t addr = smem_addr(&bar);
+    bool done = false;
+    for (int i = 0; i < polls && !done; ++i) {
+      uint32_t d;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(d)
+          : "r"(addr), "r"(0u), "r"(1000u)
+          : "memory");
+      done = d != 0;
+    }
+    if (!done) atomicOr(&g_device_error, kErrSelfTest);
+  }
+}
+
 // ------------------------------------------------------- dequantize kernel
 __global__ void __launch_bounds__(256)
     dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, int64_t G,
@@ -857,6 +886,17 @@ extern "C" int kq_dequantize(const uint8_t* q_packed, const uint8_t* scales, int
   const int64_t want = (G + 255) / 256;
   const int grid = static_cast<int>(std::min<int64_t>(want, (int64_t)di->sms * 8));
   dequant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(q_packed, scales, G, y);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return KQ_OK;
+}
+
+extern "C" int kq_selftest_wait_timeout(void* stream) {
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(64);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return KQ_OK;
