@@ -68,9 +68,10 @@ def lu_factor(a: float, b: float, c: float) -> np.ndarray:
 
 
 def block_factors(p_j: np.ndarray) -> list:
-    """The five 2x2 factors of one block from its ``[5, 3]`` parameters."""
+    """The 2x2 factors of one block from its ``[n, 3]`` parameters (n = 5 for
+    32-element blocks, 4 for the 16-element variant)."""
     p_j = np.asarray(p_j, dtype=np.float64)
-    return [lu_factor(*p_j[k]) for k in range(N_FACTORS)]
+    return [lu_factor(*p_j[k]) for k in range(p_j.shape[0])]
 
 
 def kron_factors(factors) -> np.ndarray:
@@ -83,7 +84,8 @@ def kron_factors(factors) -> np.ndarray:
 
 
 def kron_block(p_j: np.ndarray) -> np.ndarray:
-    """Dense 32x32 ``K^(j) = G1 (x) G2 (x) G3 (x) G4 (x) G5``."""
+    """Dense ``K^(j) = G1 (x) G2 (x) ...``: 32x32 from five factors, 16x16
+    from four."""
     return kron_factors(block_factors(p_j))
 
 
@@ -104,12 +106,12 @@ def hadamard_block() -> np.ndarray:
     return scipy.linalg.hadamard(BLOCK).astype(np.float64) / math.sqrt(BLOCK)
 
 
-def _apply_blocks(x64: np.ndarray, blocks) -> np.ndarray:
+def _apply_blocks(x64: np.ndarray, blocks, block: int = BLOCK) -> np.ndarray:
     x64 = np.asarray(x64, dtype=np.float64)
     M, d = x64.shape
     y = np.empty_like(x64)
-    for j in range(d // BLOCK):
-        sl = slice(BLOCK * j, BLOCK * (j + 1))
+    for j in range(d // block):
+        sl = slice(block * j, block * (j + 1))
         y[:, sl] = x64[:, sl] @ blocks(j)
     return y
 
@@ -194,15 +196,16 @@ def e2m1_decode(code: np.ndarray) -> np.ndarray:
     return np.where(s == 1, -mag, mag)
 
 
-def mxfp4_quantize(y64: np.ndarray):
-    """Quantize ``[M, d]`` values block by block.
+def mxfp4_quantize(y64: np.ndarray, block: int = BLOCK):
+    """Quantize ``[M, d]`` values block by block (``block`` elements share
+    one scale: 32 for MXFP4, 16 for the 16-element variant).
 
-    Returns ``(codes [M, d] uint8 (unpacked), scale bytes [M, d/32] uint8)``.
+    Returns ``(codes [M, d] uint8 (unpacked), scale bytes [M, d/block] uint8)``.
     """
     yq = decision_values(y64)
     M, d = yq.shape
-    nb = d // BLOCK
-    blocks = yq.reshape(M, nb, BLOCK)
+    nb = d // block
+    blocks = yq.reshape(M, nb, block)
     amax = np.abs(blocks).max(axis=2)
     e = e8m0_exponent(amax)
     v = blocks * np.ldexp(1.0, -e)[:, :, None]        # exact: power-of-two scaling
@@ -231,11 +234,11 @@ def e8m0_decode(scale: np.ndarray) -> np.ndarray:
     return np.where(s == 255, np.nan, val)
 
 
-def dequantize(q_packed: np.ndarray, scales: np.ndarray) -> np.ndarray:
+def dequantize(q_packed: np.ndarray, scales: np.ndarray, block: int = BLOCK) -> np.ndarray:
     """Exact float64 value of packed codes times their block scales."""
     codes = unpack_codes(q_packed)
     M, d = codes.shape
-    vals = e2m1_decode(codes).reshape(M, d // BLOCK, BLOCK)
+    vals = e2m1_decode(codes).reshape(M, d // block, block)
     return (vals * e8m0_decode(scales)[:, :, None]).reshape(M, d)
 
 
@@ -255,6 +258,32 @@ def quantize_hadamard(x_bits: np.ndarray):
 
 def quantize_smooth(x_bits: np.ndarray, inv_s: np.ndarray):
     codes, scales = mxfp4_quantize(transform_smooth(bf16_bits_to_float64(x_bits), inv_s))
+    return pack_codes(codes), scales
+
+
+# --------------------------------------------------------------------------
+# The 16-element variant: four factors per block, one scale per 16 elements
+# (the review's "Where Pith is reading between the lines": other blockwise
+# formats by changing the number of Kronecker factors).
+# --------------------------------------------------------------------------
+BLOCK16 = 16
+N_FACTORS16 = 4
+
+
+def transform16(x64: np.ndarray, params16: np.ndarray) -> np.ndarray:
+    """``y = x T`` with 16x16 blocks ``G1 (x) G2 (x) G3 (x) G4``."""
+    params16 = np.asarray(params16)
+    return _apply_blocks(x64, lambda j: kron_block(params16[j]), BLOCK16)
+
+
+def abs_transform16(x64: np.ndarray, params16: np.ndarray) -> np.ndarray:
+    params16 = np.asarray(params16)
+    return _apply_blocks(np.abs(x64), lambda j: np.abs(kron_block(params16[j])), BLOCK16)
+
+
+def quantize16(x_bits: np.ndarray, params16: np.ndarray):
+    """bf16 bits ``[M, d]`` -> (packed codes ``[M, d/2]``, scales ``[M, d/16]``)."""
+    codes, scales = mxfp4_quantize(transform16(bf16_bits_to_float64(x_bits), params16), BLOCK16)
     return pack_codes(codes), scales
 
 

@@ -333,3 +333,66 @@ def test_workload_generator_prefix_property():
     b = w.make_case("sana", 1, M=2100)
     assert np.array_equal(a.x_bits(), b.x_bits()[:1500])
     assert np.array_equal(a.params, b.params)
+
+
+# ------------------------------------------------- 16-element variant
+def test_block16_index_formula_det_and_inverse():
+    p = w.draw_params16(48, 21)
+    assert p.shape == (3, 4, 3)
+    for j in range(3):
+        K = o.kron_block(p[j])
+        assert K.shape == (16, 16)
+        G = o.block_factors(p[j])
+        ref = np.ones((16, 16))
+        for r in range(16):
+            for c in range(16):
+                for k in range(4):
+                    sh = 3 - k
+                    ref[r, c] *= G[k][(r >> sh) & 1, (c >> sh) & 1]
+        np.testing.assert_allclose(K, ref, rtol=1e-13, atol=1e-15)
+        assert np.linalg.det(K) == pytest.approx(1.0, rel=1e-10)
+        np.testing.assert_allclose(K @ o.inverse_block(p[j]), np.eye(16), atol=1e-11)
+
+
+def test_block16_hadamard_init_and_factorwise_transform():
+    s = 1 / math.sqrt(2)
+    G = np.array([[1, 0], [1, 1]]) @ np.array([[s, s], [0, -1 / s]])
+    np.testing.assert_allclose(o.kron_factors([G] * 4), scipy.linalg.hadamard(16) / 4, atol=1e-15)
+    rng = np.random.default_rng(22)
+    p = w.draw_params16(64, 23)
+    x = rng.standard_normal((5, 64))
+    y = o.transform16(x, p)
+    for j in range(4):
+        t = x[:, 16 * j:16 * (j + 1)].reshape(5, 2, 2, 2, 2)
+        for k, Gk in enumerate(o.block_factors(p[j])):
+            t = np.moveaxis(np.tensordot(t, Gk, axes=([k + 1], [0])), -1, k + 1)
+        np.testing.assert_allclose(y[:, 16 * j:16 * (j + 1)], t.reshape(5, 16), rtol=1e-12,
+                                   atol=1e-12)
+
+
+def test_block16_scale_per_16_elements():
+    """Each 16 elements get their own exponent: 2^k fills give k - 2 + 127,
+    and the two halves of a 32-element span are scaled independently."""
+    y = np.concatenate([np.full(16, 8.0), np.full(16, 0.5)])[None, :]
+    codes, s = o.mxfp4_quantize(y, 16)
+    assert list(s[0]) == [3 - 2 + 127, -1 - 2 + 127] and (codes == 6).all()
+    codes32, s32 = o.mxfp4_quantize(y)
+    # one 32-wide scale (exponent 1): 0.5 / 2 = 0.25 is a tie that rounds to 0
+    assert s32[0, 0] == 128 and codes[0, 16] == 6 and codes32[0, 16] == 0
+
+
+def test_block16_parameter_count_is_3_log2_n():
+    with open(os.path.join(GOLDEN, "param_counts.json")) as f:
+        g = json.load(f)
+    assert o.N_FACTORS16 * 3 == 3 * int(math.log2(16))
+    assert g["params_per_block"] == 3 * int(math.log2(32))
+
+
+def test_quantize16_identity_factors_use_16_element_scales():
+    vals = np.concatenate([np.full(16, 8.0), np.full(16, 0.5)]).astype(np.float32)
+    x = ((vals.view(np.uint32) >> 16).astype(np.uint16))[None, :]
+    p = np.zeros((2, 4, 3), dtype=np.float32)
+    p[:, :, 1] = 1.0                                     # a = c = 0, b = 1: G = I
+    q, s = o.quantize16(x, p)
+    assert list(s[0]) == [128, 124]                      # exponents 1 and -3
+    assert (o.unpack_codes(q)[0] == 6).all()             # 8/2 = 4 and 0.5*8 = 4

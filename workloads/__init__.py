@@ -115,6 +115,17 @@ def draw_params(d: int, seed: int) -> np.ndarray:
     return np.stack([a, b, c], axis=-1).astype(np.float32)
 
 
+def draw_params16(d: int, seed: int) -> np.ndarray:
+    """Parameters of the 16-element-block variant: ``[d/16, 4, 3]`` float32,
+    same distribution as ``draw_params``, from the stream ``[seed, 3]``."""
+    rng = np.random.default_rng([seed, 3])
+    nb = d // 16
+    a = rng.uniform(-1.0, 1.0, (nb, 4))
+    b = 2.0 ** rng.uniform(-1.0, 1.0, (nb, 4))
+    c = rng.uniform(-1.0, 1.0, (nb, 4))
+    return np.stack([a, b, c], axis=-1).astype(np.float32)
+
+
 def synth_inv_s(x: torch.Tensor) -> np.ndarray:
     """Reciprocal SmoothQuant channel scale for migration strength 0.5 and a
     unit weight range, from the column maxima of ``x`` (bf16 [M, d])."""
@@ -208,5 +219,5 @@ def algorithmic_bytes(M: int, d: int) -> float:
 
 
 __all__ = ["CONFIGS", "Case", "make_case", "case_seed", "all_case_keys", "random_bf16",
-           "bf16_from_float", "device_randn_bf16", "draw_params", "channel_gain", "synth_inv_s", "algorithmic_bytes",
+           "bf16_from_float", "device_randn_bf16", "draw_params", "draw_params16", "channel_gain", "synth_inv_s", "algorithmic_bytes",
            "ROW_CHUNK", "BLOCK"]
