@@ -322,6 +322,12 @@ def run_gpu(args):
     s = torch.empty((M, d // 32), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     alg_bytes = w.algorithmic_bytes(M, d)
+    # 16-element variant: [d/16, 4, 3] parameters, one scale byte per 16.
+    p16 = torch.from_numpy(w.draw_params16(d, case.seed)).to(dev)
+    s16 = torch.empty((M, d // 16), dtype=torch.uint8, device=dev)
+    bytes16 = M * d * (2.0 + 0.5 + 1.0 / 16)
+    if args.op == "kron16":
+        alg_bytes = bytes16
 
     if args.op == "kron":
         def step():
@@ -329,6 +335,9 @@ def run_gpu(args):
     elif args.op == "kron_mma":
         def step():
             kq.quantize(x, params, q, s, impl=kq.KQ_IMPL_MMA)
+    elif args.op == "kron16":
+        def step():
+            kq.quantize16(x, p16, q, s16)
     elif args.op == "hadamard":
         def step():
             kq.quantize_hadamard(x, q, s)
@@ -369,6 +378,9 @@ def run_gpu(args):
                              stream)
         ms_max_h = max_over_ranks(ms_h, dev)
         ms_max_s = max_over_ranks(ms_s, dev)
+        ms_16, _ = time_steps(lambda: kq.quantize16(x, p16, q, s16), args.steps, args.warmup,
+                              stream)
+        ms_max_16 = max_over_ranks(ms_16, dev)
         buf = torch.empty_like(x)
         ms_c, _ = time_steps(lambda: buf.copy_(x), args.steps, args.warmup, stream)
         ms_max_c = max_over_ranks(ms_c, dev)
@@ -383,6 +395,8 @@ def run_gpu(args):
             "kq_quantize_impl_gbs": impls,
             "hadamard": {"gbs": alg_bytes / (ms_max_h * 1e-3) / 1e9, "ms": ms_max_h},
             "smooth": {"gbs": alg_bytes / (ms_max_s * 1e-3) / 1e9, "ms": ms_max_s},
+            "block16": {"gbs": bytes16 / (ms_max_16 * 1e-3) / 1e9, "ms": ms_max_16,
+                        "bytes_per_launch": bytes16},
             "kronecker_over_smooth_speed": ms_max_s / ms_max,
             "d2d_copy_gbs": 2 * x.numel() * 2 / (ms_max_c * 1e-3) / 1e9,
         }
@@ -422,8 +436,12 @@ def run_gpu(args):
     khash = kernel_source_hash()
     roof = {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
             "frac": per_launch_gbs / peak, "peak_source": peak_src,
-            "traffic": profiled_traffic(khash, "kq_quantize_stress_traffic.md"),
-            "algorithmic_bytes_per_launch": alg_bytes, "kernel": "panel_kernel<kron, mx4, 2>",
+            "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.md")
+                        if args.op == "kron" else None),
+            "algorithmic_bytes_per_launch": alg_bytes,
+            "kernel": {"kron": "panel_kernel<kron, mx4>", "kron16": "panel_kernel<kron16, mx4>",
+                       "kron_mma": "mma_kernel", "hadamard": "panel_kernel<hadamard, mx4>",
+                       "smooth": "panel_kernel<smooth, mx4>"}[args.op],
             "kernel_source_hash": khash}
 
     cpu = None
@@ -470,7 +488,7 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the comparator timings")
     ap.add_argument("--launch", default="eager", choices=["graph", "eager"],
                     help="time the K steps as K calls (default) or as one CUDA graph replay")
-    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "hadamard", "smooth"],
+    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "kron16", "hadamard", "smooth"],
                     help="quantizer timed as the step (kron = kq_quantize, the metric; "
                          "the comparators are for profiling)")
     ap.add_argument("--rows", type=int, default=0,

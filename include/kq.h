@@ -98,6 +98,25 @@ int kq_quantize_smooth(const uint16_t* x, int64_t M, int64_t d, const float* inv
 int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float* params,
                  float* y, void* stream);
 
+/* 16-element variant (KroQuant review, "Where Pith is reading between the
+ * lines": other block formats by changing the number of Kronecker factors):
+ * every 16-channel block j of x is multiplied on the right by
+ * K16^(j) = G1 (x) G2 (x) G3 (x) G4 (G1 on bit 3 of the 4-bit in-block
+ * index, each G_k of the same unit-determinant LU form as above), and each
+ * transformed 16-block gets its own E8M0 scale (the same floor rule, amax over
+ * 16 elements) and 16 E2M1 codes.
+ *   params16: [d/16][4][3] float32, (a, b, c) per factor, 4-byte aligned.
+ *   q_packed: [M][d/2] bytes as for kq_quantize (element 2i low nibble).
+ *   scales16: [M][d/16] bytes, 2-byte aligned.
+ * d must be a positive multiple of 32 and at most 32 * 65535; M at most
+ * 2^31 - 1024.  Other conventions as above. */
+int kq_quantize16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
+                  uint8_t* q_packed, uint8_t* scales16, void* stream);
+
+/* y = x T16 in float32 (the kq_quantize16 transform without quantization). */
+int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
+                   float* y, void* stream);
+
 /* x = y T^-1 in float32 with T^-1 = diag(G1^-1 (x) ... (x) G5^-1) (review,
  * axiom ledger: the inverse of a Kronecker product factorizes). */
 int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,

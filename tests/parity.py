@@ -54,20 +54,22 @@ def check_transform(y_gpu: np.ndarray, y64: np.ndarray, cond: np.ndarray, tol: f
     return float(r.max()) if r.size else 0.0
 
 
-def check_mx4(q_gpu, s_gpu, y64, cond, tol: float = TOL, strict_zero_sign: bool = False):
+def check_mx4(q_gpu, s_gpu, y64, cond, tol: float = TOL, strict_zero_sign: bool = False,
+              block: int = 32):
     """Check packed codes and scale bytes against the oracle's quantization of
-    ``y64`` (decided in float32).  Returns exemption counts."""
+    ``y64`` (decided in float32), one scale per ``block`` elements.  Returns
+    exemption counts."""
     y64 = np.asarray(y64, dtype=np.float64)
     M, d = y64.shape
-    nb = d // 32
+    nb = d // block
     s_gpu = np.asarray(s_gpu, dtype=np.uint8).reshape(M, nb)
     c_gpu = unpack(q_gpu).reshape(M, d)
-    codes_ref, s_ref = o.mxfp4_quantize(y64)
+    codes_ref, s_ref = o.mxfp4_quantize(y64, block)
 
     yq = o.decision_values(y64)
     band = tol * np.asarray(cond, dtype=np.float64)
-    blk = np.abs(yq).reshape(M, nb, 32)
-    bblk = band.reshape(M, nb, 32)
+    blk = np.abs(yq).reshape(M, nb, block)
+    bblk = band.reshape(M, nb, block)
     amax_lo = np.maximum(blk - bblk, 0).max(axis=2)
     amax_hi = (blk + bblk).max(axis=2)
     e_lo = o.e8m0_exponent(amax_lo) + 127
@@ -81,7 +83,7 @@ def check_mx4(q_gpu, s_gpu, y64, cond, tol: float = TOL, strict_zero_sign: bool 
             f"{[(tuple(i), int(s_gpu[tuple(i)]), int(s_ref[tuple(i)])) for i in idx]}")
 
     # Codes under the scale the GPU chose (one of the allowed ones).
-    X = np.repeat(np.ldexp(1.0, s_int - 127), 32, axis=1)
+    X = np.repeat(np.ldexp(1.0, s_int - 127), block, axis=1)
     v = yq / X
     vb = band / X
     lo = _signed_value(o.e2m1_encode(v - vb))

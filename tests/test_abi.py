@@ -54,6 +54,8 @@ def test_bad_shapes(lib, M, d):
     assert lib.kq_transform(FAKE, M, d, FAKE, FAKE, None) == 1
     assert lib.kq_inverse_transform(FAKE, M, d, FAKE, FAKE, None) == 1
     assert lib.kq_dequantize(FAKE, FAKE, M, d, FAKE, None) == 1
+    assert lib.kq_quantize16(FAKE, M, d, FAKE, FAKE, FAKE, None) == 1
+    assert lib.kq_transform16(FAKE, M, d, FAKE, FAKE, None) == 1
 
 
 def test_null_and_misaligned_pointers(lib):
@@ -68,11 +70,16 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.kq_quantize_ex(FAKE, 4, 64, FAKE, FAKE, FAKE, 7, None) == 1
     assert lib.kq_dequantize(FAKE, FAKE, 4, 64, FAKE + 4, None) == 1
     assert lib.kq_device_status(None) == 1
+    assert lib.kq_quantize16(FAKE, 4, 64, FAKE, FAKE, FAKE + 1, None) == 1    # scales16 not 2-B
+    assert lib.kq_quantize16(FAKE, 4, 64, None, FAKE, FAKE, None) == 1
+    assert lib.kq_quantize16(FAKE, 1, 32 * 65536, FAKE, FAKE, FAKE, None) == 1   # too wide
+    assert lib.kq_transform16(FAKE, 4, 64, FAKE, FAKE + 8, None) == 1         # y not 16-B
 
 
 def test_empty_input_needs_no_device(lib):
     assert lib.kq_quantize(None, 0, 64, None, None, None, None) == 0
     assert lib.kq_dequantize(None, None, 0, 64, None, None) == 0
+    assert lib.kq_quantize16(None, 0, 64, None, None, None, None) == 0
 
 
 def test_binding_refuses_host_tensors():

@@ -1,0 +1,148 @@
+"""GPU parity of the 16-element variant (16x16 Kronecker blocks of four
+factors, one E8M0 scale per 16 elements) against the CPU oracle.
+
+KroQuant review, "Where Pith is reading between the lines": the transform
+extends to other block formats by changing the number of Kronecker factors.
+Inputs are the seeded DiT-shaped activations of ``workloads`` with their
+16-block parameters from ``workloads.draw_params16``; expected values come
+only from ``oracle.kq_oracle``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as w
+from oracle import kq_oracle as o
+from tests.parity import TOL, check_mx4, check_transform
+
+pytestmark = pytest.mark.gpu
+
+kq = pytest.importorskip("w4a4_post_quantization_b200")
+DEV = "cuda:0"
+REDUCED_M = 67
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def _run(x_t, params16):
+    xd = x_t.to(DEV)
+    pd = _dev(params16)
+    q, s = kq.quantize16(xd, pd)
+    y = kq.transform16(xd, pd)
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), s.cpu().numpy(), y.cpu().numpy()
+
+
+def _check(x_bits, params16, q, s, y, bound=True):
+    x64 = o.bf16_bits_to_float64(x_bits)
+    y64 = o.transform16(x64, params16)
+    cond = o.abs_transform16(x64, params16)
+    worst = check_transform(y, y64, cond)
+    st = check_mx4(q, s, y64, cond, block=16)
+    if bound:
+        assert st["scale_exempt"] <= max(2, st["blocks"] // 1000)
+        assert st["code_exempt"] <= max(4, st["elements"] // 10000)
+    return worst, st
+
+
+def _bits(x_t):
+    return x_t.view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("key", w.all_case_keys(), ids=lambda k: f"{k[0]}-d{k[1]}-g{k[2]}")
+def test_block16_reduced_configs_elementwise(key):
+    name, di, gi = key
+    M = w.CONFIGS[name]["M"] if name == "tiny" else REDUCED_M
+    c = w.make_case(name, di, gi, M=M)
+    p16 = w.draw_params16(c.d, c.seed)
+    q, s, y = _run(c.x, p16)
+    worst, _ = _check(c.x_bits(), p16, q, s, y)
+    assert worst < TOL
+
+
+@pytest.mark.parametrize("key", [("stress", 0, 0), ("flux_schnell", 1, 2), ("sana", 0, 0)],
+                         ids=lambda k: f"{k[0]}-d{k[1]}-g{k[2]}")
+def test_block16_full_size_sampled_rows(key):
+    name, di, gi = key
+    c = w.make_case(name, di, gi)
+    p16 = w.draw_params16(c.d, c.seed)
+    q, s, y = _run(c.x, p16)
+    rng = np.random.default_rng(c.seed)
+    rows = np.array(sorted(set(range(3)) | set(range(c.M - 3, c.M)) |
+                           set(rng.choice(c.M, 12, replace=False).tolist())))
+    _check(c.x_bits()[rows], p16, q[rows], s[rows], y[rows])
+
+
+def test_block16_matches_oracle_bytes_on_tiny():
+    """Packed codes and scales equal the oracle's bytes except inside the
+    tolerance band (counted, and rare)."""
+    c = w.make_case("tiny", 0, 0)
+    p16 = w.draw_params16(c.d, c.seed)
+    q, s, y = _run(c.x, p16)
+    q_ref, s_ref = o.quantize16(c.x_bits(), p16)
+    assert q.shape == q_ref.shape and s.shape == s_ref.shape
+    assert (q != q_ref).mean() < 1e-3 and (s != s_ref).mean() < 1e-3
+
+
+def test_block16_singular_factor_takes_the_plain_form():
+    """(a, b, c) = (-1, 1, 1) gives g11 = 0: that CTA's units run the plain
+    four-term stages, in either 16-block of a unit."""
+    c = w.make_case("flux_schnell", 0, 0, M=150)
+    p16 = w.draw_params16(c.d, c.seed)
+    p16[10, 1] = [-1.0, 1.0, 1.0]               # block 0 of unit 5
+    p16[181, 3] = [-1.0, 1.0, 1.0]              # block 1 of unit 90
+    q, s, y = _run(c.x, p16)
+    _check(c.x_bits(), p16, q, s, y)
+
+
+def test_block16_large_shear_growth_takes_the_plain_form():
+    c = w.make_case("tiny", 0, 0, M=40)
+    p16 = w.draw_params16(c.d, c.seed)
+    p16[7] = [[300.0, 1.0, 0.0]] * 4             # growth 301^4 > 2^24
+    q, s, y = _run(c.x, p16)
+    _check(c.x_bits(), p16, q, s, y)
+
+
+@pytest.mark.parametrize("d", [32, 64, 32 * 389, 32 * 1031])
+def test_block16_odd_widths(d):
+    """One unit per row, and prime unit counts (panels of one column unit)."""
+    x = w.random_bf16((37, d), seed=d)
+    p16 = w.draw_params16(d, seed=d)
+    q, s, y = _run(x, p16)
+    _check(_bits(x), p16, q, s, y)
+
+
+def test_block16_zero_and_huge_blocks():
+    d = 128
+    x = w.random_bf16((9, d), seed=5).float().numpy()
+    x[0] = 0.0                                   # all-zero row: scale byte 0
+    x[1, :16] = 0.0                              # one zero 16-block next to a live one
+    x[2] *= 2.0 ** 60
+    x[3] *= 2.0 ** -100
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    p16 = w.draw_params16(d, seed=11)
+    q, s, y = _run(xt, p16)
+    _check(_bits(xt), p16, q, s, y, bound=False)
+    assert (s[0] == 0).all() and s[1, 0] == 0 and s[1, 1] != 0
+    assert ((q[0] & 0x77) == 0).all()
+
+
+def test_block16_empty_and_invalid():
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device=DEV)
+    p16 = torch.zeros((4, 4, 3), dtype=torch.float32, device=DEV)
+    q, s = kq.quantize16(x, p16)
+    assert q.shape == (0, 32) and s.shape == (0, 4)
+    lib = kq.lib()
+    xd = torch.zeros((4, 64), dtype=torch.bfloat16, device=DEV)
+    qd = torch.empty((4, 32), dtype=torch.uint8, device=DEV)
+    sd = torch.empty((4 * 4 + 1,), dtype=torch.uint8, device=DEV)
+    # A scale array that is not 2-byte aligned is rejected before any launch.
+    st = lib.kq_quantize16(xd.data_ptr(), 4, 64, p16.data_ptr(), qd.data_ptr(),
+                           sd.data_ptr() + 1, torch.cuda.current_stream().cuda_stream)
+    assert st == 1
+    st = lib.kq_transform16(xd.data_ptr(), 4, 48, p16.data_ptr(), qd.data_ptr(),
+                            torch.cuda.current_stream().cuda_stream)
+    assert st == 1
+    assert kq.device_status() == 0

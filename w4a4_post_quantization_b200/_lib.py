@@ -30,6 +30,8 @@ SIGNATURES = {
     "kq_quantize_hadamard": [_p, _i64, _i64, _p, _p, _p],
     "kq_quantize_smooth": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_transform": [_p, _i64, _i64, _p, _p, _p],
+    "kq_quantize16": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_transform16": [_p, _i64, _i64, _p, _p, _p],
     "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
     "kq_quantize_host": [_p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p],
@@ -170,6 +172,47 @@ def transform(x: torch.Tensor, params: torch.Tensor, y=None):
     _dev_tensor(y, torch.float32, "y")
     st = lib().kq_transform(x.data_ptr(), M, d, params.data_ptr(), y.data_ptr(), _stream(x.device))
     _check("kq_transform", st)
+    return y
+
+
+def _params16(params16: torch.Tensor, d: int) -> torch.Tensor:
+    _dev_tensor(params16, torch.float32, "params16")
+    if params16.numel() != (d // 16) * 12:
+        raise ValueError("params16 must hold [d/16, 4, 3] float32 values")
+    return params16
+
+
+def quantize16(x: torch.Tensor, params16: torch.Tensor, q=None, scales16=None):
+    """16-element variant: returns (packed codes uint8 [M, d/2], scale bytes
+    uint8 [M, d/16])."""
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    _params16(params16, d)
+    if q is None:
+        q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
+    if scales16 is None:
+        scales16 = torch.empty((M, d // 16), dtype=torch.uint8, device=x.device)
+    _dev_tensor(q, torch.uint8, "q")
+    _dev_tensor(scales16, torch.uint8, "scales16")
+    if tuple(q.shape) != (M, d // 2) or tuple(scales16.shape) != (M, d // 16):
+        raise ValueError("output shapes must be [M, d/2] and [M, d/16]")
+    st = lib().kq_quantize16(x.data_ptr(), M, d, params16.data_ptr(), q.data_ptr(),
+                             scales16.data_ptr(), _stream(x.device))
+    _check("kq_quantize16", st)
+    return q, scales16
+
+
+def transform16(x: torch.Tensor, params16: torch.Tensor, y=None):
+    """y = x T16 in float32 (16-element blocks)."""
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    _params16(params16, d)
+    if y is None:
+        y = torch.empty((M, d), dtype=torch.float32, device=x.device)
+    _dev_tensor(y, torch.float32, "y")
+    st = lib().kq_transform16(x.data_ptr(), M, d, params16.data_ptr(), y.data_ptr(),
+                              _stream(x.device))
+    _check("kq_transform16", st)
     return y
 
 

@@ -380,6 +380,139 @@ __device__ __forceinline__ void plain_apply(f2 (&u)[16], const PlainFactors& f) 
   }
 }
 
+// -------------------------------------------- 16-element blocks, in pairs
+// The 16-element variant keeps two adjacent 16-blocks in one 32-element unit:
+// u[0..7] is block 0, u[8..15] block 1, each with its own four factors
+// (index bits 3..0 of the block, G1 on bit 3).
+struct ShearDiag16 {
+  f2 r10[2][3], r01[2][3];   // per block: stages on index bits 3, 2, 1
+  float r10b[2], r01b[2];    // per block: bit 0
+  f2 delta[16];              // (delta_2m, delta_2m+1), block 0 then block 1
+};
+
+struct PlainFactors16 {
+  f2 g00[2][3], g10[2][3], g01[2][3], g11[2][3];
+  float h00[2], h10[2], h01[2], h11[2];
+};
+
+constexpr int kFactors16 = 4;
+
+// p: the 2 x 4 x 3 parameters of the unit's two blocks.
+__device__ __forceinline__ bool load_shear_diag16(ShearDiag16& f, const float* p) {
+  bool ok = true;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const float* ph = p + 12 * h;
+    double g00[kFactors16], g11[kFactors16];
+    double growth = 1.0;
+    float r10[kFactors16], r01[kFactors16];
+#pragma unroll
+    for (int k = 0; k < kFactors16; ++k) {
+      double a00, a01, a10, a11;
+      factor_entries(ph, k, a00, a01, a10, a11);
+      g00[k] = a00;
+      g11[k] = a11;
+      const double ra = ph[3 * k + 0], rb = a01 / a11;
+      ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
+      growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
+      r10[k] = (float)ra;
+      r01[k] = (float)rb;
+    }
+    ok = ok && (growth <= kShearGrowthMax);
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+      f.r10[h][k] = pack2(r10[k], r10[k]);
+      f.r01[h][k] = pack2(r01[k], r01[k]);
+    }
+    f.r10b[h] = r10[3];
+    f.r01b[h] = r01[3];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      double d0 = 1.0;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) d0 *= ((2 * m) >> (3 - k)) & 1 ? g11[k] : g00[k];
+      f.delta[8 * h + m] = pack2((float)(d0 * g00[3]), (float)(d0 * g11[3]));
+    }
+  }
+  return ok;
+}
+
+__device__ __forceinline__ void load_plain16(PlainFactors16& f, const float* p) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+#pragma unroll
+    for (int k = 0; k < kFactors16; ++k) {
+      double g00, g01, g10, g11;
+      factor_entries(p + 12 * h, k, g00, g01, g10, g11);
+      const float f00 = (float)g00, f01 = (float)g01, f10 = (float)g10, f11 = (float)g11;
+      if (k < 3) {
+        f.g00[h][k] = pack2(f00, f00);
+        f.g01[h][k] = pack2(f01, f01);
+        f.g10[h][k] = pack2(f10, f10);
+        f.g11[h][k] = pack2(f11, f11);
+      } else {
+        f.h00[h] = f00; f.h01[h] = f01; f.h10[h] = f10; f.h11[h] = f11;
+      }
+    }
+  }
+}
+
+// One stage on registers u[kOff .. kOff + 8) (one 16-block).
+template <int kHalfDist, int kOff>
+__device__ __forceinline__ void shear_stage8(f2 (&u)[16], f2 r10, f2 r01) {
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    if (m & kHalfDist) continue;
+    const f2 lo = u[kOff + m], hi = u[kOff + m + kHalfDist];
+    u[kOff + m] = fma2(r10, hi, lo);
+    u[kOff + m + kHalfDist] = fma2(r01, lo, hi);
+  }
+}
+
+template <int kHalfDist, int kOff>
+__device__ __forceinline__ void plain_stage8(f2 (&u)[16], f2 g00, f2 g10, f2 g01, f2 g11) {
+#pragma unroll
+  for (int m = 0; m < 8; ++m) {
+    if (m & kHalfDist) continue;
+    const f2 lo = u[kOff + m], hi = u[kOff + m + kHalfDist];
+    u[kOff + m] = fma2(g10, hi, mul2(g00, lo));
+    u[kOff + m + kHalfDist] = fma2(g11, hi, mul2(g01, lo));
+  }
+}
+
+__device__ __forceinline__ void shear_apply16(f2 (&u)[16], const ShearDiag16& f) {
+  shear_stage8<4, 0>(u, f.r10[0][0], f.r01[0][0]);
+  shear_stage8<2, 0>(u, f.r10[0][1], f.r01[0][1]);
+  shear_stage8<1, 0>(u, f.r10[0][2], f.r01[0][2]);
+  shear_stage8<4, 8>(u, f.r10[1][0], f.r01[1][0]);
+  shear_stage8<2, 8>(u, f.r10[1][1], f.r01[1][1]);
+  shear_stage8<1, 8>(u, f.r10[1][2], f.r01[1][2]);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const int h = m >> 3;
+    float lo, hi;
+    unpack2(u[m], lo, hi);
+    u[m] = pack2(__fmaf_rn(f.r10b[h], hi, lo), __fmaf_rn(f.r01b[h], lo, hi));
+  }
+}
+
+__device__ __forceinline__ void plain_apply16(f2 (&u)[16], const PlainFactors16& f) {
+  plain_stage8<4, 0>(u, f.g00[0][0], f.g10[0][0], f.g01[0][0], f.g11[0][0]);
+  plain_stage8<2, 0>(u, f.g00[0][1], f.g10[0][1], f.g01[0][1], f.g11[0][1]);
+  plain_stage8<1, 0>(u, f.g00[0][2], f.g10[0][2], f.g01[0][2], f.g11[0][2]);
+  plain_stage8<4, 8>(u, f.g00[1][0], f.g10[1][0], f.g01[1][0], f.g11[1][0]);
+  plain_stage8<2, 8>(u, f.g00[1][1], f.g10[1][1], f.g01[1][1], f.g11[1][1]);
+  plain_stage8<1, 8>(u, f.g00[1][2], f.g10[1][2], f.g01[1][2], f.g11[1][2]);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const int h = m >> 3;
+    float lo, hi;
+    unpack2(u[m], lo, hi);
+    u[m] = pack2(__fmaf_rn(f.h10[h], hi, __fmul_rn(f.h00[h], lo)),
+                 __fmaf_rn(f.h11[h], hi, __fmul_rn(f.h01[h], lo)));
+  }
+}
+
 // Fixed block Hadamard H_32 (Sylvester order: H2 = [[1,1],[1,-1]] on every
 // bit), then the orthonormal factor 1/sqrt(32) as one float32 multiply.
 __device__ __forceinline__ void hadamard_apply(f2 (&u)[16]) {
@@ -448,6 +581,49 @@ __device__ __forceinline__ float block_amax(const f2 (&u)[16]) {
   const float c0 = max3(b[0], b[1], b[2]), c1 = max3(b[3], b[4], b[5]);
   const float c2 = max3(b[6], b[7], b[8]), c3 = fmaxf(b[9], b[10]);
   return fmaxf(max3(c0, c1, c2), c3);
+}
+
+// Scale byte of a block from its largest magnitude, and 2^-e as a float.
+__device__ __forceinline__ uint32_t e8m0_from_amax(float amax, f2& inv_x2) {
+  const int field = static_cast<int>(__float_as_uint(amax) >> 23);
+  const int sbyte = field > 2 ? field - 2 : 0;
+  const float inv_x = __uint_as_float(static_cast<uint32_t>(254 - sbyte) << 23);
+  inv_x2 = pack2(inv_x, inv_x);
+  return static_cast<uint32_t>(sbyte);
+}
+
+// Two 16-element blocks (u[0..7], u[8..15]): 16 bytes of codes (block 0 in
+// the first 8) and the two scale bytes (block 0 in bits 0..7).
+__device__ __forceinline__ Mx4Block mxfp4_block16x2(const f2 (&u)[16]) {
+  uint32_t w[4];
+  uint32_t scales = 0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float a[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      unpack2(u[8 * h + i], a[2 * i], a[2 * i + 1]);
+      a[2 * i] = fabsf(a[2 * i]);
+      a[2 * i + 1] = fabsf(a[2 * i + 1]);
+    }
+    const float b0 = max3(a[0], a[1], a[2]), b1 = max3(a[3], a[4], a[5]);
+    const float b2 = max3(a[6], a[7], a[8]), b3 = max3(a[9], a[10], a[11]);
+    const float b4 = max3(a[12], a[13], a[14]);
+    const float amax = fmaxf(max3(b0, b1, b2), max3(b3, b4, a[15]));
+    f2 s2;
+    scales |= e8m0_from_amax(amax, s2) << (8 * h);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) unpack2(mul2(u[8 * h + 4 * k + i], s2), v[2 * i], v[2 * i + 1]);
+      w[2 * h + k] = e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+    }
+  }
+  Mx4Block r;
+  r.codes = make_uint4(w[0], w[1], w[2], w[3]);
+  r.scale = scales;
+  return r;
 }
 
 __device__ __forceinline__ Mx4Block mxfp4_block(const f2 (&u)[16]) {

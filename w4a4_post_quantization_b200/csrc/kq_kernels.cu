@@ -16,6 +16,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <mutex>
+#include <type_traits>
 
 #include "kq.h"
 #include "kq_device.cuh"
@@ -33,7 +34,9 @@ int record_cuda_error(cudaError_t e) {
   return KQ_ERR_CUDA;
 }
 
-enum Xform { kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2 };
+// kXfKron16: 16-element Kronecker blocks (four factors each) with a scale
+// per 16 elements; a thread owns a unit of two adjacent 16-blocks.
+enum Xform { kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2, kXfKron16 = 3 };
 enum Out { kOutMx4 = 0, kOutF32 = 1 };
 
 constexpr int kConsumerWarps = 8;
@@ -246,11 +249,11 @@ __device__ __forceinline__ void release_stage(uint64_t* bar, int lane) {
   if (lane == 0) mbar_arrive(bar);
 }
 
-template <int kXf, int kOut, class Cfg, int kForm>
+template <int kXf, int kOut, class Cfg, int kForm, class SD, class PF>
 __device__ __forceinline__ void panel_consume(const PanelArgs& a, const uint8_t* stages,
                                               uint64_t* full, uint64_t* empty, int n_local,
                                               int k0, int cpp, int tid, bool active, int rho,
-                                              int j, const ShearDiag& sd, const PlainFactors& pf) {
+                                              int j, const SD& sd, const PF& pf) {
   constexpr int kRpt = Cfg::kRpt;
   const int S = a.stages;
   const int lane = tid & 31;
@@ -303,16 +306,28 @@ __device__ __forceinline__ void panel_consume(const PanelArgs& a, const uint8_t*
         u[4 * q + 2] = bf16x2_to_f2(c[r][q].z);
         u[4 * q + 3] = bf16x2_to_f2(c[r][q].w);
       }
-      if (kXf == kXfKron && kForm == 1) {
+      if constexpr (kXf == kXfKron16) {
+        if constexpr (kForm == 1) {
+          plain_apply16(u, pf);
+        } else {
+          shear_apply16(u, sd);
+          diag_mul(u, sd.delta);
+        }
+      } else if constexpr (kXf == kXfKron && kForm == 1) {
         plain_apply(u, pf);
-      } else if (kXf == kXfHadamard) {
+      } else if constexpr (kXf == kXfHadamard) {
         hadamard_apply(u);
       } else {
-        if (kXf == kXfKron) shear_apply(u, sd);
+        if constexpr (kXf == kXfKron) shear_apply(u, sd);
         diag_mul(u, sd.delta);
       }
       const int64_t g = rr * a.nb + j;
-      if (kOut == kOutMx4) {
+      if constexpr (kOut == kOutMx4 && kXf == kXfKron16) {
+        // Two scale bytes per unit, block 0 at the lower address.
+        const Mx4Block b = mxfp4_block16x2(u);
+        __stcs(reinterpret_cast<uint4*>(a.q + g * 16), b.codes);
+        reinterpret_cast<uint16_t*>(a.scales)[g] = static_cast<uint16_t>(b.scale);
+      } else if constexpr (kOut == kOutMx4) {
         const Mx4Block b = mxfp4_block(u);
         __stcs(reinterpret_cast<uint4*>(a.q + g * 16), b.codes);
         a.scales[g] = static_cast<uint8_t>(b.scale);
@@ -391,11 +406,21 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   const bool active = tid < a.W * a.R;
   const int rho = tid / a.W;
   const int j = panel * a.W + (tid % a.W);
-  ShearDiag sd;
-  PlainFactors pf;
+  using SD = std::conditional_t<kXf == kXfKron16, ShearDiag16, ShearDiag>;
+  using PF = std::conditional_t<kXf == kXfKron16, PlainFactors16, PlainFactors>;
+  SD sd;
+  PF pf;
   int plain = 0;
-  if (kXf == kXfKron) {
-    if (active) plain = load_shear_diag(sd, a.aux + (int64_t)j * 15) ? 0 : 1;
+  if constexpr (kXf == kXfKron || kXf == kXfKron16) {
+    // Parameters per thread unit: 5 x 3 for a 32-block, 2 x 4 x 3 for a pair
+    // of 16-blocks.
+    constexpr int kUnitParams = kXf == kXfKron ? 15 : 24;
+    const float* p = a.aux + (int64_t)j * kUnitParams;
+    if constexpr (kXf == kXfKron) {
+      if (active) plain = load_shear_diag(sd, p) ? 0 : 1;
+    } else {
+      if (active) plain = load_shear_diag16(sd, p) ? 0 : 1;
+    }
     // One form for the whole CTA: the plain one if any of its blocks needs it.
     asm volatile(
         "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
@@ -403,8 +428,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         : "=r"(plain)
         : "r"(plain), "r"(kCons)
         : "memory");
-    if (plain && active) load_plain(pf, a.aux + (int64_t)j * 15);
-  } else if (kXf == kXfSmooth) {
+    if (plain && active) {
+      if constexpr (kXf == kXfKron) load_plain(pf, p);
+      else load_plain16(pf, p);
+    }
+  } else if constexpr (kXf == kXfSmooth) {
     if (active) {
       const float4* v = reinterpret_cast<const float4*>(a.aux + (int64_t)j * kBlock);
 #pragma unroll
@@ -683,7 +711,9 @@ int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, 
   constexpr int kRpt = Cfg::kRpt;
   const int nb = static_cast<int>(d / kBlock);
   PanelArgs a{};
-  if (panel_use<Cfg>(nb, di.sms, &a.W, &a.R) < 0.5) return KQ_ERR_INVALID;
+  // The 16-element variant has no other kernel, so it takes any shape.
+  const double min_use = kXf == kXfKron16 ? 0.0 : 0.5;
+  if (panel_use<Cfg>(nb, di.sms, &a.W, &a.R) < min_use) return KQ_ERR_INVALID;
   a.M = M;
   a.nb = nb;
   a.panels = nb / a.W;
@@ -782,24 +812,30 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
   a.inverse = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nb = d / kBlock;
-  if (impl == KQ_IMPL_AUTO) {
-    if (nb <= 65535 && panel_fits(static_cast<int>(nb), di->sms) && M < (int64_t(1) << 30))
-      impl = KQ_IMPL_PANEL;
-    else
-      impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
-  }
-  if (impl == KQ_IMPL_MMA) {
-    if (kXf != kXfKron) return KQ_ERR_INVALID;
-    return launch_mma_kron(x, M, d, aux, kOut == kOutMx4 ? q : nullptr,
-                           kOut == kOutMx4 ? scales : nullptr, kOut == kOutF32 ? y : nullptr, st);
-  }
-  if (impl == KQ_IMPL_PANEL) {
-    if (nb > 65535) return KQ_ERR_INVALID;
+  if constexpr (kXf == kXfKron16) {
+    // Only the panel kernel carries the 16-element variant.
+    if (impl != KQ_IMPL_PANEL || nb > 65535) return KQ_ERR_INVALID;
     return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
+  } else {
+    if (impl == KQ_IMPL_AUTO) {
+      if (nb <= 65535 && panel_fits(static_cast<int>(nb), di->sms) && M < (int64_t(1) << 30))
+        impl = KQ_IMPL_PANEL;
+      else
+        impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
+    }
+    if (impl == KQ_IMPL_MMA) {
+      if (kXf != kXfKron) return KQ_ERR_INVALID;
+      return launch_mma_kron(x, M, d, aux, kOut == kOutMx4 ? q : nullptr,
+                             kOut == kOutMx4 ? scales : nullptr, kOut == kOutF32 ? y : nullptr, st);
+    }
+    if (impl == KQ_IMPL_PANEL) {
+      if (nb > 65535) return KQ_ERR_INVALID;
+      return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
+    }
+    if (impl == KQ_IMPL_TMA) return launch_tma<kXf, kOut>(x, M, d, a, st, *di, dev);
+    if (impl == KQ_IMPL_DIRECT) return launch_direct<kXf, kOut, false>(x, M, d, a, st, *di, dev);
+    return KQ_ERR_INVALID;
   }
-  if (impl == KQ_IMPL_TMA) return launch_tma<kXf, kOut>(x, M, d, a, st, *di, dev);
-  if (impl == KQ_IMPL_DIRECT) return launch_direct<kXf, kOut, false>(x, M, d, a, st, *di, dev);
-  return KQ_ERR_INVALID;
 }
 
 int check_quant_args(const uint16_t* x, int64_t M, int64_t d, const void* aux, bool need_aux,
@@ -853,6 +889,25 @@ extern "C" int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float
   if (!x || !params || !y || !aligned(x, 16) || !aligned(y, 16) || !aligned(params, 4))
     return KQ_ERR_INVALID;
   return run<kXfKron, kOutF32>(x, M, d, params, nullptr, nullptr, y, KQ_IMPL_AUTO, stream);
+}
+
+extern "C" int kq_quantize16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
+                             uint8_t* q_packed, uint8_t* scales16, void* stream) {
+  int rc = check_quant_args(x, M, d, params16, true, q_packed, scales16);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!aligned(scales16, 2) || d / kBlock > 65535) return KQ_ERR_INVALID;
+  return run<kXfKron16, kOutMx4>(x, M, d, params16, q_packed, scales16, nullptr, KQ_IMPL_PANEL,
+                                 stream);
+}
+
+extern "C" int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
+                              float* y, void* stream) {
+  int rc = check_shape(M, d);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!x || !params16 || !y || !aligned(x, 16) || !aligned(y, 16) || !aligned(params16, 4) ||
+      d / kBlock > 65535)
+    return KQ_ERR_INVALID;
+  return run<kXfKron16, kOutF32>(x, M, d, params16, nullptr, nullptr, y, KQ_IMPL_PANEL, stream);
 }
 
 extern "C" int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,
