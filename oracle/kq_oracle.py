@@ -288,6 +288,46 @@ def quantize16(x_bits: np.ndarray, params16: np.ndarray):
 
 
 # --------------------------------------------------------------------------
+# Weight side and the W4A4 product (review, "Circularity Check", Eq. 1:
+# ``A T (W T^-T)^T = A W^T``, the inverse folded into the weights offline)
+# --------------------------------------------------------------------------
+def fold_weight(w64: np.ndarray, params: np.ndarray) -> np.ndarray:
+    """``W' = W T^-T`` for weights ``W [N, d]`` (rows are output channels):
+    each 32-column block of a row is multiplied on the right by
+    ``(K^(j))^-T``, so that ``(x T) W'^T = x W^T``."""
+    params = np.asarray(params)
+    return _apply_blocks(w64, lambda j: inverse_block(params[j]).T)
+
+
+def abs_fold_weight(w64: np.ndarray, params: np.ndarray) -> np.ndarray:
+    """``|W| |K^-T|`` blockwise, the magnitude the fold's rounding is stated
+    against."""
+    params = np.asarray(params)
+    return _apply_blocks(np.abs(w64), lambda j: np.abs(inverse_block(params[j]).T))
+
+
+def quantize_weight(w_bits: np.ndarray, params: np.ndarray):
+    """MXFP4 of the folded weights: bf16 bits ``[N, d]`` -> (packed codes
+    ``[N, d/2]``, scales ``[N, d/32]``), the same quantizer as activations."""
+    codes, scales = mxfp4_quantize(fold_weight(bf16_bits_to_float64(w_bits), params))
+    return pack_codes(codes), scales
+
+
+def mxfp4_gemm(qa: np.ndarray, sa: np.ndarray, qb: np.ndarray, sb: np.ndarray,
+               block: int = BLOCK) -> np.ndarray:
+    """``C = A B^T`` in float64 for MXFP4 operands ``A [M, K]`` and ``B [N, K]``
+    (packed codes and per-``block`` scales along K): the product the W4A4
+    layer computes, from the exact values the codes and scales stand for."""
+    return dequantize(qa, sa, block) @ dequantize(qb, sb, block).T
+
+
+def abs_mxfp4_gemm(qa: np.ndarray, sa: np.ndarray, qb: np.ndarray, sb: np.ndarray,
+                   block: int = BLOCK) -> np.ndarray:
+    """``|A| |B|^T``: the sum of the magnitudes of the products in each output."""
+    return np.abs(dequantize(qa, sa, block)) @ np.abs(dequantize(qb, sb, block)).T
+
+
+# --------------------------------------------------------------------------
 # Magnitudes the tolerance rule is stated against
 # --------------------------------------------------------------------------
 def abs_transform(x64: np.ndarray, params: np.ndarray) -> np.ndarray:

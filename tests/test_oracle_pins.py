@@ -396,3 +396,105 @@ def test_quantize16_identity_factors_use_16_element_scales():
     q, s = o.quantize16(x, p)
     assert list(s[0]) == [128, 124]                      # exponents 1 and -3
     assert (o.unpack_codes(q)[0] == 6).all()             # 8/2 = 4 and 0.5*8 = 4
+
+
+# --------------------------------------------- weight fold and W4A4 product
+def test_fold_weight_keeps_the_layer_output_eq1():
+    """Eq. 1 through the oracle's own fold: (x T) fold(W)^T = x W^T.  A fold
+    that used K instead of K^-1, or forgot the transpose, fails."""
+    rng = np.random.default_rng(21)
+    nb = 4
+    p = rand_params(nb, 22)
+    x = rng.standard_normal((7, 32 * nb))
+    W = rng.standard_normal((9, 32 * nb))
+    lhs = o.transform(x, p) @ o.fold_weight(W, p).T
+    np.testing.assert_allclose(lhs, x @ W.T, rtol=1e-10, atol=1e-10)
+
+
+def test_fold_weight_of_an_orthonormal_block_is_the_transform():
+    """(a, b, c) = (-1, 1/sqrt2, 1/sqrt2) makes every factor orthonormal, so
+    K^-T = K and folding a weight row equals transforming it."""
+    s = 1 / math.sqrt(2)
+    p = np.tile(np.array([-1.0, s, s]), (2, 5, 1))
+    W = np.random.default_rng(23).standard_normal((3, 64))
+    np.testing.assert_allclose(o.fold_weight(W, p), o.transform(W, p), atol=1e-12)
+
+
+def test_fold_weight_single_factor_closed_form():
+    """Only G5 non-trivial (bit 0 of the in-block index): the fold acts on
+    adjacent pairs with G5^-T = [[g11, -g10], [-g01, g00]] (row-vector form,
+    w' = w G5^-T)."""
+    a, b, c = 0.5, 2.0, -0.75
+    p = np.zeros((1, 5, 3))
+    p[:, :, 1] = 1.0
+    p[0, 4] = [a, b, c]
+    g00, g01, g10, g11 = b, c, a * b, a * c + 1 / b
+    W = np.random.default_rng(24).standard_normal((2, 32))
+    got = o.fold_weight(W, p)
+    w0, w1 = W[:, 0::2], W[:, 1::2]
+    np.testing.assert_allclose(got[:, 0::2], w0 * g11 + w1 * (-g01), atol=1e-12)
+    np.testing.assert_allclose(got[:, 1::2], w0 * (-g10) + w1 * g00, atol=1e-12)
+
+
+def _pack_hand(codes):
+    codes = np.asarray(codes, dtype=np.uint8)
+    return (codes[:, 0::2] | (codes[:, 1::2] << 4)).astype(np.uint8)
+
+
+def test_mxfp4_gemm_brute_force():
+    """Every output of the product equals a triple loop over values decoded
+    by hand from the E2M1 table {0, .5, 1, 1.5, 2, 3, 4, 6} and 2^(s-127)."""
+    rng = np.random.default_rng(25)
+    M, N, K = 3, 4, 64
+    ca = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    cb = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    sa = rng.integers(120, 135, (M, K // 32), dtype=np.uint8)
+    sb = rng.integers(120, 135, (N, K // 32), dtype=np.uint8)
+    table = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+
+    def val(code, s):
+        v = table[int(code) & 7] * 2.0 ** (int(s) - 127)
+        return -v if code & 8 else v
+
+    C = o.mxfp4_gemm(_pack_hand(ca), sa, _pack_hand(cb), sb)
+    for m in range(M):
+        for n in range(N):
+            ref = sum(val(ca[m, k], sa[m, k // 32]) * val(cb[n, k], sb[n, k // 32])
+                      for k in range(K))
+            assert C[m, n] == ref
+
+
+def test_mxfp4_gemm_constant_operands_closed_form():
+    """All codes 1.0 (code 2): C = K 2^(sa + sb - 254); code 6 (value 4)
+    against code 0xB (value -1.5): C = -6 K."""
+    M, N, K = 5, 6, 96
+    qa = _pack_hand(np.full((M, K), 2))
+    qb = _pack_hand(np.full((N, K), 2))
+    sa = np.full((M, K // 32), 130, dtype=np.uint8)
+    sb = np.full((N, K // 32), 121, dtype=np.uint8)
+    assert (o.mxfp4_gemm(qa, sa, qb, sb) == K * 2.0 ** (130 + 121 - 254)).all()
+    qa = _pack_hand(np.full((M, K), 6))
+    qb = _pack_hand(np.full((N, K), 0xB))
+    one_a = np.full((M, K // 32), 127, dtype=np.uint8)
+    one_b = np.full((N, K // 32), 127, dtype=np.uint8)
+    assert (o.mxfp4_gemm(qa, one_a, qb, one_b) == -6.0 * K).all()
+
+
+def test_quantize_weight_with_identity_factors_is_the_activation_quantizer():
+    """With G_k = I the fold is the identity, so the weight quantizer gives
+    the activation quantizer's bytes on the same bf16 matrix."""
+    rng = np.random.default_rng(26)
+    W = rng.standard_normal((12, 96)).astype(np.float32)
+    Wb = (W.view(np.uint32) >> 16).astype(np.uint16)
+    p = np.zeros((3, 5, 3), dtype=np.float32)
+    p[:, :, 1] = 1.0
+    qw, sw = o.quantize_weight(Wb, p)
+    qa, sa = o.quantize(Wb, p)
+    assert np.array_equal(qw, qa) and np.array_equal(sw, sa)
+    # and with an orthonormal block (K^-T = K) it is the transformed quantizer
+    s2 = 1 / math.sqrt(2)
+    p = np.tile(np.array([-1.0, s2, s2], dtype=np.float32), (3, 5, 1))
+    qw, sw = o.quantize_weight(Wb, p)
+    qa, sa = o.quantize(Wb, p)
+    assert np.array_equal(sw, sa)
+    assert (o.unpack_codes(qw) != o.unpack_codes(qa)).mean() < 0.01
