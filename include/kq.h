@@ -117,6 +117,21 @@ int kq_quantize16(const uint16_t* x, int64_t M, int64_t d, const float* params16
 int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
                    float* y, void* stream);
 
+/* Weight side of the transformed layer (review, "Circularity Check", Eq. 1:
+ * A T (W T^-T)^T = A W^T, the inverse folded into the weights offline).
+ * w is the bf16 weight matrix [N][d] of a linear layer y = x W^T (row n holds
+ * output channel n, d = input channels, the same d and params as the
+ * activations it meets).  kq_quantize_weight writes MXFP4(W T^-T): each
+ * 32-column block of a row is multiplied on the right by
+ * (K^(j))^-T = (G1^-1)^T (x) ... (x) (G5^-1)^T, then quantized exactly as
+ * kq_quantize does (codes [N][d/2], scales [N][d/32], 16-byte aligned w and
+ * q_packed).  kq_fold_weight writes W T^-T in float32 [N][d] (16-byte
+ * aligned).  d at most 32 * 65535; N at most 2^31 - 1024. */
+int kq_quantize_weight(const uint16_t* w, int64_t N, int64_t d, const float* params,
+                       uint8_t* q_packed, uint8_t* scales, void* stream);
+int kq_fold_weight(const uint16_t* w, int64_t N, int64_t d, const float* params,
+                   float* w_folded, void* stream);
+
 /* x = y T^-1 in float32 with T^-1 = diag(G1^-1 (x) ... (x) G5^-1) (review,
  * axiom ledger: the inverse of a Kronecker product factorizes). */
 int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,

@@ -56,6 +56,8 @@ def test_bad_shapes(lib, M, d):
     assert lib.kq_dequantize(FAKE, FAKE, M, d, FAKE, None) == 1
     assert lib.kq_quantize16(FAKE, M, d, FAKE, FAKE, FAKE, None) == 1
     assert lib.kq_transform16(FAKE, M, d, FAKE, FAKE, None) == 1
+    assert lib.kq_quantize_weight(FAKE, M, d, FAKE, FAKE, FAKE, None) == 1
+    assert lib.kq_fold_weight(FAKE, M, d, FAKE, FAKE, None) == 1
 
 
 def test_null_and_misaligned_pointers(lib):

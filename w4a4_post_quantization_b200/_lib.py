@@ -32,6 +32,8 @@ SIGNATURES = {
     "kq_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_quantize16": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_transform16": [_p, _i64, _i64, _p, _p, _p],
+    "kq_quantize_weight": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_fold_weight": [_p, _i64, _i64, _p, _p, _p],
     "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
     "kq_quantize_host": [_p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p],
@@ -214,6 +216,32 @@ def transform16(x: torch.Tensor, params16: torch.Tensor, y=None):
                               _stream(x.device))
     _check("kq_transform16", st)
     return y
+
+
+def quantize_weight(w: torch.Tensor, params: torch.Tensor, q=None, scales=None):
+    """MXFP4(W T^-T) of bf16 weights [N, d]: (codes uint8 [N, d/2], scales
+    uint8 [N, d/32]), the operand that meets quantize(x, params)."""
+    _dev_tensor(w, torch.bfloat16, "w")
+    N, d, q, scales = _out_codes(w, q, scales)
+    _params(params, d)
+    st = lib().kq_quantize_weight(w.data_ptr(), N, d, params.data_ptr(), q.data_ptr(),
+                                  scales.data_ptr(), _stream(w.device))
+    _check("kq_quantize_weight", st)
+    return q, scales
+
+
+def fold_weight(w: torch.Tensor, params: torch.Tensor, out=None):
+    """W T^-T in float32 [N, d]."""
+    _dev_tensor(w, torch.bfloat16, "w")
+    N, d = _shape(w)
+    _params(params, d)
+    if out is None:
+        out = torch.empty((N, d), dtype=torch.float32, device=w.device)
+    _dev_tensor(out, torch.float32, "out")
+    st = lib().kq_fold_weight(w.data_ptr(), N, d, params.data_ptr(), out.data_ptr(),
+                              _stream(w.device))
+    _check("kq_fold_weight", st)
+    return out
 
 
 def inverse_transform(y: torch.Tensor, params: torch.Tensor, x=None):

@@ -257,18 +257,32 @@ struct PlainFactors {
 // stay inside the float32 range.
 constexpr double kShearGrowthMax = 16777216.0;   // 2^24
 
-// The four entries of G_k (row-vector form) from (a, b, c), in double.
+// The four entries of G_k (row-vector form) from (a, b, c), in double; with
+// kInvT those of (G_k^-1)^T = [[g11, -g10], [-g01, g00]] (det G_k = 1), the
+// factor of the weight-side fold W T^-T.
+template <bool kInvT = false>
 __device__ __forceinline__ void factor_entries(const float* p, int k, double& g00, double& g01,
                                                double& g10, double& g11) {
   const double a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
-  g00 = b;
-  g01 = c;
-  g10 = a * b;
-  g11 = __fma_rn(a, c, 1.0 / b);
+  const double e00 = b, e01 = c, e10 = a * b, e11 = __fma_rn(a, c, 1.0 / b);
+  if (kInvT) {
+    g00 = e11;
+    g01 = -e10;
+    g10 = -e01;
+    g11 = e00;
+  } else {
+    g00 = e00;
+    g01 = e01;
+    g10 = e10;
+    g11 = e11;
+  }
 }
 
 // Fills the shear form for the block with parameters p[15]; returns false if
-// the block must use the plain form instead.
+// the block must use the plain form instead.  The shear below a factor is
+// r10 = g10 / g00 (which is exactly a for G_k itself) and above it
+// r01 = g01 / g11.
+template <bool kInvT = false>
 __device__ __forceinline__ bool load_shear_diag(ShearDiag& f, const float* p) {
   double g00[kFactors], g11[kFactors];
   double growth = 1.0;
@@ -277,10 +291,10 @@ __device__ __forceinline__ bool load_shear_diag(ShearDiag& f, const float* p) {
 #pragma unroll
   for (int k = 0; k < kFactors; ++k) {
     double a00, a01, a10, a11;
-    factor_entries(p, k, a00, a01, a10, a11);
+    factor_entries<kInvT>(p, k, a00, a01, a10, a11);
     g00[k] = a00;
     g11[k] = a11;
-    const double ra = p[3 * k + 0];
+    const double ra = kInvT ? a10 / a00 : static_cast<double>(p[3 * k + 0]);
     const double rb = a01 / a11;
     ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
     growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
@@ -307,11 +321,12 @@ __device__ __forceinline__ bool load_shear_diag(ShearDiag& f, const float* p) {
   return ok;
 }
 
+template <bool kInvT = false>
 __device__ __forceinline__ void load_plain(PlainFactors& f, const float* p) {
 #pragma unroll
   for (int k = 0; k < kFactors; ++k) {
     double g00, g01, g10, g11;
-    factor_entries(p, k, g00, g01, g10, g11);
+    factor_entries<kInvT>(p, k, g00, g01, g10, g11);
     const float f00 = (float)g00, f01 = (float)g01, f10 = (float)g10, f11 = (float)g11;
     if (k < 4) {
       f.g00[k] = pack2(f00, f00);

@@ -36,7 +36,11 @@ int record_cuda_error(cudaError_t e) {
 
 // kXfKron16: 16-element Kronecker blocks (four factors each) with a scale
 // per 16 elements; a thread owns a unit of two adjacent 16-blocks.
-enum Xform { kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2, kXfKron16 = 3 };
+// kXfKronInvT: the weight-side fold W T^-T, factors (G_k^-1)^T.
+enum Xform { kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2, kXfKron16 = 3, kXfKronInvT = 4 };
+
+// Transforms made of five 2x2 factors per 32-block.
+__host__ __device__ constexpr bool kron5(int xf) { return xf == kXfKron || xf == kXfKronInvT; }
 enum Out { kOutMx4 = 0, kOutF32 = 1 };
 
 constexpr int kConsumerWarps = 8;
@@ -313,12 +317,12 @@ __device__ __forceinline__ void panel_consume(const PanelArgs& a, const uint8_t*
           shear_apply16(u, sd);
           diag_mul(u, sd.delta);
         }
-      } else if constexpr (kXf == kXfKron && kForm == 1) {
+      } else if constexpr (kron5(kXf) && kForm == 1) {
         plain_apply(u, pf);
       } else if constexpr (kXf == kXfHadamard) {
         hadamard_apply(u);
       } else {
-        if constexpr (kXf == kXfKron) shear_apply(u, sd);
+        if constexpr (kron5(kXf)) shear_apply(u, sd);
         diag_mul(u, sd.delta);
       }
       const int64_t g = rr * a.nb + j;
@@ -411,13 +415,13 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   SD sd;
   PF pf;
   int plain = 0;
-  if constexpr (kXf == kXfKron || kXf == kXfKron16) {
+  if constexpr (kron5(kXf) || kXf == kXfKron16) {
     // Parameters per thread unit: 5 x 3 for a 32-block, 2 x 4 x 3 for a pair
     // of 16-blocks.
-    constexpr int kUnitParams = kXf == kXfKron ? 15 : 24;
+    constexpr int kUnitParams = kron5(kXf) ? 15 : 24;
     const float* p = a.aux + (int64_t)j * kUnitParams;
-    if constexpr (kXf == kXfKron) {
-      if (active) plain = load_shear_diag(sd, p) ? 0 : 1;
+    if constexpr (kron5(kXf)) {
+      if (active) plain = load_shear_diag<kXf == kXfKronInvT>(sd, p) ? 0 : 1;
     } else {
       if (active) plain = load_shear_diag16(sd, p) ? 0 : 1;
     }
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         : "r"(plain), "r"(kCons)
         : "memory");
     if (plain && active) {
-      if constexpr (kXf == kXfKron) load_plain(pf, p);
+      if constexpr (kron5(kXf)) load_plain<kXf == kXfKronInvT>(pf, p);
       else load_plain16(pf, p);
     }
   } else if constexpr (kXf == kXfSmooth) {
@@ -711,8 +715,9 @@ int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, 
   constexpr int kRpt = Cfg::kRpt;
   const int nb = static_cast<int>(d / kBlock);
   PanelArgs a{};
-  // The 16-element variant has no other kernel, so it takes any shape.
-  const double min_use = kXf == kXfKron16 ? 0.0 : 0.5;
+  // The 16-element variant and the weight fold have no other kernel, so
+  // they take any shape.
+  const double min_use = (kXf == kXfKron16 || kXf == kXfKronInvT) ? 0.0 : 0.5;
   if (panel_use<Cfg>(nb, di.sms, &a.W, &a.R) < min_use) return KQ_ERR_INVALID;
   a.M = M;
   a.nb = nb;
@@ -812,8 +817,8 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
   a.inverse = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nb = d / kBlock;
-  if constexpr (kXf == kXfKron16) {
-    // Only the panel kernel carries the 16-element variant.
+  if constexpr (kXf == kXfKron16 || kXf == kXfKronInvT) {
+    // Only the panel kernel carries the 16-element variant and the fold.
     if (impl != KQ_IMPL_PANEL || nb > 65535) return KQ_ERR_INVALID;
     return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
   } else {
@@ -908,6 +913,26 @@ extern "C" int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const flo
       d / kBlock > 65535)
     return KQ_ERR_INVALID;
   return run<kXfKron16, kOutF32>(x, M, d, params16, nullptr, nullptr, y, KQ_IMPL_PANEL, stream);
+}
+
+extern "C" int kq_quantize_weight(const uint16_t* w, int64_t N, int64_t d, const float* params,
+                                  uint8_t* q_packed, uint8_t* scales, void* stream) {
+  int rc = check_quant_args(w, N, d, params, true, q_packed, scales);
+  if (rc != KQ_OK || N == 0) return rc;
+  if (d / kBlock > 65535) return KQ_ERR_INVALID;
+  return run<kXfKronInvT, kOutMx4>(w, N, d, params, q_packed, scales, nullptr, KQ_IMPL_PANEL,
+                                   stream);
+}
+
+extern "C" int kq_fold_weight(const uint16_t* w, int64_t N, int64_t d, const float* params,
+                              float* w_folded, void* stream) {
+  int rc = check_shape(N, d);
+  if (rc != KQ_OK || N == 0) return rc;
+  if (!w || !params || !w_folded || !aligned(w, 16) || !aligned(w_folded, 16) ||
+      !aligned(params, 4) || d / kBlock > 65535)
+    return KQ_ERR_INVALID;
+  return run<kXfKronInvT, kOutF32>(w, N, d, params, nullptr, nullptr, w_folded, KQ_IMPL_PANEL,
+                                   stream);
 }
 
 extern "C" int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,

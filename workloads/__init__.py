@@ -126,6 +126,15 @@ def draw_params16(d: int, seed: int) -> np.ndarray:
     return np.stack([a, b, c], axis=-1).astype(np.float32)
 
 
+def draw_weight(N: int, d: int, seed: int) -> torch.Tensor:
+    """Synthetic bf16 weight matrix ``[N, d]`` of a linear layer (row = output
+    channel): ``N(0, 1/d)`` entries from the stream ``[seed, 4]``, rounded to
+    float32 and then bf16."""
+    rng = np.random.default_rng([seed, 4])
+    v = rng.standard_normal((N, d)) / np.sqrt(d)
+    return torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
+
+
 def synth_inv_s(x: torch.Tensor) -> np.ndarray:
     """Reciprocal SmoothQuant channel scale for migration strength 0.5 and a
     unit weight range, from the column maxima of ``x`` (bf16 [M, d])."""
@@ -219,5 +228,5 @@ def algorithmic_bytes(M: int, d: int) -> float:
 
 
 __all__ = ["CONFIGS", "Case", "make_case", "case_seed", "all_case_keys", "random_bf16",
-           "bf16_from_float", "device_randn_bf16", "draw_params", "draw_params16", "channel_gain", "synth_inv_s", "algorithmic_bytes",
+           "bf16_from_float", "device_randn_bf16", "draw_params", "draw_params16", "draw_weight", "channel_gain", "synth_inv_s", "algorithmic_bytes",
            "ROW_CHUNK", "BLOCK"]
