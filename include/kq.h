@@ -132,6 +132,27 @@ int kq_quantize_weight(const uint16_t* w, int64_t N, int64_t d, const float* par
 int kq_fold_weight(const uint16_t* w, int64_t N, int64_t d, const float* params,
                    float* w_folded, void* stream);
 
+/* Output types of kq_gemm_mxfp4. */
+enum {
+    KQ_OUT_F32 = 0,
+    KQ_OUT_BF16 = 1
+};
+
+/* W4A4 product of the transformed layer (review, "Circularity Check",
+ * Eq. 1): C = A B^T for A = kq_quantize(x) and B = kq_quantize_weight(W),
+ * so that C approximates x W^T.  On the tensor cores (block-scaled
+ * tcgen05.mma, kind::mxf4), accumulating in float32.
+ *   qa: [M][K/2] packed E2M1 codes, sa: [M][K/32] E8M0 scale bytes;
+ *   qb: [N][K/2] codes, sb: [N][K/32] scales (same layout as kq_quantize);
+ *   c:  [M][N] row-major, float32 (c_dtype KQ_OUT_F32) or bf16
+ *       (KQ_OUT_BF16, rounded to nearest even once from the float32 sum).
+ * K must be a positive multiple of 32; M and N any size up to about 2^31
+ * (M at most 128 * 65535).  qa, qb and c 16-byte aligned.  Each output is
+ * the float32 accumulation of the exact products A[m][k] B[n][k]; scale byte
+ * 0xFF (NaN) gives NaN. */
+int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
+                  int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream);
+
 /* x = y T^-1 in float32 with T^-1 = diag(G1^-1 (x) ... (x) G5^-1) (review,
  * axiom ledger: the inverse of a Kronecker product factorizes). */
 int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,

@@ -58,6 +58,9 @@ def test_bad_shapes(lib, M, d):
     assert lib.kq_transform16(FAKE, M, d, FAKE, FAKE, None) == 1
     assert lib.kq_quantize_weight(FAKE, M, d, FAKE, FAKE, FAKE, None) == 1
     assert lib.kq_fold_weight(FAKE, M, d, FAKE, FAKE, None) == 1
+    if d < 32 or d % 32:
+        assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 4, 4, d, FAKE, 0, None) == 1
+    assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, -1, 4, 64, FAKE, 0, None) == 1
 
 
 def test_null_and_misaligned_pointers(lib):
@@ -76,12 +79,18 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.kq_quantize16(FAKE, 4, 64, None, FAKE, FAKE, None) == 1
     assert lib.kq_quantize16(FAKE, 1, 32 * 65536, FAKE, FAKE, FAKE, None) == 1   # too wide
     assert lib.kq_transform16(FAKE, 4, 64, FAKE, FAKE + 8, None) == 1         # y not 16-B
+    assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 4, 4, 64, FAKE, 2, None) == 1   # dtype
+    assert lib.kq_gemm_mxfp4(FAKE + 8, FAKE, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1
+    assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 4, 4, 64, FAKE + 4, 1, None) == 1
+    assert lib.kq_gemm_mxfp4(FAKE, None, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1
+    assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 128 * 65536, 4, 64, FAKE, 0, None) == 1
 
 
 def test_empty_input_needs_no_device(lib):
     assert lib.kq_quantize(None, 0, 64, None, None, None, None) == 0
     assert lib.kq_dequantize(None, None, 0, 64, None, None) == 0
     assert lib.kq_quantize16(None, 0, 64, None, None, None, None) == 0
+    assert lib.kq_gemm_mxfp4(None, None, None, None, 0, 16, 64, None, 0, None) == 0
 
 
 def test_binding_refuses_host_tensors():

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libkq.so")
 
 KQ_OK, KQ_ERR_INVALID, KQ_ERR_CUDA, KQ_ERR_DEVICE, KQ_ERR_TIMEOUT = 0, 1, 2, 3, 4
 KQ_IMPL_AUTO, KQ_IMPL_TMA, KQ_IMPL_DIRECT, KQ_IMPL_WARP, KQ_IMPL_PANEL, KQ_IMPL_MMA = 0, 1, 2, 3, 4, 5
+KQ_OUT_F32, KQ_OUT_BF16 = 0, 1
 
 _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
@@ -34,6 +35,7 @@ SIGNATURES = {
     "kq_transform16": [_p, _i64, _i64, _p, _p, _p],
     "kq_quantize_weight": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_fold_weight": [_p, _i64, _i64, _p, _p, _p],
+    "kq_gemm_mxfp4": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p],
     "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
     "kq_quantize_host": [_p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p],
@@ -241,6 +243,33 @@ def fold_weight(w: torch.Tensor, params: torch.Tensor, out=None):
     st = lib().kq_fold_weight(w.data_ptr(), N, d, params.data_ptr(), out.data_ptr(),
                               _stream(w.device))
     _check("kq_fold_weight", st)
+    return out
+
+
+def gemm_mxfp4(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+               out=None, out_dtype=torch.float32):
+    """C = A B^T for MXFP4 operands A (codes [M, K/2], scales [M, K/32]) and
+    B (codes [N, K/2], scales [N, K/32]); C is [M, N] float32 or bf16."""
+    for t, n in ((qa, "qa"), (sa, "sa"), (qb, "qb"), (sb, "sb")):
+        _dev_tensor(t, torch.uint8, n)
+        if t.dim() != 2:
+            raise ValueError(f"{n} must be 2-D")
+    M, K = qa.shape[0], 2 * qa.shape[1]
+    N = qb.shape[0]
+    if tuple(qb.shape) != (N, K // 2) or tuple(sa.shape) != (M, K // 32) or \
+            tuple(sb.shape) != (N, K // 32):
+        raise ValueError("operand shapes must be [M, K/2], [M, K/32], [N, K/2], [N, K/32]")
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    _dev_tensor(out, out_dtype, "out")
+    if tuple(out.shape) != (M, N):
+        raise ValueError("out must be [M, N]")
+    code = KQ_OUT_F32 if out_dtype == torch.float32 else KQ_OUT_BF16
+    st = lib().kq_gemm_mxfp4(qa.data_ptr(), sa.data_ptr(), qb.data_ptr(), sb.data_ptr(), M, N, K,
+                             out.data_ptr(), code, _stream(qa.device))
+    _check("kq_gemm_mxfp4", st)
     return out
 
 

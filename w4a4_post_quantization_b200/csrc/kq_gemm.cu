@@ -1,0 +1,393 @@
+// W4A4 MXFP4 GEMM on the 5th-generation tensor cores (sm_100a):
+//
+//   C[M][N] = A[M][K] . B[N][K]^T
+//
+// with A and B as the quantizer writes them: packed E2M1 codes (element 2i
+// in the low nibble of byte i) and one E8M0 scale byte per 32 elements along
+// K, row-major.  This is the product the transformed layer computes
+// (KroQuant review, "Circularity Check", Eq. 1: A = Q(x T), B = Q(W T^-T)).
+//
+// One CTA computes a 128 x 256 tile of C and walks K in tiles of 256:
+//   warp 0      TMA: A tile [128 rows][128 B] and B tile [256 rows][128 B],
+//               128-byte swizzle, into a ring of stages
+//   warps 6, 7  scale loaders: the tile's E8M0 bytes from the row-major
+//               scale arrays into shared memory in the tensor core's scale
+//               layout (128-row x 4-scale chunks of 512 bytes: row r, scale
+//               i at byte 16 (r mod 32) + 4 (r div 32) + i)
+//   warp 1      allocates TMEM; one lane copies the stage's scales into TMEM
+//               (tcgen05.cp) and issues four block-scaled MMAs
+//               (tcgen05.mma kind::mxf4, K = 64 each) into a float32
+//               accumulator of 256 TMEM columns
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows, stores to C
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "kq.h"
+#include "kq_device.cuh"
+#include "kq_internal.h"
+#include "kq_tc.cuh"
+
+namespace kq {
+namespace {
+
+constexpr int kBM = 128;                       // UMMA M: rows of A per tile
+constexpr int kBN = 256;                       // UMMA N: rows of B per tile
+constexpr int kBK = 256;                       // K elements per stage
+constexpr int kBKBytes = kBK / 2;              // 128 bytes of codes per row
+constexpr int kMmaK = 64;                      // K elements per MMA
+constexpr int kStages = 4;
+constexpr int kATile = kBM * kBKBytes;         // 16 KiB
+constexpr int kBTile = kBN * kBKBytes;         // 32 KiB
+constexpr int kSfChunk = 512;                  // 128 rows x 4 scale bytes
+constexpr int kChunksPerStage = kBK / 128;     // 2 chunks of 4 scales per row
+constexpr int kSfaBytes = kChunksPerStage * kSfChunk;
+constexpr int kSfbBytes = kChunksPerStage * (kBN / 128) * kSfChunk;
+constexpr int kStageBytes = kATile + kBTile + kSfaBytes + kSfbBytes;
+static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
+constexpr int kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 2) * 8 + 16;
+
+constexpr int kGemmThreads = 256;
+constexpr int kSfWarp0 = 6;                    // warps 6 and 7 load scales
+constexpr int kSfThreads = 64;
+
+// TMEM: the accumulator in columns [0, 256), then per stage 4 columns per
+// scale chunk of A and 8 per chunk of B (two 128-row groups).
+constexpr int kSfColsA = 4 * kChunksPerStage;
+constexpr int kSfColsB = 8 * kChunksPerStage;
+constexpr int kSfCol0 = kBN;
+constexpr int kTmemCols = 512;
+static_assert(kSfCol0 + kStages * (kSfColsA + kSfColsB) <= kTmemCols, "TMEM columns");
+
+// Instruction descriptor, block-scaled kinds: A and B E2M1 (format 1 of
+// kind::mxf4), K-major, N = 256, E8M0 scales, M = 128, dense K = 64.  The
+// scale-factor ids (byte of the 32-bit TMEM word holding the first scale of
+// the MMA's K range) go in bits 29-30 (A) and 4-5 (B).
+constexpr uint32_t kIdescMxf4 = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (1u << 23) |
+                                (uint32_t(kBM >> 4) << 24);
+
+struct GemmArgs {
+  int32_t M, N, K;
+  int32_t k_tiles;
+  int32_t sf_stride;        // scale bytes per row: K / 32
+  int32_t out_bf16;
+  const uint8_t* sa;
+  const uint8_t* sb;
+  void* c;
+  int* err;
+};
+
+__device__ __forceinline__ void mma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                         uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
+      "\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Four scale bytes of row `row` (of `rows`) starting at scale index k0, as one
+// little-endian word; indices at or past `nsf` (and rows past the end) read
+// as 0 (2^-127, finite: those codes are zero-filled by the TMA loads).
+template <bool kAligned>
+__device__ __forceinline__ uint32_t load_sf_word(const uint8_t* s, int64_t row, int rows, int k0,
+                                                 int nsf) {
+  if (row >= rows || k0 >= nsf) return 0u;
+  const uint8_t* p = s + row * nsf + k0;
+  if (kAligned) return __ldg(reinterpret_cast<const uint32_t*>(p));
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    if (k0 + i < nsf) w |= static_cast<uint32_t>(__ldg(p + i)) << (8 * i);
+  return w;
+}
+
+// Byte offset of (row r of a 128-row group, 4-scale word) inside a chunk.
+__device__ __forceinline__ int sf_chunk_offset(int r) { return 16 * (r & 31) + 4 * (r >> 5); }
+
+template <bool kSfAligned>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap,
+                     const __grid_constant__ CUtensorMap bmap, const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* mma_done = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n0 = blockIdx.x * kBN;
+  const int m0 = blockIdx.y * kBM;
+  const int nk = a.k_tiles;
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1 + kSfThreads / 32);   // TMA bytes + one arrival per scale warp
+      mbar_init(&empty[s], 1);                     // tcgen05.commit of the stage's MMAs
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA codes
+    if (lane == 0) {
+      tma_prefetch_map(&amap);
+      tma_prefetch_map(&bmap);
+      int s = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kt = 0; kt < nk; ++kt) {
+        if (kt >= kStages && !mbar_wait(&empty[s], phase)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = base + s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], kATile + kBTile);
+        tma_load_2d(st, &amap, kt * kBKBytes, m0, &full[s]);
+        tma_load_2d(st + kATile, &bmap, kt * kBKBytes, n0, &full[s]);
+        issued = kt + 1;
+        if (++s == kStages) {
+          s = 0;
+          if (kt >= kStages) phase ^= 1;
+        }
+      }
+      if (!ok) {
+        atomicOr(a.err, kErrProducerWait);
+        for (int i = issued > kStages ? issued - kStages : 0; i < issued; ++i)
+          mbar_wait(&full[i % kStages], (i / kStages) & 1);
+      }
+    }
+    return;
+  }
+
+  if (warp >= kSfWarp0) {
+    // ---------------------------------------------------------- scale loader
+    const int t = tid - kSfWarp0 * 32;
+    int s = 0;
+    uint32_t phase = 0;
+    for (int kt = 0; kt < nk; ++kt) {
+      if (kt >= kStages && !__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], phase))) {
+        if (lane == 0) atomicOr(a.err, kErrProducerWait);
+        break;
+      }
+      uint8_t* sfa = base + s * kStageBytes + kATile + kBTile;
+      uint8_t* sfb = sfa + kSfaBytes;
+      const int kb = kt * (kBK / 32);
+      // A: 128 rows x 2 words, then B: 256 rows x 2 words; word c of a row
+      // holds scales kb + 4c .. kb + 4c + 3 (chunk c).
+      for (int w = t; w < (kBM + kBN) * kChunksPerStage; w += kSfThreads) {
+        const int c = w & 1;
+        if (w < kBM * kChunksPerStage) {
+          const int r = w >> 1;
+          const uint32_t v = load_sf_word<kSfAligned>(a.sa, (int64_t)m0 + r, a.M, kb + 4 * c,
+                                                      a.sf_stride);
+          *reinterpret_cast<uint32_t*>(sfa + c * kSfChunk + sf_chunk_offset(r)) = v;
+        } else {
+          const int r = (w - kBM * kChunksPerStage) >> 1;
+          const uint32_t v = load_sf_word<kSfAligned>(a.sb, (int64_t)n0 + r, a.N, kb + 4 * c,
+                                                      a.sf_stride);
+          *reinterpret_cast<uint32_t*>(sfb + (2 * c + (r >> 7)) * kSfChunk +
+                                       sf_chunk_offset(r & 127)) = v;
+        }
+      }
+      fence_proxy_async_smem();      // generic stores -> tcgen05.cp reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[s]);
+      if (++s == kStages) {
+        s = 0;
+        if (kt >= kStages) phase ^= 1;
+      }
+    }
+    return;
+  }
+
+  if (warp == 1) {
+    // -------------------------------------------------- scale copies + MMA
+    if (lane == 0) {
+      int s = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kt = 0; kt < nk; ++kt) {
+        if (!mbar_wait(&full[s], phase)) {
+          ok = false;
+          break;
+        }
+        tmem_fence_after();
+        const uint8_t* st = base + s * kStageBytes;
+        const uint8_t* sfa = st + kATile + kBTile;
+        const uint8_t* sfb = sfa + kSfaBytes;
+        const uint32_t tsfa = tmem_base + kSfCol0 + s * (kSfColsA + kSfColsB);
+        const uint32_t tsfb = tsfa + kSfColsA;
+#pragma unroll
+        for (int c = 0; c < kChunksPerStage; ++c) {
+          tmem_cp_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
+#pragma unroll
+          for (int g = 0; g < kBN / 128; ++g)
+            tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * g,
+                               smem_desc_rows16(smem_addr(sfb + (2 * c + g) * kSfChunk)));
+        }
+        const uint64_t adesc = smem_desc_sw128(smem_addr(st));
+        const uint64_t bdesc = smem_desc_sw128(smem_addr(st + kATile));
+#pragma unroll
+        for (int kk = 0; kk < kBK / kMmaK; ++kk) {
+          // 64 codes = 32 bytes per MMA: the start address steps by 2 (x16 B).
+          const uint32_t sf_id = 2u * (kk & 1);
+          const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
+          mma_mxf4(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
+                   tsfb + 8 * (kk >> 1), (kt | kk) != 0);
+        }
+        mma_commit(&empty[s]);         // stage (codes and scales) free once read
+        if (++s == kStages) {
+          s = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) atomicOr(a.err, kErrConsumerWait);
+      mma_commit(acc_full);
+      // Every issued MMA completes before the columns are released.
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------- epilogue
+    const int quarter = warp & 3;                  // TMEM lanes 32 quarter .. +31
+    const int row = m0 + quarter * 32 + lane;
+    const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0));
+    if (!ok) {
+      if (lane == 0) atomicOr(a.err, kErrConsumerWait);
+    } else {
+      tmem_fence_after();
+      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
+      const bool vec = (a.N & 7) == 0;
+#pragma unroll 1
+      for (int v = 0; v < kBN / 32; ++v) {
+        uint32_t r[32];
+        tmem_ld32(taddr + 32 * v, r);
+        tmem_wait_ld();
+        const int col = n0 + 32 * v;
+        if (row >= a.M || col >= a.N) continue;
+        if (a.out_bf16) {
+          __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(a.c) + (int64_t)row * a.N + col;
+          if (vec && col + 32 <= a.N) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t wv[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(r[8 * q + 2 * h]),
+                                                              __uint_as_float(r[8 * q + 2 * h + 1]));
+                wv[h] = *reinterpret_cast<const uint32_t*>(&p);
+              }
+              *reinterpret_cast<uint4*>(dst + 8 * q) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col + i < a.N) dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+          }
+        } else {
+          float* dst = static_cast<float*>(a.c) + (int64_t)row * a.N + col;
+          if (vec && col + 32 <= a.N) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<float4*>(dst + 4 * q) =
+                  make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                              __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col + i < a.N) dst[i] = __uint_as_float(r[i]);
+          }
+        }
+      }
+    }
+    tmem_fence_before();
+  }
+  // Warps 1..5 meet here; then warp 1 returns the TMEM columns.
+  asm volatile("bar.sync 2, %0;" ::"r"(5 * 32) : "memory");
+  if (warp == 1) {
+    tmem_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// Row-major packed codes [rows][K/2] as a 2-D byte tensor; a box is
+// `box_rows` rows of 128 bytes (256 codes), 128-byte swizzle.
+bool encode_codes_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t K, int box_rows) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  const cuuint32_t box[2] = {kBKBytes, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return tensor_map_encoder()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(q), dims,
+                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace kq
+
+using namespace kq;
+
+extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb,
+                             const uint8_t* sb, int64_t M, int64_t N, int64_t K, void* c,
+                             int c_dtype, void* stream) {
+  if (M < 0 || N < 0 || K < 32 || K % 32 != 0) return KQ_ERR_INVALID;
+  if (c_dtype != KQ_OUT_F32 && c_dtype != KQ_OUT_BF16) return KQ_ERR_INVALID;
+  if (M == 0 || N == 0) return KQ_OK;
+  if (M > (int64_t(1) << 31) - kBM || N > (int64_t(1) << 31) - kBN || K > (int64_t(1) << 31) - kBK)
+    return KQ_ERR_INVALID;
+  if ((M + kBM - 1) / kBM > 65535) return KQ_ERR_INVALID;
+  if (!qa || !sa || !qb || !sb || !c) return KQ_ERR_INVALID;
+  auto al = [](const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; };
+  if (!al(qa, 16) || !al(qb, 16) || !al(c, 16)) return KQ_ERR_INVALID;
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  GemmArgs a{};
+  rc = device_error_word(dev, &a.err);
+  if (rc != KQ_OK) return rc;
+  a.M = static_cast<int32_t>(M);
+  a.N = static_cast<int32_t>(N);
+  a.K = static_cast<int32_t>(K);
+  a.k_tiles = static_cast<int32_t>((K + kBK - 1) / kBK);
+  a.sf_stride = static_cast<int32_t>(K / 32);
+  a.out_bf16 = c_dtype == KQ_OUT_BF16;
+  a.sa = sa;
+  a.sb = sb;
+  a.c = c;
+  CUtensorMap amap, bmap;
+  if (!encode_codes_map(&amap, qa, M, K, kBM) || !encode_codes_map(&bmap, qb, N, K, kBN))
+    return record_cuda_error(cudaErrorInvalidValue);
+  const bool aligned4 = (a.sf_stride % 4 == 0) && al(sa, 4) && al(sb, 4);
+  const dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN),
+                  static_cast<unsigned>((M + kBM - 1) / kBM));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (aligned4) {
+    rc = allow_smem<gemm_mxf4_kernel<true>>(kSmemBytes, dev);
+    if (rc != KQ_OK) return rc;
+    gemm_mxf4_kernel<true><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
+  } else {
+    rc = allow_smem<gemm_mxf4_kernel<false>>(kSmemBytes, dev);
+    if (rc != KQ_OK) return rc;
+    gemm_mxf4_kernel<false><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return record_cuda_error(e);
+  return KQ_OK;
+}
