@@ -10,10 +10,10 @@
 // One CTA computes a 128 x 256 tile of C and walks K in tiles of 256:
 //   warp 0      TMA: A tile [128 rows][128 B] and B tile [256 rows][128 B],
 //               128-byte swizzle, into a ring of stages
-//   warps 6, 7  scale loaders: the tile's E8M0 bytes from the row-major
-//               scale arrays into shared memory in the tensor core's scale
-//               layout (128-row x 4-scale chunks of 512 bytes: row r, scale
-//               i at byte 16 (r mod 32) + 4 (r div 32) + i)
+//   warps 6..9  scale loaders, one per stage: the tile's E8M0 bytes from the
+//               row-major scale arrays into shared memory in the tensor
+//               core's scale layout (128-row x 4-scale chunks of 512 bytes:
+//               row r, scale i at byte 16 (r mod 32) + 4 (r div 32) + i)
 //   warp 1      allocates TMEM; one lane copies the stage's scales into TMEM
 //               (tcgen05.cp) and issues four block-scaled MMAs
 //               (tcgen05.mma kind::mxf4, K = 64 each) into a float32
@@ -49,9 +49,12 @@ constexpr int kStageBytes = kATile + kBTile + kSfaBytes + kSfbBytes;
 static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 2) * 8 + 16;
 
-constexpr int kGemmThreads = 256;
-constexpr int kSfWarp0 = 6;                    // warps 6 and 7 load scales
-constexpr int kSfThreads = 64;
+constexpr int kSfWarp0 = 6;                    // warps 6..9 load scales, one stage each
+constexpr int kSfWarps = kStages;
+constexpr int kGemmThreads = 32 * (kSfWarp0 + kSfWarps);
+// Scale words (4 bytes) per stage: 2 per row of A and of B.
+constexpr int kSfWordsPerStage = (kBM + kBN) * kChunksPerStage;
+constexpr int kSfWordsPerLane = kSfWordsPerStage / 32;
 
 // TMEM: the accumulator in columns [0, 256), then per stage 4 columns per
 // scale chunk of A and 8 per chunk of B (two 128-row groups).
@@ -109,6 +112,23 @@ __device__ __forceinline__ uint32_t load_sf_word(const uint8_t* s, int64_t row, 
 // Byte offset of (row r of a 128-row group, 4-scale word) inside a chunk.
 __device__ __forceinline__ int sf_chunk_offset(int r) { return 16 * (r & 31) + 4 * (r >> 5); }
 
+// This lane's scale words of k-tile kt: word w = lane + 32 i of the stage is
+// (A row w / 2, chunk w mod 2) for w < 256, then (B row (w - 256) / 2, ...).
+template <bool kAligned>
+__device__ __forceinline__ void load_sf_words(uint32_t (&v)[kSfWordsPerLane], const GemmArgs& a,
+                                              int m0, int n0, int kt, int lane) {
+  const int kb = kt * (kBK / 32);
+#pragma unroll
+  for (int i = 0; i < kSfWordsPerLane; ++i) {
+    const int w = lane + 32 * i, c = w & 1;
+    if (w < kBM * kChunksPerStage)
+      v[i] = load_sf_word<kAligned>(a.sa, (int64_t)m0 + (w >> 1), a.M, kb + 4 * c, a.sf_stride);
+    else
+      v[i] = load_sf_word<kAligned>(a.sb, (int64_t)n0 + ((w - kBM * kChunksPerStage) >> 1), a.N,
+                                    kb + 4 * c, a.sf_stride);
+  }
+}
+
 template <bool kSfAligned>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap,
@@ -128,7 +148,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1 + kSfThreads / 32);   // TMA bytes + one arrival per scale warp
+      mbar_init(&full[s], 2);                      // TMA bytes + the stage's scale warp
       mbar_init(&empty[s], 1);                     // tcgen05.commit of the stage's MMAs
     }
     mbar_init(acc_full, 1);
@@ -175,41 +195,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp >= kSfWarp0) {
     // ---------------------------------------------------------- scale loader
-    const int t = tid - kSfWarp0 * 32;
-    int s = 0;
-    uint32_t phase = 0;
-    for (int kt = 0; kt < nk; ++kt) {
-      if (kt >= kStages && !__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], phase))) {
+    // Loader warp sw owns stage sw (k-tiles sw, sw + 4, ...): it loads the
+    // scales of its next k-tile into registers while the current ones are
+    // stored, so that its global loads are always one owned stage ahead.
+    const int sw = warp - kSfWarp0;
+    const int s = sw;
+    uint8_t* sfa = base + s * kStageBytes + kATile + kBTile;
+    uint8_t* sfb = sfa + kSfaBytes;
+    uint32_t cur[kSfWordsPerLane], nxt[kSfWordsPerLane];
+    if (sw < nk) load_sf_words<kSfAligned>(cur, a, m0, n0, sw, lane);
+    for (int kt = sw, n = 0; kt < nk; kt += kStages, ++n) {
+      if (kt + kStages < nk) load_sf_words<kSfAligned>(nxt, a, m0, n0, kt + kStages, lane);
+      if (n >= 1 && !__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], (n - 1) & 1))) {
         if (lane == 0) atomicOr(a.err, kErrProducerWait);
         break;
       }
-      uint8_t* sfa = base + s * kStageBytes + kATile + kBTile;
-      uint8_t* sfb = sfa + kSfaBytes;
-      const int kb = kt * (kBK / 32);
-      // A: 128 rows x 2 words, then B: 256 rows x 2 words; word c of a row
-      // holds scales kb + 4c .. kb + 4c + 3 (chunk c).
-      for (int w = t; w < (kBM + kBN) * kChunksPerStage; w += kSfThreads) {
-        const int c = w & 1;
+#pragma unroll
+      for (int i = 0; i < kSfWordsPerLane; ++i) {
+        const int w = lane + 32 * i, c = w & 1;
         if (w < kBM * kChunksPerStage) {
           const int r = w >> 1;
-          const uint32_t v = load_sf_word<kSfAligned>(a.sa, (int64_t)m0 + r, a.M, kb + 4 * c,
-                                                      a.sf_stride);
-          *reinterpret_cast<uint32_t*>(sfa + c * kSfChunk + sf_chunk_offset(r)) = v;
+          *reinterpret_cast<uint32_t*>(sfa + c * kSfChunk + sf_chunk_offset(r)) = cur[i];
         } else {
           const int r = (w - kBM * kChunksPerStage) >> 1;
-          const uint32_t v = load_sf_word<kSfAligned>(a.sb, (int64_t)n0 + r, a.N, kb + 4 * c,
-                                                      a.sf_stride);
           *reinterpret_cast<uint32_t*>(sfb + (2 * c + (r >> 7)) * kSfChunk +
-                                       sf_chunk_offset(r & 127)) = v;
+                                       sf_chunk_offset(r & 127)) = cur[i];
         }
       }
       fence_proxy_async_smem();      // generic stores -> tcgen05.cp reads
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
-      if (++s == kStages) {
-        s = 0;
-        if (kt >= kStages) phase ^= 1;
-      }
+#pragma unroll
+      for (int i = 0; i < kSfWordsPerLane; ++i) cur[i] = nxt[i];
     }
     return;
   }
