@@ -288,6 +288,53 @@ def quantize16(x_bits: np.ndarray, params16: np.ndarray):
 
 
 # --------------------------------------------------------------------------
+# The normalization in front of the quantizer (review, "Core claim" and the
+# axiom ledger: normalization layers and AdaLN between blocks are why the
+# transform must run online; handbook page "Quantization: where diffusion
+# differs from an LLM": AdaLN multiplies timestep-dependent scales and adds
+# shifts onto the activations).  Reading: DiT's modulation
+# ``h = LN(x) (1 + scale[b]) + shift[b]``, LayerNorm over the row without an
+# affine part, row m belonging to sample ``b = m // tokens_per_sample``.
+# --------------------------------------------------------------------------
+def adaln_modulate(x64: np.ndarray, shift64: np.ndarray, scale64: np.ndarray,
+                   tokens_per_sample: int, eps: float) -> np.ndarray:
+    """``h = (x - mean) / sqrt(var + eps) * (1 + scale[b]) + shift[b]`` per
+    row, mean and (biased) variance over the row's d channels, float64."""
+    x64 = np.asarray(x64, dtype=np.float64)
+    M = x64.shape[0]
+    mu = x64.mean(axis=1, keepdims=True)
+    var = ((x64 - mu) ** 2).mean(axis=1, keepdims=True)
+    n = (x64 - mu) / np.sqrt(var + eps)
+    b = np.arange(M) // int(tokens_per_sample)
+    return n * (1.0 + np.asarray(scale64, dtype=np.float64)[b]) + \
+        np.asarray(shift64, dtype=np.float64)[b]
+
+
+def adaln_terms(x64: np.ndarray, shift64: np.ndarray, scale64: np.ndarray,
+                tokens_per_sample: int, eps: float) -> np.ndarray:
+    """``(|x| + |mean|) / sqrt(var + eps) |1 + scale[b]| + |shift[b]|``: the
+    magnitude of the terms each modulated value is made of."""
+    x64 = np.asarray(x64, dtype=np.float64)
+    M = x64.shape[0]
+    mu = x64.mean(axis=1, keepdims=True)
+    var = ((x64 - mu) ** 2).mean(axis=1, keepdims=True)
+    b = np.arange(M) // int(tokens_per_sample)
+    return (np.abs(x64) + np.abs(mu)) / np.sqrt(var + eps) * \
+        np.abs(1.0 + np.asarray(scale64, dtype=np.float64)[b]) + \
+        np.abs(np.asarray(shift64, dtype=np.float64)[b])
+
+
+def quantize_adaln(x_bits: np.ndarray, shift_bits: np.ndarray, scale_bits: np.ndarray,
+                   tokens_per_sample: int, eps: float, params: np.ndarray):
+    """MXFP4(AdaLN(x) T): bf16 bits of x ``[M, d]`` and of shift / scale
+    ``[B, d]`` -> (packed codes, scales)."""
+    h = adaln_modulate(bf16_bits_to_float64(x_bits), bf16_bits_to_float64(shift_bits),
+                       bf16_bits_to_float64(scale_bits), tokens_per_sample, eps)
+    codes, scales = mxfp4_quantize(transform(h, params))
+    return pack_codes(codes), scales
+
+
+# --------------------------------------------------------------------------
 # Weight side and the W4A4 product (review, "Circularity Check", Eq. 1:
 # ``A T (W T^-T)^T = A W^T``, the inverse folded into the weights offline)
 # --------------------------------------------------------------------------

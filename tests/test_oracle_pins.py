@@ -498,3 +498,63 @@ def test_quantize_weight_with_identity_factors_is_the_activation_quantizer():
     qa, sa = o.quantize(Wb, p)
     assert np.array_equal(sw, sa)
     assert (o.unpack_codes(qw) != o.unpack_codes(qa)).mean() < 0.01
+
+
+# ----------------------------------------------------- LayerNorm + AdaLN
+def test_adaln_without_modulation_is_torch_layer_norm():
+    """scale = shift = 0: the oracle's modulation is LayerNorm without an
+    affine part, as torch's layer_norm computes it (float64)."""
+    import torch
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((9, 96)) * 3 + 1.5
+    z = np.zeros((1, 96))
+    h = o.adaln_modulate(x, z, z, tokens_per_sample=9, eps=1e-6)
+    ref = torch.nn.functional.layer_norm(torch.from_numpy(x), (96,), eps=1e-6).numpy()
+    np.testing.assert_allclose(h, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_adaln_normalized_rows_have_zero_mean_and_known_variance():
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal((5, 64)) * 7 - 3
+    z = np.zeros((1, 64))
+    eps = 0.25
+    h = o.adaln_modulate(x, z, z, 5, eps)
+    var = x.var(axis=1)
+    np.testing.assert_allclose(h.mean(axis=1), 0, atol=1e-12)
+    np.testing.assert_allclose(h.var(axis=1), var / (var + eps), rtol=1e-12)
+
+
+def test_adaln_constant_row_gives_the_shift_and_samples_take_their_own_rows():
+    """A constant row normalizes to 0, so h = shift[b]; rows [b T, (b+1) T)
+    use sample b's shift and scale."""
+    d, T = 32, 3
+    x = np.full((7, d), 2.5)
+    shift = np.arange(3 * d, dtype=np.float64).reshape(3, d)
+    scale = np.full((3, d), 9.0)
+    h = o.adaln_modulate(x, shift, scale, T, 1e-6)
+    for m in range(7):
+        np.testing.assert_array_equal(h[m], shift[m // T])
+    # with a non-constant row the scale of its own sample applies
+    x = np.tile(np.array([1.0, -1.0] * (d // 2)), (4, 1))          # mean 0, var 1
+    scale = np.array([[0.0] * d, [1.0] * d])
+    h = o.adaln_modulate(x, np.zeros((2, d)), scale, 2, 0.0)
+    np.testing.assert_allclose(h[:2], x[:2], rtol=1e-15)
+    np.testing.assert_allclose(h[2:], 2 * x[2:], rtol=1e-15)
+
+
+def test_quantize_adaln_with_identity_factors_quantizes_the_modulated_rows():
+    """G_k = I: the fused path is MXFP4 of AdaLN(x) itself.  A row of +-1
+    (mean 0, variance 1) with scale 1, shift 0 and eps 0 gives h = +-2
+    exactly: amax 2, e = floor(log2 2) - 2 = -1 (byte 126), 2 / 2^-1 = 4 is
+    code 6, with the sign of x."""
+    d = 64
+    vals = np.array([1.0, -1.0] * (d // 2), dtype=np.float32)
+    xb = ((vals.view(np.uint32) >> 16).astype(np.uint16))[None, :]
+    one = ((np.full((1, d), 1.0, dtype=np.float32).view(np.uint32) >> 16).astype(np.uint16))
+    zero = np.zeros((1, d), dtype=np.uint16)
+    p = np.zeros((2, 5, 3), dtype=np.float32)
+    p[:, :, 1] = 1.0
+    q, s = o.quantize_adaln(xb, zero, one, 1, 0.0, p)
+    assert list(s[0]) == [126, 126]
+    codes = o.unpack_codes(q)[0]
+    assert (codes[0::2] == 6).all() and (codes[1::2] == 0xE).all()
