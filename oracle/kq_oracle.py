@@ -312,14 +312,15 @@ def adaln_modulate(x64: np.ndarray, shift64: np.ndarray, scale64: np.ndarray,
 
 def adaln_terms(x64: np.ndarray, shift64: np.ndarray, scale64: np.ndarray,
                 tokens_per_sample: int, eps: float) -> np.ndarray:
-    """``(|x| + |mean|) / sqrt(var + eps) |1 + scale[b]| + |shift[b]|``: the
-    magnitude of the terms each modulated value is made of."""
+    """``(|x| + mean(|x|)) / sqrt(var + eps) |1 + scale[b]| + |shift[b]|``:
+    the magnitude of the terms each modulated value is made of (the mean is
+    the sum of the terms ``x_i / d``, whose magnitudes add to ``mean(|x|)``)."""
     x64 = np.asarray(x64, dtype=np.float64)
     M = x64.shape[0]
     mu = x64.mean(axis=1, keepdims=True)
     var = ((x64 - mu) ** 2).mean(axis=1, keepdims=True)
     b = np.arange(M) // int(tokens_per_sample)
-    return (np.abs(x64) + np.abs(mu)) / np.sqrt(var + eps) * \
+    return (np.abs(x64) + np.abs(x64).mean(axis=1, keepdims=True)) / np.sqrt(var + eps) * \
         np.abs(1.0 + np.asarray(scale64, dtype=np.float64)[b]) + \
         np.abs(np.asarray(shift64, dtype=np.float64)[b])
 

@@ -83,6 +83,13 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.kq_gemm_mxfp4(FAKE + 8, FAKE, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1
     assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 4, 4, 64, FAKE + 4, 1, None) == 1
     assert lib.kq_gemm_mxfp4(FAKE, None, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1
+    ada = lambda *a: lib.kq_quantize_adaln(*a)
+    assert ada(FAKE, 4, 64, FAKE, FAKE, 0, 1e-6, FAKE, FAKE, FAKE, None) == 1      # tokens
+    assert ada(FAKE, 4, 64, FAKE, FAKE, 4, -1.0, FAKE, FAKE, FAKE, None) == 1      # eps
+    assert ada(FAKE, 4, 64, FAKE + 2, FAKE, 4, 1e-6, FAKE, FAKE, FAKE, None) == 1  # shift
+    assert ada(FAKE, 4, 64, FAKE, FAKE, 4, float("nan"), FAKE, FAKE, FAKE, None) == 1
+    assert ada(FAKE, 4, 32 * 385, FAKE, FAKE, 4, 1e-6, FAKE, FAKE, FAKE, None) == 1
+    assert lib.kq_transform_adaln(FAKE, 4, 64, FAKE, FAKE, 4, 1e-6, FAKE, FAKE + 8, None) == 1
     assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 128 * 65536, 4, 64, FAKE, 0, None) == 1
 
 
@@ -91,6 +98,7 @@ def test_empty_input_needs_no_device(lib):
     assert lib.kq_dequantize(None, None, 0, 64, None, None) == 0
     assert lib.kq_quantize16(None, 0, 64, None, None, None, None) == 0
     assert lib.kq_gemm_mxfp4(None, None, None, None, 0, 16, 64, None, 0, None) == 0
+    assert lib.kq_quantize_adaln(None, 0, 64, None, None, 4, 1e-6, None, None, None, None) == 0
 
 
 def test_binding_refuses_host_tensors():

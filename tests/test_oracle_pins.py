@@ -558,3 +558,15 @@ def test_quantize_adaln_with_identity_factors_quantizes_the_modulated_rows():
     assert list(s[0]) == [126, 126]
     codes = o.unpack_codes(q)[0]
     assert (codes[0::2] == 6).all() and (codes[1::2] == 0xE).all()
+
+
+def test_adaln_terms_bound_the_modulated_values():
+    """|h| <= terms everywhere (the terms are the magnitudes h is summed
+    from), with equality-level tightness on a row of one sign."""
+    rng = np.random.default_rng(33)
+    x = rng.standard_normal((6, 64)) * 4
+    shift = rng.standard_normal((2, 64))
+    scale = rng.standard_normal((2, 64))
+    h = o.adaln_modulate(x, shift, scale, 3, 1e-6)
+    t = o.adaln_terms(x, shift, scale, 3, 1e-6)
+    assert (np.abs(h) <= t * (1 + 1e-12)).all()
