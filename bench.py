@@ -74,6 +74,22 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# Dense FP4 : BF16 tensor throughput on B200, nominal (9 : 2.25 PFLOP/s).
+FP4_PER_BF16 = 4.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def measured_fp4_peak():
+    """FP4 tensor peak in TFLOP/s: the measured burst bf16 GEMM rate times
+    the nominal FP4 : BF16 ratio."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return FP4_PER_BF16 * float(json.load(f)["bf16_tflops"]), "measured bf16 x 4"
+    except (OSError, KeyError, ValueError):
+        return FP4_PER_BF16 * FALLBACK_BF16_TFLOPS, "fallback bf16 x 4"
+
+
 KERNEL_SOURCES = ("kq_kernels.cu", "kq_device.cuh")
 
 
@@ -328,6 +344,10 @@ def run_gpu(args):
     bytes16 = M * d * (2.0 + 0.5 + 1.0 / 16)
     if args.op == "kron16":
         alg_bytes = bytes16
+    # AdaLN modulation of the batch's samples (bf16 [B, d], read once per
+    # CTA and sample: not counted in the algorithmic bytes).
+    tokens = w.TOKENS_PER_SAMPLE[WORKLOAD]
+    ada_shift, ada_scale = (t.to(dev) for t in w.draw_adaln(-(-M // tokens), d, case.seed))
 
     if args.op == "kron":
         def step():
@@ -338,6 +358,9 @@ def run_gpu(args):
     elif args.op == "kron16":
         def step():
             kq.quantize16(x, p16, q, s16)
+    elif args.op == "adaln":
+        def step():
+            kq.quantize_adaln(x, ada_shift, ada_scale, tokens, params, 1e-6, q, s)
     elif args.op == "hadamard":
         def step():
             kq.quantize_hadamard(x, q, s)
@@ -381,6 +404,10 @@ def run_gpu(args):
         ms_16, _ = time_steps(lambda: kq.quantize16(x, p16, q, s16), args.steps, args.warmup,
                               stream)
         ms_max_16 = max_over_ranks(ms_16, dev)
+        ms_a, _ = time_steps(
+            lambda: kq.quantize_adaln(x, ada_shift, ada_scale, tokens, params, 1e-6, q, s),
+            args.steps, args.warmup, stream)
+        ms_max_a = max_over_ranks(ms_a, dev)
         buf = torch.empty_like(x)
         ms_c, _ = time_steps(lambda: buf.copy_(x), args.steps, args.warmup, stream)
         ms_max_c = max_over_ranks(ms_c, dev)
@@ -397,10 +424,33 @@ def run_gpu(args):
             "smooth": {"gbs": alg_bytes / (ms_max_s * 1e-3) / 1e9, "ms": ms_max_s},
             "block16": {"gbs": bytes16 / (ms_max_16 * 1e-3) / 1e9, "ms": ms_max_16,
                         "bytes_per_launch": bytes16},
+            "adaln_fused": {"gbs": alg_bytes / (ms_max_a * 1e-3) / 1e9, "ms": ms_max_a,
+                            "tokens_per_sample": tokens,
+                            "op": "LayerNorm + AdaLN modulate + transform + MXFP4, one pass"},
             "kronecker_over_smooth_speed": ms_max_s / ms_max,
             "d2d_copy_gbs": 2 * x.numel() * 2 / (ms_max_c * 1e-3) / 1e9,
         }
         del buf
+        # The layer the codes feed: C = Q(x T) Q(W T^-T)^T with a square
+        # synthetic weight (d x d), bf16 output, block-scaled tcgen05 GEMM.
+        W = w.device_randn_bf16((d, d), case.seed + 7, dev)
+        qw = torch.empty((d, d // 2), dtype=torch.uint8, device=dev)
+        sw = torch.empty((d, d // 32), dtype=torch.uint8, device=dev)
+        kq.quantize_weight(W, params, qw, sw)
+        del W
+        kq.quantize(x, params, q, s)
+        cg = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+        g_steps = max(3, min(args.steps, 40))
+        ms_g, _ = time_steps(lambda: kq.gemm_mxfp4(q, s, qw, sw, out=cg, out_dtype=torch.bfloat16),
+                             g_steps, 3, stream)
+        ms_max_g = max_over_ranks(ms_g, dev)
+        fp4_peak, fp4_src = measured_fp4_peak()
+        tflops = 2.0 * M * d * d / (ms_max_g * 1e-3) / 1e12
+        variants["w4a4_gemm"] = {
+            "shape_mnk": [M, d, d], "out": "bf16", "steps": g_steps, "ms": ms_max_g,
+            "tflops": tflops, "peak_tflops": fp4_peak, "peak_source": fp4_src,
+            "frac": tflops / fp4_peak, "kernel": "gemm_mxf4_kernel (tcgen05.mma kind::mxf4)"}
+        del qw, sw, cg
 
     # End to end through the public API: pinned host x in, pinned host codes
     # and scales out, streamed through a device workspace (kq_quantize_host).
@@ -440,7 +490,8 @@ def run_gpu(args):
                         if args.op == "kron" else None),
             "algorithmic_bytes_per_launch": alg_bytes,
             "kernel": {"kron": "panel_kernel<kron, mx4>", "kron16": "panel_kernel<kron16, mx4>",
-                       "kron_mma": "mma_kernel", "hadamard": "panel_kernel<hadamard, mx4>",
+                       "kron_mma": "mma_kernel", "adaln": "adaln_kernel<mx4>",
+                       "hadamard": "panel_kernel<hadamard, mx4>",
                        "smooth": "panel_kernel<smooth, mx4>"}[args.op],
             "kernel_source_hash": khash}
 
@@ -488,7 +539,7 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the comparator timings")
     ap.add_argument("--launch", default="eager", choices=["graph", "eager"],
                     help="time the K steps as K calls (default) or as one CUDA graph replay")
-    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "kron16", "hadamard", "smooth"],
+    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "kron16", "adaln", "hadamard", "smooth"],
                     help="quantizer timed as the step (kron = kq_quantize, the metric; "
                          "the comparators are for profiling)")
     ap.add_argument("--rows", type=int, default=0,

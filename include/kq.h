@@ -117,6 +117,27 @@ int kq_quantize16(const uint16_t* x, int64_t M, int64_t d, const float* params16
 int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
                    float* y, void* stream);
 
+/* LayerNorm + AdaLN modulation fused in front of the quantizer: the
+ * normalization that forces the transform to run online (review, "Core
+ * claim" and the axiom ledger; handbook page "Quantization: where diffusion
+ * differs from an LLM", AdaLN's per-timestep scales and shifts):
+ *   h[m][c] = (x[m][c] - mean_m) / sqrt(var_m + eps) * (1 + scale[b][c])
+ *             + shift[b][c],   b = m / tokens_per_sample,
+ * mean and biased variance over the row's d channels (LayerNorm without an
+ * affine part), then q_packed/scales = MXFP4(h T) exactly as kq_quantize
+ * (kq_transform_adaln writes h T in float32 instead).
+ *   shift, scale: bf16 [B][d], B = ceil(M / tokens_per_sample), 16-byte
+ *   aligned; tokens_per_sample >= 1; 0 <= eps (finite).
+ * d must be a positive multiple of 32 and at most 12288 (384 blocks).  The
+ * statistics are float32 (two-pass per block, combined pairwise across the
+ * row in a fixed order); h, the transform and the decision are float32. */
+int kq_quantize_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
+                      const uint16_t* scale, int64_t tokens_per_sample, float eps,
+                      const float* params, uint8_t* q_packed, uint8_t* scales, void* stream);
+int kq_transform_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
+                       const uint16_t* scale, int64_t tokens_per_sample, float eps,
+                       const float* params, float* y, void* stream);
+
 /* Weight side of the transformed layer (review, "Circularity Check", Eq. 1:
  * A T (W T^-T)^T = A W^T, the inverse folded into the weights offline).
  * w is the bf16 weight matrix [N][d] of a linear layer y = x W^T (row n holds

@@ -36,6 +36,8 @@ SIGNATURES = {
     "kq_quantize_weight": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_fold_weight": [_p, _i64, _i64, _p, _p, _p],
     "kq_gemm_mxfp4": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p],
+    "kq_quantize_adaln": [_p, _i64, _i64, _p, _p, _i64, ctypes.c_float, _p, _p, _p, _p],
+    "kq_transform_adaln": [_p, _i64, _i64, _p, _p, _i64, ctypes.c_float, _p, _p, _p],
     "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
     "kq_quantize_host": [_p, _i64, _i64, _p, _p, _p, _p, ctypes.c_size_t, _p],
@@ -271,6 +273,47 @@ def gemm_mxfp4(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.T
                              out.data_ptr(), code, _stream(qa.device))
     _check("kq_gemm_mxfp4", st)
     return out
+
+
+def _adaln_args(x, shift, scale, tokens_per_sample):
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    B = max(1, -(-M // int(tokens_per_sample)))
+    for t, n in ((shift, "shift"), (scale, "scale")):
+        _dev_tensor(t, torch.bfloat16, n)
+        if t.dim() != 2 or t.shape[1] != d or t.shape[0] < B:
+            raise ValueError(f"{n} must be bf16 [B, d] with B >= ceil(M / tokens_per_sample)")
+    return M, d
+
+
+def quantize_adaln(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
+                   tokens_per_sample: int, params: torch.Tensor, eps: float = 1e-6,
+                   q=None, scales=None):
+    """MXFP4((LN(x) (1 + scale[b]) + shift[b]) T): LayerNorm without affine,
+    AdaLN modulation per sample, transform and quantizer in one pass."""
+    M, d = _adaln_args(x, shift, scale, tokens_per_sample)
+    _, _, q, scales = _out_codes(x, q, scales)
+    _params(params, d)
+    st = lib().kq_quantize_adaln(x.data_ptr(), M, d, shift.data_ptr(), scale.data_ptr(),
+                                 int(tokens_per_sample), float(eps), params.data_ptr(),
+                                 q.data_ptr(), scales.data_ptr(), _stream(x.device))
+    _check("kq_quantize_adaln", st)
+    return q, scales
+
+
+def transform_adaln(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
+                    tokens_per_sample: int, params: torch.Tensor, eps: float = 1e-6, y=None):
+    """(LN(x) (1 + scale[b]) + shift[b]) T in float32."""
+    M, d = _adaln_args(x, shift, scale, tokens_per_sample)
+    _params(params, d)
+    if y is None:
+        y = torch.empty((M, d), dtype=torch.float32, device=x.device)
+    _dev_tensor(y, torch.float32, "y")
+    st = lib().kq_transform_adaln(x.data_ptr(), M, d, shift.data_ptr(), scale.data_ptr(),
+                                  int(tokens_per_sample), float(eps), params.data_ptr(),
+                                  y.data_ptr(), _stream(x.device))
+    _check("kq_transform_adaln", st)
+    return y
 
 
 def inverse_transform(y: torch.Tensor, params: torch.Tensor, x=None):

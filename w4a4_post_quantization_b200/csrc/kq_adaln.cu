@@ -1,0 +1,402 @@
+// LayerNorm + AdaLN modulation fused with the Kronecker transform and the
+// MXFP4 quantizer:
+//
+//   h = (x - mean) / sqrt(var + eps) * (1 + scale[b]) + shift[b],
+//   codes, scales = MXFP4(h T)
+//
+// with mean and (biased) variance over each row's d channels and row m in
+// sample b = m / tokens_per_sample.  This is the normalization that keeps
+// the transform from being folded offline (KroQuant review, "Core claim" and
+// the axiom ledger; handbook page "Quantization: where diffusion differs from
+// an LLM": AdaLN scales and shifts the activations per timestep), done in the
+// same pass that quantizes, so that x is read from HBM once.
+//
+// A CTA owns whole rows: R rows of nb = d/32 blocks per group, one thread
+// per (row, block), R = floor(384 / nb).  Each group arrives by TMA (3-D boxes
+// {32, Wb, R} of the view x[M][nb][32], 64-byte swizzle) into a ring of
+// stages; thread 0 refills a stage right after the group's statistics
+// barrier, by which every thread has read it, so no producer warp or empty
+// barrier is needed and 12 warps keep 168 registers.  Row statistics: each
+// thread's 32 values give (mean, M2); a segmented warp reduction combines the
+// lanes of the same row (Chan's pairwise rule), the head lane of each
+// segment writes a slot, and after one named barrier every thread combines
+// its row's slots in a fixed order, so the result does not depend on timing.
+// Each thread keeps its block's factors and its sample's 32 shift and 32
+// scale values (bf16 pairs) in registers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "kq.h"
+#include "kq_device.cuh"
+#include "kq_internal.h"
+#include "kq_tc.cuh"
+
+namespace kq {
+namespace {
+
+constexpr int kAdaWarps = 12;                     // 3 warps per scheduler: 168 registers
+constexpr int kAdaCons = 32 * kAdaWarps;          // threads, all consumers
+constexpr int kAdaMaxStages = 8;
+constexpr int kAdaMaxRows = 256;                  // TMA box limit on R
+constexpr int kAdaSlots = kAdaWarps + kAdaMaxRows;   // segment slots per buffer
+
+struct AdaArgs {
+  int64_t M;
+  int64_t tokens;            // rows per sample
+  int32_t nb, R, Wb, boxes;
+  int32_t groups, stages, stage_bytes, box_bytes, tx_bytes;
+  float eps;
+  const float* params;       // [nb][5][3]
+  const uint32_t* shift;     // bf16 [B][d], read as bf16 pairs
+  const uint32_t* scale;
+  uint8_t* q;
+  uint8_t* scales;
+  float* y;
+  int* err;
+};
+
+struct Moments {
+  float mean, m2, n;
+};
+
+__device__ __forceinline__ Moments combine(Moments a, Moments b) {
+  if (b.n == 0.f) return a;
+  if (a.n == 0.f) return b;
+  const float n = a.n + b.n;
+  const float delta = b.mean - a.mean;
+  const float wb = b.n / n;
+  Moments r;
+  r.mean = __fmaf_rn(delta, wb, a.mean);
+  r.m2 = a.m2 + b.m2 + delta * delta * (a.n * wb);
+  r.n = n;
+  return r;
+}
+
+// Mean and sum of squared deviations of a block's 32 values (two passes).
+__device__ __forceinline__ Moments block_moments(const f2 (&u)[16]) {
+  f2 s = u[0];
+#pragma unroll
+  for (int m = 1; m < 16; ++m) s = add2(s, u[m]);
+  float s0, s1;
+  unpack2(s, s0, s1);
+  const float mean = (s0 + s1) * (1.0f / 32.0f);
+  const f2 mean2 = pack2(mean, mean);
+  f2 q = pack2(0.f, 0.f);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const f2 dv = sub2(u[m], mean2);
+    q = fma2(dv, dv, q);
+  }
+  float q0, q1;
+  unpack2(q, q0, q1);
+  return Moments{mean, q0 + q1, 32.f};
+}
+
+__device__ __forceinline__ Moments shfl_down_moments(Moments m, int off) {
+  Moments r;
+  r.mean = __shfl_down_sync(0xFFFFFFFFu, m.mean, off);
+  r.m2 = __shfl_down_sync(0xFFFFFFFFu, m.m2, off);
+  r.n = __shfl_down_sync(0xFFFFFFFFu, m.n, off);
+  return r;
+}
+
+// Thread 0 issues the TMA load of a group into a stage.
+__device__ __forceinline__ void adaln_issue(const AdaArgs& a, const CUtensorMap* xmap,
+                                            uint8_t* stage, uint64_t* bar, int g) {
+  mbar_arrive_expect_tx(bar, a.tx_bytes);
+  for (int b = 0; b < a.boxes; ++b)
+    tma_load_3d(stage + b * a.box_bytes, xmap, 0, b * a.Wb, g * a.R, bar);
+}
+
+template <int kOut, int kForm>
+__device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMap* xmap,
+                                              uint8_t* stages, uint64_t* full, float4* slots,
+                                              int tid, const ShearDiag& sd,
+                                              const PlainFactors& pf) {
+  const int lane = tid & 31, warp = tid >> 5;
+  const int nb = a.nb, R = a.R;
+  const bool active = tid < R * nb;
+  const int rr = active ? tid / nb : R;         // inactive threads form their own "row"
+  const int j = tid - rr * nb;
+  // Byte offsets of this thread's four 16-byte chunks inside a stage: box
+  // j / Wb, line rr Wb + j mod Wb, chunk q at q ^ ((line >> 1) & 3).
+  uint32_t off[4];
+  {
+    const int line = rr * a.Wb + (j % a.Wb);
+    const uint32_t boff = (j / a.Wb) * a.box_bytes;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) off[q] = boff + line * 64 + 16 * (q ^ ((line >> 1) & 3));
+  }
+  // Segments: the lanes of a warp that share a row.  Slot of (row, warp) is
+  // warp + row, unique and increasing along the rows.
+  const int w_first = active ? (rr * nb) >> 5 : 0;
+  const int w_last = active ? ((rr + 1) * nb - 1) >> 5 : -1;
+  const int prev_rr = (tid > 0 && tid - 1 < R * nb) ? (tid - 1) / nb : -1;
+  const bool head = active && (lane == 0 || prev_rr != rr);
+  const float inv_d = 1.0f / static_cast<float>(nb * 32);
+
+  int64_t cur_b = -1;
+  uint32_t sh[16], sc[16];                        // shift / scale of block j, bf16 pairs
+  const int S = a.stages;
+  int s = 0;
+  uint32_t phase = 0;
+  int buf = 0;
+  int i = 0;                                      // groups consumed so far
+  for (int g = blockIdx.x; g < a.groups; g += gridDim.x, ++i) {
+    // A warp whose wait gives up carries on to the statistics barrier, which
+    // also ANDs the outcome, so that the CTA leaves together.
+    const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], phase));
+    const uint8_t* st = stages + s * a.stage_bytes;
+    uint4 c[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      c[q] = active ? *reinterpret_cast<const uint4*>(st + off[q]) : make_uint4(0, 0, 0, 0);
+    // Reads of the stage are ordered before the refill that follows the
+    // statistics barrier below.
+    fence_proxy_async_smem();
+    const int s_used = s;
+    if (++s == S) {
+      s = 0;
+      phase ^= 1;
+    }
+    const int64_t row = (int64_t)g * R + rr;
+    const bool live = active && row < a.M;
+    f2 u[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      u[4 * q + 0] = bf16x2_to_f2(c[q].x);
+      u[4 * q + 1] = bf16x2_to_f2(c[q].y);
+      u[4 * q + 2] = bf16x2_to_f2(c[q].z);
+      u[4 * q + 3] = bf16x2_to_f2(c[q].w);
+    }
+    if (live) {
+      const int64_t b = row / a.tokens;
+      if (b != cur_b) {
+        cur_b = b;
+        const uint4* ps = reinterpret_cast<const uint4*>(a.shift + (b * nb + j) * 16);
+        const uint4* pc = reinterpret_cast<const uint4*>(a.scale + (b * nb + j) * 16);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const uint4 vs = __ldg(ps + t), vc = __ldg(pc + t);
+          sh[4 * t] = vs.x; sh[4 * t + 1] = vs.y; sh[4 * t + 2] = vs.z; sh[4 * t + 3] = vs.w;
+          sc[4 * t] = vc.x; sc[4 * t + 1] = vc.y; sc[4 * t + 2] = vc.z; sc[4 * t + 3] = vc.w;
+        }
+      }
+    }
+    // Row statistics.  Rows past M are zero-filled by the TMA load and only
+    // need to stay finite.
+    Moments mo = active ? block_moments(u) : Moments{0.f, 0.f, 0.f};
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const Moments other = shfl_down_moments(mo, o);
+      const int other_rr = __shfl_down_sync(0xFFFFFFFFu, rr, o);
+      if (lane + o < 32 && other_rr == rr) mo = combine(mo, other);
+    }
+    float4* sl = slots + buf * kAdaSlots;
+    if (head) sl[warp + rr] = make_float4(mo.mean, mo.m2, mo.n, 0.f);
+    if (!bar_and(1, kAdaCons, got)) {
+      if (tid == 0) {
+        atomicOr(a.err, kErrConsumerWait);
+        // Let the loads still in flight land before the CTA leaves.
+        const int issued = min(i + S, (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) /
+                                          (int)gridDim.x);
+        for (int k = i; k < issued; ++k) mbar_wait(&full[k % S], (k / S) & 1);
+      }
+      return;
+    }
+    // Every thread has read stage s_used: refill it with the group S ahead.
+    if (tid == 0) {
+      const int64_t gn = (int64_t)g + (int64_t)S * gridDim.x;
+      if (gn < a.groups)
+        adaln_issue(a, xmap, stages + s_used * a.stage_bytes, &full[s_used], (int)gn);
+    }
+    Moments tot{0.f, 0.f, 0.f};
+    for (int w = w_first; w <= w_last; ++w) {
+      const float4 v = sl[w + rr];
+      tot = combine(tot, Moments{v.x, v.y, v.z});
+    }
+    buf ^= 1;
+    if (!live) continue;
+    const float rstd = 1.0f / sqrtf(__fmaf_rn(tot.m2, inv_d, a.eps));
+    const f2 mean2 = pack2(tot.mean, tot.mean), r2 = pack2(rstd, rstd);
+    const f2 one2 = pack2(1.f, 1.f);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const f2 t = mul2(sub2(u[m], mean2), r2);
+      u[m] = fma2(t, add2(bf16x2_to_f2(sc[m]), one2), bf16x2_to_f2(sh[m]));
+    }
+    if (kForm == 1) {
+      plain_apply(u, pf);
+    } else {
+      shear_apply(u, sd);
+      diag_mul(u, sd.delta);
+    }
+    const int64_t gi = row * nb + j;
+    if (kOut == 0) {
+      const Mx4Block blk = mxfp4_block(u);
+      __stcs(reinterpret_cast<uint4*>(a.q + gi * 16), blk.codes);
+      a.scales[gi] = static_cast<uint8_t>(blk.scale);
+    } else {
+      float4* dst = reinterpret_cast<float4*>(a.y + gi * 32);
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        float x0, x1, x2, x3;
+        unpack2(u[2 * t], x0, x1);
+        unpack2(u[2 * t + 1], x2, x3);
+        __stcs(dst + t, make_float4(x0, x1, x2, x3));
+      }
+    }
+  }
+}
+
+template <int kOut>
+__global__ void __launch_bounds__(kAdaCons, 1)
+    adaln_kernel(const __grid_constant__ CUtensorMap xmap, const AdaArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = base;
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + a.stages * a.stage_bytes);
+  float4* slots = reinterpret_cast<float4*>(full + 2 * kAdaMaxStages);   // 16-byte aligned
+  const int tid = threadIdx.x;
+  const int S = a.stages;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
+    tma_prefetch_map(&xmap);
+    // The first S groups of this CTA.
+    for (int s = 0; s < S; ++s) {
+      const int64_t g = (int64_t)blockIdx.x + (int64_t)s * gridDim.x;
+      if (g < a.groups) adaln_issue(a, &xmap, stages + s * a.stage_bytes, &full[s], (int)g);
+    }
+  }
+  __syncthreads();
+
+  const bool active = tid < a.R * a.nb;
+  const int j = active ? tid % a.nb : 0;
+  ShearDiag sd;
+  PlainFactors pf;
+  int plain = 0;
+  if (active) plain = load_shear_diag(sd, a.params + (int64_t)j * 15) ? 0 : 1;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(plain)
+      : "r"(plain), "r"(kAdaCons)
+      : "memory");
+  if (plain) {
+    if (active) load_plain(pf, a.params + (int64_t)j * 15);
+    adaln_consume<kOut, 1>(a, &xmap, stages, full, slots, tid, sd, pf);
+  } else {
+    adaln_consume<kOut, 0>(a, &xmap, stages, full, slots, tid, sd, pf);
+  }
+}
+
+// Launches the fused kernel; the shapes were checked by the caller.
+int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
+                 const uint16_t* scale, int64_t tokens, float eps, const float* params,
+                 uint8_t* q, uint8_t* scales, float* y, cudaStream_t st) {
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  const int nb = static_cast<int>(d / kBlock);
+  if (nb > kAdaCons) return KQ_ERR_INVALID;
+  AdaArgs a{};
+  rc = device_error_word(dev, &a.err);
+  if (rc != KQ_OK) return rc;
+  a.M = M;
+  a.tokens = tokens;
+  a.nb = nb;
+  a.R = std::min(kAdaCons / nb, kAdaMaxRows);
+  // Boxes of at most 256 blocks; the last may run past the row and is
+  // zero-filled there.
+  a.boxes = (nb + 255) / 256;
+  a.Wb = (nb + a.boxes - 1) / a.boxes;
+  const int box_raw = a.R * a.Wb * kBlock * 2;
+  a.box_bytes = (box_raw + 1023) / 1024 * 1024;
+  a.stage_bytes = a.boxes * a.box_bytes;
+  a.tx_bytes = a.boxes * box_raw;
+  const int64_t groups = (M + a.R - 1) / a.R;
+  if (M > (int64_t(1) << 31) - 1 - a.R || groups > (int64_t(1) << 30)) return KQ_ERR_INVALID;
+  a.groups = static_cast<int32_t>(groups);
+  a.eps = eps;
+  a.params = params;
+  a.shift = reinterpret_cast<const uint32_t*>(shift);
+  a.scale = reinterpret_cast<const uint32_t*>(scale);
+  a.q = q;
+  a.scales = scales;
+  a.y = y;
+  const int fixed = 1024 + 2 * kAdaMaxStages * 8 + 2 * kAdaSlots * 16;
+  a.stages = std::min(kAdaMaxStages, (di->smem_optin - fixed) / a.stage_bytes);
+  if (a.stages < 2) return KQ_ERR_INVALID;
+  const int smem = a.stages * a.stage_bytes + fixed;
+  CUtensorMap map;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBlock), static_cast<cuuint64_t>(nb),
+                              static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[2] = {kBlock * 2, static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[3] = {kBlock, static_cast<cuuint32_t>(a.Wb), static_cast<cuuint32_t>(a.R)};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult cr = tensor_map_encoder()(
+      &map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box,
+      estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) return record_cuda_error(cudaErrorInvalidValue);
+  const int grid = static_cast<int>(std::min<int64_t>(groups, di->sms));
+  if (y) {
+    rc = allow_smem<adaln_kernel<1>>(smem, dev);
+    if (rc != KQ_OK) return rc;
+    adaln_kernel<1><<<grid, kAdaCons, smem, st>>>(map, a);
+  } else {
+    rc = allow_smem<adaln_kernel<0>>(smem, dev);
+    if (rc != KQ_OK) return rc;
+    adaln_kernel<0><<<grid, kAdaCons, smem, st>>>(map, a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return record_cuda_error(e);
+  return KQ_OK;
+}
+
+}  // namespace
+}  // namespace kq
+
+using namespace kq;
+
+namespace {
+
+int check_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
+                const uint16_t* scale, int64_t tokens, float eps, const float* params) {
+  if (M < 0 || d < kBlock || d % kBlock != 0 || d / kBlock > kAdaCons) return KQ_ERR_INVALID;
+  if (M > 0 && d > (int64_t(1) << 40) / M) return KQ_ERR_INVALID;
+  if (tokens < 1 || !(eps >= 0.0f) || !(eps < 3.0e38f)) return KQ_ERR_INVALID;
+  if (M == 0) return KQ_OK;
+  if (!x || !shift || !scale || !params) return KQ_ERR_INVALID;
+  auto al = [](const void* p, uintptr_t n) { return reinterpret_cast<uintptr_t>(p) % n == 0; };
+  if (!al(x, 16) || !al(shift, 16) || !al(scale, 16) || !al(params, 4)) return KQ_ERR_INVALID;
+  return KQ_OK;
+}
+
+}  // namespace
+
+extern "C" int kq_quantize_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
+                                 const uint16_t* scale, int64_t tokens_per_sample, float eps,
+                                 const float* params, uint8_t* q_packed, uint8_t* scales,
+                                 void* stream) {
+  int rc = check_adaln(x, M, d, shift, scale, tokens_per_sample, eps, params);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!q_packed || !scales || reinterpret_cast<uintptr_t>(q_packed) % 16 != 0)
+    return KQ_ERR_INVALID;
+  return launch_adaln(x, M, d, shift, scale, tokens_per_sample, eps, params, q_packed, scales,
+                      nullptr, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int kq_transform_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
+                                  const uint16_t* scale, int64_t tokens_per_sample, float eps,
+                                  const float* params, float* y, void* stream) {
+  int rc = check_adaln(x, M, d, shift, scale, tokens_per_sample, eps, params);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!y || reinterpret_cast<uintptr_t>(y) % 16 != 0) return KQ_ERR_INVALID;
+  return launch_adaln(x, M, d, shift, scale, tokens_per_sample, eps, params, nullptr, nullptr, y,
+                      static_cast<cudaStream_t>(stream));
+}

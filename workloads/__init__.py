@@ -135,6 +135,29 @@ def draw_weight(N: int, d: int, seed: int) -> torch.Tensor:
     return torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
 
 
+# Tokens per sample of each DiT-shaped config: PixArt-Sigma 1024^2 (64 x 64
+# latent patches, batch 2), SANA 1024^2 (32 x 32, batch 4), FLUX.1-schnell
+# (4096 image + 512 text tokens, batch 1), the stress case 4 x 4096.
+TOKENS_PER_SAMPLE = {"tiny": 128, "pixart_sigma": 4096, "sana": 1024,
+                     "flux_schnell": 4608, "stress": 4096}
+
+
+def draw_adaln(B: int, d: int, seed: int):
+    """AdaLN modulation of B samples as a bf16 modulation MLP would emit it:
+    ``shift ~ N(0, 0.5)``, ``scale ~ N(0, 0.5)`` with 1 % of the channels
+    amplified (scale ``~ U(5, 30)``, channels drawn per sample), from the stream
+    ``[seed, 5]``.  Returns (shift, scale) as bf16 ``[B, d]``."""
+    rng = np.random.default_rng([seed, 5])
+    shift = rng.normal(0.0, 0.5, (B, d))
+    scale = rng.normal(0.0, 0.5, (B, d))
+    n_amp = max(1, int(round(0.01 * d)))
+    for b in range(B):
+        ch = rng.choice(d, size=n_amp, replace=False)
+        scale[b, ch] = rng.uniform(5.0, 30.0, n_amp)
+    cast = lambda v: torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
+    return cast(shift), cast(scale)
+
+
 def synth_inv_s(x: torch.Tensor) -> np.ndarray:
     """Reciprocal SmoothQuant channel scale for migration strength 0.5 and a
     unit weight range, from the column maxima of ``x`` (bf16 [M, d])."""
@@ -228,5 +251,5 @@ def algorithmic_bytes(M: int, d: int) -> float:
 
 
 __all__ = ["CONFIGS", "Case", "make_case", "case_seed", "all_case_keys", "random_bf16",
-           "bf16_from_float", "device_randn_bf16", "draw_params", "draw_params16", "draw_weight", "channel_gain", "synth_inv_s", "algorithmic_bytes",
+           "bf16_from_float", "device_randn_bf16", "draw_params", "draw_params16", "draw_weight", "draw_adaln", "TOKENS_PER_SAMPLE", "channel_gain", "synth_inv_s", "algorithmic_bytes",
            "ROW_CHUNK", "BLOCK"]
