@@ -269,13 +269,20 @@ def run_reference(args):
     return 0
 
 
-def _config(d, M, impl):
+L2_BYTES = 126e6
+
+
+def _config(d, M, impl, block=32):
+    x_mb = M * d * 2 / 1e6
     return {
         "workload": f"bandwidth stress: M={M} tokens x d={d} bf16, Student-t(3), "
                     "0.5% outlier channels x100, learned Kronecker-LU block params",
-        "M": M, "d": d, "block": 32, "format": "MXFP4 (E2M1 codes + E8M0 scale per 32)",
+        "M": M, "d": d, "block": block,
+        "format": f"MXFP4 (E2M1 codes + E8M0 scale per {block})",
         "impl": impl,
-        "l2": "inputs larger than L2 (403 MB x vs 126 MB L2); no flush",
+        "l2": (f"inputs larger than L2 ({x_mb:.0f} MB x vs 126 MB L2); no flush"
+               if M * d * 2 > L2_BYTES else
+               f"x ({x_mb:.0f} MB) fits in L2: not a bandwidth measurement"),
     }
 
 
@@ -514,7 +521,10 @@ def run_gpu(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
-            "config": dict(_config(d, M, "panel"), op=args.op,
+            "config": dict(_config(d, M, {"kron": "panel", "kron16": "panel", "hadamard": "panel",
+                                          "smooth": "panel", "kron_mma": "tcgen05 dense K",
+                                          "adaln": "fused rows"}[args.op],
+                                   16 if args.op == "kron16" else 32), op=args.op,
                            launch=("cuda_graph: the K steps captured once, replayed once"
                                    if args.launch == "graph" else "eager: one call per step"), global_batch_rows=M * world,
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3),

@@ -17,10 +17,12 @@
 // stages; thread 0 refills a stage right after the group's statistics
 // barrier, by which every thread has read it, so no producer warp or empty
 // barrier is needed and 12 warps keep 168 registers.  Row statistics: each
-// thread's 32 values give (mean, M2); a segmented warp reduction combines the
-// lanes of the same row (Chan's pairwise rule), the head lane of each
-// segment writes a slot, and after one named barrier every thread combines
-// its row's slots in a fixed order, so the result does not depend on timing.
+// thread's 32 values give a sum and a sum of squared deviations; shuffle sums
+// over the lanes of the same row in a warp (a segment) give the segment's
+// mean and, from the block means' deviations, its M2 (Chan's decomposition
+// M2 = sum M2_i + n_i (m_i - m)^2, with no divisions); the segment's first
+// lane writes a slot, and after one named barrier every thread combines its
+// row's slots in a fixed order, so the result does not depend on timing.
 // Each thread keeps its block's factors and its sample's 32 shift and 32
 // scale values (bf16 pairs) in registers.
 #include <cuda.h>
@@ -57,49 +59,42 @@ struct AdaArgs {
   int* err;
 };
 
-struct Moments {
-  float mean, m2, n;
-};
+constexpr int kAdaMaxSegs = kAdaWarps + 1;       // warps one row can touch
 
-__device__ __forceinline__ Moments combine(Moments a, Moments b) {
-  if (b.n == 0.f) return a;
-  if (a.n == 0.f) return b;
-  const float n = a.n + b.n;
-  const float delta = b.mean - a.mean;
-  const float wb = b.n / n;
-  Moments r;
-  r.mean = __fmaf_rn(delta, wb, a.mean);
-  r.m2 = a.m2 + b.m2 + delta * delta * (a.n * wb);
-  r.n = n;
-  return r;
-}
-
-// Mean and sum of squared deviations of a block's 32 values (two passes).
-__device__ __forceinline__ Moments block_moments(const f2 (&u)[16]) {
-  f2 s = u[0];
+// Sum of a block's 32 values, and of their squared deviations from the
+// block's own mean (two passes over the registers).
+__device__ __forceinline__ void block_sums(const f2 (&u)[16], float& sum, float& m2) {
+  f2 s = add2(u[0], u[1]);
 #pragma unroll
-  for (int m = 1; m < 16; ++m) s = add2(s, u[m]);
+  for (int m = 2; m < 16; m += 2) s = add2(s, add2(u[m], u[m + 1]));
   float s0, s1;
   unpack2(s, s0, s1);
-  const float mean = (s0 + s1) * (1.0f / 32.0f);
+  sum = s0 + s1;
+  const float mean = sum * (1.0f / 32.0f);
   const f2 mean2 = pack2(mean, mean);
-  f2 q = pack2(0.f, 0.f);
+  f2 q0 = pack2(0.f, 0.f), q1 = q0;
 #pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    const f2 dv = sub2(u[m], mean2);
-    q = fma2(dv, dv, q);
+  for (int m = 0; m < 16; m += 2) {
+    const f2 d0 = sub2(u[m], mean2), d1 = sub2(u[m + 1], mean2);
+    q0 = fma2(d0, d0, q0);
+    q1 = fma2(d1, d1, q1);
   }
-  float q0, q1;
-  unpack2(q, q0, q1);
-  return Moments{mean, q0 + q1, 32.f};
+  float a0, a1, b0, b1;
+  unpack2(q0, a0, a1);
+  unpack2(q1, b0, b1);
+  m2 = (a0 + a1) + (b0 + b1);
 }
 
-__device__ __forceinline__ Moments shfl_down_moments(Moments m, int off) {
-  Moments r;
-  r.mean = __shfl_down_sync(0xFFFFFFFFu, m.mean, off);
-  r.m2 = __shfl_down_sync(0xFFFFFFFFu, m.m2, off);
-  r.n = __shfl_down_sync(0xFFFFFFFFu, m.n, off);
-  return r;
+// Sum of v over this lane's segment (the lanes of the warp in the same row),
+// left in the segment's first lane: shuffle-down steps that stay inside the
+// segment (bit k of `inside` says whether lane + 2^k is in it).
+__device__ __forceinline__ float segment_sum(float v, uint32_t inside) {
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    const float o = __shfl_down_sync(0xFFFFFFFFu, v, 1 << k);
+    if (inside & (1u << k)) v += o;
+  }
+  return v;
 }
 
 // Thread 0 issues the TMA load of a group into a stage.
@@ -136,6 +131,18 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
   const int prev_rr = (tid > 0 && tid - 1 < R * nb) ? (tid - 1) / nb : -1;
   const bool head = active && (lane == 0 || prev_rr != rr);
   const float inv_d = 1.0f / static_cast<float>(nb * 32);
+  // This lane's segment: first lane, element count, and which shuffle-down
+  // distances stay inside it.
+  const int seg_lo = active ? max(32 * warp, rr * nb) : tid;
+  const int seg_hi = active ? min(32 * (warp + 1), (rr + 1) * nb) : tid + 1;
+  const int head_lane = seg_lo - 32 * warp;
+  const float seg_n = 32.0f * static_cast<float>(seg_hi - seg_lo);
+  const float inv_seg_n = 1.0f / seg_n;
+  uint32_t inside = 0;
+#pragma unroll
+  for (int k = 0; k < 5; ++k)
+    if (tid + (1 << k) < seg_hi) inside |= 1u << k;
+  const int n_slots = w_last - w_first + 1;
 
   int64_t cur_b = -1;
   uint32_t sh[16], sc[16];                        // shift / scale of block j, bf16 pairs
@@ -186,16 +193,17 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
       }
     }
     // Row statistics.  Rows past M are zero-filled by the TMA load and only
-    // need to stay finite.
-    Moments mo = active ? block_moments(u) : Moments{0.f, 0.f, 0.f};
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const Moments other = shfl_down_moments(mo, o);
-      const int other_rr = __shfl_down_sync(0xFFFFFFFFu, rr, o);
-      if (lane + o < 32 && other_rr == rr) mo = combine(mo, other);
-    }
+    // need to stay finite.  Segment sums of the block sums give the segment
+    // mean; then the block M2 plus 32 (block mean - segment mean)^2 summed
+    // over the segment is the segment's M2 (no divisions on the way).
+    float bsum = 0.f, bm2 = 0.f;
+    if (active) block_sums(u, bsum, bm2);
+    const float seg_sum = __shfl_sync(0xFFFFFFFFu, segment_sum(bsum, inside), head_lane);
+    const float seg_mean = seg_sum * inv_seg_n;
+    const float dm = __fmaf_rn(bsum, 1.0f / 32.0f, -seg_mean);
+    const float seg_m2 = segment_sum(__fmaf_rn(32.0f * dm, dm, bm2), inside);
     float4* sl = slots + buf * kAdaSlots;
-    if (head) sl[warp + rr] = make_float4(mo.mean, mo.m2, mo.n, 0.f);
+    if (head) sl[warp + rr] = make_float4(seg_mean, seg_m2, seg_n, 0.f);
     if (!bar_and(1, kAdaCons, got)) {
       if (tid == 0) {
         atomicOr(a.err, kErrConsumerWait);
@@ -212,15 +220,29 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
       if (gn < a.groups)
         adaln_issue(a, xmap, stages + s_used * a.stage_bytes, &full[s_used], (int)gn);
     }
-    Moments tot{0.f, 0.f, 0.f};
-    for (int w = w_first; w <= w_last; ++w) {
-      const float4 v = sl[w + rr];
-      tot = combine(tot, Moments{v.x, v.y, v.z});
-    }
+    // The row's segments in a fixed order: mean = sum n_k m_k / d, then
+    // M2 = sum M2_k + n_k (m_k - mean)^2.
+    const float4* rs = sl + w_first + rr;
+    float msum = 0.f;
+#pragma unroll
+    for (int k = 0; k < kAdaMaxSegs; ++k)
+      if (k < n_slots) {
+        const float2 v = *reinterpret_cast<const float2*>(&rs[k]);   // (m_k, M2_k)
+        msum = __fmaf_rn(rs[k].z, v.x, msum);
+      }
+    const float mean = msum * inv_d;
+    float m2 = 0.f;
+#pragma unroll
+    for (int k = 0; k < kAdaMaxSegs; ++k)
+      if (k < n_slots) {
+        const float4 v = rs[k];
+        const float dk = v.x - mean;
+        m2 += __fmaf_rn(v.z * dk, dk, v.y);
+      }
     buf ^= 1;
     if (!live) continue;
-    const float rstd = 1.0f / sqrtf(__fmaf_rn(tot.m2, inv_d, a.eps));
-    const f2 mean2 = pack2(tot.mean, tot.mean), r2 = pack2(rstd, rstd);
+    const float rstd = 1.0f / sqrtf(__fmaf_rn(m2, inv_d, a.eps));
+    const f2 mean2 = pack2(mean, mean), r2 = pack2(rstd, rstd);
     const f2 one2 = pack2(1.f, 1.f);
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
