@@ -43,6 +43,7 @@ constexpr int kAdaCons = 32 * kAdaWarps;          // threads, all consumers
 constexpr int kAdaMaxStages = 8;
 constexpr int kAdaMaxRows = 256;                  // TMA box limit on R
 constexpr int kAdaSlots = kAdaWarps + kAdaMaxRows;   // segment slots per buffer
+constexpr int kAdaSlotBufs = 4;
 
 struct AdaArgs {
   int64_t M;
@@ -105,11 +106,17 @@ __device__ __forceinline__ void adaln_issue(const AdaArgs& a, const CUtensorMap*
     tma_load_3d(stage + b * a.box_bytes, xmap, 0, b * a.Wb, g * a.R, bar);
 }
 
+// The loop of one thread over its CTA's groups, software-pipelined by one
+// group: the statistics of group i + 1 (slots written, arrival on a
+// statistics mbarrier) are produced before group i is normalized, so no
+// warp waits for the whole CTA inside a group.  Slots rotate through four
+// buffers, enough that a warp writing group i + 3's slots can only have got
+// there after every warp finished reading group i - 1's.
 template <int kOut, int kForm>
 __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMap* xmap,
-                                              uint8_t* stages, uint64_t* full, float4* slots,
-                                              int tid, const ShearDiag& sd,
-                                              const PlainFactors& pf) {
+                                              uint8_t* stages, uint64_t* full, uint64_t* statbar,
+                                              float4* slots, const float* delta_tab, int tid,
+                                              const ShearDiag& sd, const PlainFactors& pf) {
   const int lane = tid & 31, warp = tid >> 5;
   const int nb = a.nb, R = a.R;
   const bool active = tid < R * nb;
@@ -128,11 +135,10 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
   // warp + row, unique and increasing along the rows.
   const int w_first = active ? (rr * nb) >> 5 : 0;
   const int w_last = active ? ((rr + 1) * nb - 1) >> 5 : -1;
+  const int n_slots = w_last - w_first + 1;
   const int prev_rr = (tid > 0 && tid - 1 < R * nb) ? (tid - 1) / nb : -1;
   const bool head = active && (lane == 0 || prev_rr != rr);
   const float inv_d = 1.0f / static_cast<float>(nb * 32);
-  // This lane's segment: first lane, element count, and which shuffle-down
-  // distances stay inside it.
   const int seg_lo = active ? max(32 * warp, rr * nb) : tid;
   const int seg_hi = active ? min(32 * (warp + 1), (rr + 1) * nb) : tid + 1;
   const int head_lane = seg_lo - 32 * warp;
@@ -142,34 +148,27 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
 #pragma unroll
   for (int k = 0; k < 5; ++k)
     if (tid + (1 << k) < seg_hi) inside |= 1u << k;
-  const int n_slots = w_last - w_first + 1;
 
-  int64_t cur_b = -1;
-  uint32_t sh[16], sc[16];                        // shift / scale of block j, bf16 pairs
   const int S = a.stages;
-  int s = 0;
-  uint32_t phase = 0;
-  int buf = 0;
-  int i = 0;                                      // groups consumed so far
-  for (int g = blockIdx.x; g < a.groups; g += gridDim.x, ++i) {
-    // A warp whose wait gives up carries on to the statistics barrier, which
-    // also ANDs the outcome, so that the CTA leaves together.
-    const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(&full[s], phase));
-    const uint8_t* st = stages + s * a.stage_bytes;
-    uint4 c[4];
+  const int n_local = (int)blockIdx.x < a.groups
+                          ? (a.groups - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  int issued = min(S, n_local);                   // meaningful in thread 0
+
+  // Group k's data from its stage: waits for the TMA, reads, and orders the
+  // reads before the stage's refill.
+  auto read_group = [&](int k, uint4 (&c)[4]) -> bool {
+    const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(&full[k % S], (k / S) & 1));
+    const uint8_t* st = stages + (k % S) * a.stage_bytes;
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       c[q] = active ? *reinterpret_cast<const uint4*>(st + off[q]) : make_uint4(0, 0, 0, 0);
-    // Reads of the stage are ordered before the refill that follows the
-    // statistics barrier below.
     fence_proxy_async_smem();
-    const int s_used = s;
-    if (++s == S) {
-      s = 0;
-      phase ^= 1;
-    }
-    const int64_t row = (int64_t)g * R + rr;
-    const bool live = active && row < a.M;
+    return got;
+  };
+  // Group k's slots: segment sums of the block sums give the segment mean,
+  // then the block M2 plus 32 (block mean - segment mean)^2 summed over the
+  // segment is the segment's M2.  Rows past M hold zeros (TMA fill).
+  auto post_stats = [&](int k, const uint4 (&c)[4]) {
     f2 u[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -178,57 +177,53 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
       u[4 * q + 2] = bf16x2_to_f2(c[q].z);
       u[4 * q + 3] = bf16x2_to_f2(c[q].w);
     }
-    if (live) {
-      const int64_t b = row / a.tokens;
-      if (b != cur_b) {
-        cur_b = b;
-        const uint4* ps = reinterpret_cast<const uint4*>(a.shift + (b * nb + j) * 16);
-        const uint4* pc = reinterpret_cast<const uint4*>(a.scale + (b * nb + j) * 16);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const uint4 vs = __ldg(ps + t), vc = __ldg(pc + t);
-          sh[4 * t] = vs.x; sh[4 * t + 1] = vs.y; sh[4 * t + 2] = vs.z; sh[4 * t + 3] = vs.w;
-          sc[4 * t] = vc.x; sc[4 * t + 1] = vc.y; sc[4 * t + 2] = vc.z; sc[4 * t + 3] = vc.w;
-        }
-      }
-    }
-    // Row statistics.  Rows past M are zero-filled by the TMA load and only
-    // need to stay finite.  Segment sums of the block sums give the segment
-    // mean; then the block M2 plus 32 (block mean - segment mean)^2 summed
-    // over the segment is the segment's M2 (no divisions on the way).
     float bsum = 0.f, bm2 = 0.f;
     if (active) block_sums(u, bsum, bm2);
     const float seg_sum = __shfl_sync(0xFFFFFFFFu, segment_sum(bsum, inside), head_lane);
     const float seg_mean = seg_sum * inv_seg_n;
     const float dm = __fmaf_rn(bsum, 1.0f / 32.0f, -seg_mean);
     const float seg_m2 = segment_sum(__fmaf_rn(32.0f * dm, dm, bm2), inside);
-    float4* sl = slots + buf * kAdaSlots;
-    if (head) sl[warp + rr] = make_float4(seg_mean, seg_m2, seg_n, 0.f);
-    if (!bar_and(1, kAdaCons, got)) {
-      if (tid == 0) {
-        atomicOr(a.err, kErrConsumerWait);
-        // Let the loads still in flight land before the CTA leaves.
-        const int issued = min(i + S, (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) /
-                                          (int)gridDim.x);
-        for (int k = i; k < issued; ++k) mbar_wait(&full[k % S], (k / S) & 1);
-      }
-      return;
+    if (head) slots[(k & 3) * kAdaSlots + warp + rr] = make_float4(seg_mean, seg_m2, seg_n, 0.f);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&statbar[k & 1]);
+  };
+
+  int64_t cur_b = -1;
+  uint32_t sh[16], sc[16];                        // shift / scale of block j, bf16 pairs
+  uint4 cn[4];
+  bool ok = n_local > 0;
+  int read = 0;                                   // groups whose data arrived
+  if (ok) {
+    ok = read_group(0, cn);
+    read = ok ? 1 : 0;
+    post_stats(0, cn);
+  }
+  for (int i = 0; ok && i < n_local; ++i) {
+    uint4 cc[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) cc[q] = cn[q];
+    if (i + 1 < n_local) {
+      ok = read_group(i + 1, cn);
+      read += ok ? 1 : 0;
+      post_stats(i + 1, cn);
     }
-    // Every thread has read stage s_used: refill it with the group S ahead.
-    if (tid == 0) {
-      const int64_t gn = (int64_t)g + (int64_t)S * gridDim.x;
-      if (gn < a.groups)
-        adaln_issue(a, xmap, stages + s_used * a.stage_bytes, &full[s_used], (int)gn);
+    // Every warp has posted group i's slots and read its stage.
+    ok = __all_sync(0xFFFFFFFFu, mbar_wait(&statbar[i & 1], (i >> 1) & 1)) && ok;
+    if (!ok) break;
+    if (tid == 0 && i + S < n_local) {
+      adaln_issue(a, xmap, stages + (i % S) * a.stage_bytes, &full[i % S],
+                  (int)blockIdx.x + (i + S) * (int)gridDim.x);
+      ++issued;
     }
     // The row's segments in a fixed order: mean = sum n_k m_k / d, then
     // M2 = sum M2_k + n_k (m_k - mean)^2.
-    const float4* rs = sl + w_first + rr;
+    const float4* rs = slots + (i & 3) * kAdaSlots + w_first + rr;
     float msum = 0.f;
 #pragma unroll
     for (int k = 0; k < kAdaMaxSegs; ++k)
       if (k < n_slots) {
-        const float2 v = *reinterpret_cast<const float2*>(&rs[k]);   // (m_k, M2_k)
-        msum = __fmaf_rn(rs[k].z, v.x, msum);
+        const float4 v = rs[k];
+        msum = __fmaf_rn(v.z, v.x, msum);
       }
     const float mean = msum * inv_d;
     float m2 = 0.f;
@@ -239,21 +234,50 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
         const float dk = v.x - mean;
         m2 += __fmaf_rn(v.z * dk, dk, v.y);
       }
-    buf ^= 1;
-    if (!live) continue;
+    const int64_t row = ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * R + rr;
+    if (!active || row >= a.M) continue;
+    const int64_t b = row / a.tokens;
+    if (b != cur_b) {
+      cur_b = b;
+      const uint4* ps = reinterpret_cast<const uint4*>(a.shift + (b * nb + j) * 16);
+      const uint4* pc = reinterpret_cast<const uint4*>(a.scale + (b * nb + j) * 16);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint4 vs = __ldg(ps + t), vc = __ldg(pc + t);
+        sh[4 * t] = vs.x; sh[4 * t + 1] = vs.y; sh[4 * t + 2] = vs.z; sh[4 * t + 3] = vs.w;
+        sc[4 * t] = vc.x; sc[4 * t + 1] = vc.y; sc[4 * t + 2] = vc.z; sc[4 * t + 3] = vc.w;
+      }
+    }
     const float rstd = 1.0f / sqrtf(__fmaf_rn(m2, inv_d, a.eps));
-    const f2 mean2 = pack2(mean, mean), r2 = pack2(rstd, rstd);
+    // h = (x - mean) rstd (1 + scale) + shift, as x rstd - mean rstd, then
+    // one multiply-add with the modulation.
+    const f2 r2 = pack2(rstd, rstd), nmr2 = pack2(-mean * rstd, -mean * rstd);
     const f2 one2 = pack2(1.f, 1.f);
+    f2 u[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      u[4 * q + 0] = bf16x2_to_f2(cc[q].x);
+      u[4 * q + 1] = bf16x2_to_f2(cc[q].y);
+      u[4 * q + 2] = bf16x2_to_f2(cc[q].z);
+      u[4 * q + 3] = bf16x2_to_f2(cc[q].w);
+    }
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
-      const f2 t = mul2(sub2(u[m], mean2), r2);
+      const f2 t = fma2(u[m], r2, nmr2);
       u[m] = fma2(t, add2(bf16x2_to_f2(sc[m]), one2), bf16x2_to_f2(sh[m]));
     }
     if (kForm == 1) {
       plain_apply(u, pf);
     } else {
       shear_apply(u, sd);
-      diag_mul(u, sd.delta);
+      // The diagonal of the shear form, from the block's row of the table.
+      const float* dt = delta_tab + j * 32;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const float4 v = *reinterpret_cast<const float4*>(dt + 4 * (c8 ^ (j & 7)));
+        u[2 * c8] = mul2(u[2 * c8], pack2(v.x, v.y));
+        u[2 * c8 + 1] = mul2(u[2 * c8 + 1], pack2(v.z, v.w));
+      }
     }
     const int64_t gi = row * nb + j;
     if (kOut == 0) {
@@ -271,6 +295,12 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
       }
     }
   }
+  if (!ok) {
+    if (lane == 0) atomicOr(a.err, kErrConsumerWait);
+    // Let this CTA's loads still in flight land before it leaves.
+    if (tid == 0)
+      for (int k = read; k < issued; ++k) mbar_wait(&full[k % S], (k / S) & 1);
+  }
 }
 
 template <int kOut>
@@ -280,11 +310,15 @@ __global__ void __launch_bounds__(kAdaCons, 1)
   uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = base;
   uint64_t* full = reinterpret_cast<uint64_t*>(base + a.stages * a.stage_bytes);
-  float4* slots = reinterpret_cast<float4*>(full + 2 * kAdaMaxStages);   // 16-byte aligned
+  uint64_t* statbar = full + kAdaMaxStages;
+  float4* slots = reinterpret_cast<float4*>(statbar + 2);            // 16-byte aligned
+  float* delta_tab = reinterpret_cast<float*>(slots + kAdaSlotBufs * kAdaSlots);
   const int tid = threadIdx.x;
   const int S = a.stages;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
+    mbar_init(&statbar[0], kAdaWarps);
+    mbar_init(&statbar[1], kAdaWarps);
     fence_mbar_init();
     tma_prefetch_map(&xmap);
     // The first S groups of this CTA.
@@ -293,7 +327,6 @@ __global__ void __launch_bounds__(kAdaCons, 1)
       if (g < a.groups) adaln_issue(a, &xmap, stages + s * a.stage_bytes, &full[s], (int)g);
     }
   }
-  __syncthreads();
 
   const bool active = tid < a.R * a.nb;
   const int j = active ? tid % a.nb : 0;
@@ -301,6 +334,18 @@ __global__ void __launch_bounds__(kAdaCons, 1)
   PlainFactors pf;
   int plain = 0;
   if (active) plain = load_shear_diag(sd, a.params + (int64_t)j * 15) ? 0 : 1;
+  // The shear form's diagonal goes to a shared table (row j, 16-byte chunk
+  // c at c ^ (j mod 8), conflict-free for eight consecutive blocks).
+  if (active && tid < a.nb) {
+#pragma unroll
+    for (int c8 = 0; c8 < 8; ++c8) {
+      float d0, d1, d2, d3;
+      unpack2(sd.delta[2 * c8], d0, d1);
+      unpack2(sd.delta[2 * c8 + 1], d2, d3);
+      *reinterpret_cast<float4*>(delta_tab + j * 32 + 4 * (c8 ^ (j & 7))) =
+          make_float4(d0, d1, d2, d3);
+    }
+  }
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
       "bar.red.or.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
@@ -309,9 +354,9 @@ __global__ void __launch_bounds__(kAdaCons, 1)
       : "memory");
   if (plain) {
     if (active) load_plain(pf, a.params + (int64_t)j * 15);
-    adaln_consume<kOut, 1>(a, &xmap, stages, full, slots, tid, sd, pf);
+    adaln_consume<kOut, 1>(a, &xmap, stages, full, statbar, slots, delta_tab, tid, sd, pf);
   } else {
-    adaln_consume<kOut, 0>(a, &xmap, stages, full, slots, tid, sd, pf);
+    adaln_consume<kOut, 0>(a, &xmap, stages, full, statbar, slots, delta_tab, tid, sd, pf);
   }
 }
 
@@ -350,7 +395,8 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   a.q = q;
   a.scales = scales;
   a.y = y;
-  const int fixed = 1024 + 2 * kAdaMaxStages * 8 + 2 * kAdaSlots * 16;
+  // Barriers, four slot buffers and the diagonal table (128 bytes a block).
+  const int fixed = 1024 + (kAdaMaxStages + 2) * 8 + kAdaSlotBufs * kAdaSlots * 16 + nb * 128;
   a.stages = std::min(kAdaMaxStages, (di->smem_optin - fixed) / a.stage_bytes);
   if (a.stages < 2) return KQ_ERR_INVALID;
   const int smem = a.stages * a.stage_bytes + fixed;
