@@ -60,7 +60,6 @@ struct AdaArgs {
   int* err;
 };
 
-constexpr int kAdaMaxSegs = kAdaWarps + 1;       // warps one row can touch
 
 // Sum of a block's 32 values, and of their squared deviations from the
 // block's own mean (two passes over the registers).
@@ -148,6 +147,12 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
 #pragma unroll
   for (int k = 0; k < 5; ++k)
     if (tid + (1 << k) < seg_hi) inside |= 1u << k;
+  // Rows this warp's active lanes belong to: with at most two, the row
+  // combine runs lane-parallel (blocks per row >= 32, every DiT width).
+  const int row_lo = min((32 * warp) / nb, R - 1);
+  const int row_hi = min((32 * warp + 31) / nb, R - 1);
+  const int n_rows_here = 32 * warp < R * nb ? row_hi - row_lo + 1 : 0;
+  const bool lane_parallel = nb >= 32;
 
   const int S = a.stages;
   const int n_local = (int)blockIdx.x < a.groups
@@ -217,23 +222,42 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
     }
     // The row's segments in a fixed order: mean = sum n_k m_k / d, then
     // M2 = sum M2_k + n_k (m_k - mean)^2.
-    const float4* rs = slots + (i & 3) * kAdaSlots + w_first + rr;
-    float msum = 0.f;
+    const float4* sbuf = slots + (i & 3) * kAdaSlots;
+    float mean, m2;
+    if (lane_parallel) {
+      // Lane k takes slot k of the warp's first (then last) row; xor sums
+      // give every lane the same totals.
+      mean = 0.f;
+      m2 = 0.f;
+      for (int t = 0; t < n_rows_here; ++t) {
+        const int r = t == 0 ? row_lo : row_hi;
+        const int base = ((r * nb) >> 5) + r, cnt = (((r + 1) * nb - 1) >> 5) - ((r * nb) >> 5) + 1;
+        const float4 v = lane < cnt ? sbuf[base + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
+        float ms = v.z * v.x;
 #pragma unroll
-    for (int k = 0; k < kAdaMaxSegs; ++k)
-      if (k < n_slots) {
-        const float4 v = rs[k];
-        msum = __fmaf_rn(v.z, v.x, msum);
+        for (int o = 16; o > 0; o >>= 1) ms += __shfl_xor_sync(0xFFFFFFFFu, ms, o);
+        const float mr = ms * inv_d;
+        const float dk = v.x - mr;
+        float q = __fmaf_rn(v.z * dk, dk, v.y);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xFFFFFFFFu, q, o);
+        if (rr == r) {
+          mean = mr;
+          m2 = q;
+        }
       }
-    const float mean = msum * inv_d;
-    float m2 = 0.f;
-#pragma unroll
-    for (int k = 0; k < kAdaMaxSegs; ++k)
-      if (k < n_slots) {
+    } else {
+      const float4* rs = sbuf + w_first + rr;
+      float msum = 0.f;
+      for (int k = 0; k < n_slots; ++k) msum = __fmaf_rn(rs[k].z, rs[k].x, msum);
+      mean = msum * inv_d;
+      m2 = 0.f;
+      for (int k = 0; k < n_slots; ++k) {
         const float4 v = rs[k];
         const float dk = v.x - mean;
         m2 += __fmaf_rn(v.z * dk, dk, v.y);
       }
+    }
     const int64_t row = ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * R + rr;
     if (!active || row >= a.M) continue;
     const int64_t b = row / a.tokens;
@@ -249,10 +273,9 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
       }
     }
     const float rstd = 1.0f / sqrtf(__fmaf_rn(m2, inv_d, a.eps));
-    // h = (x - mean) rstd (1 + scale) + shift, as x rstd - mean rstd, then
-    // one multiply-add with the modulation.
+    // h = (x - mean) rstd (1 + scale) + shift, as t = x rstd - mean rstd,
+    // then h = t scale + (t + shift).
     const f2 r2 = pack2(rstd, rstd), nmr2 = pack2(-mean * rstd, -mean * rstd);
-    const f2 one2 = pack2(1.f, 1.f);
     f2 u[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -264,7 +287,7 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
       const f2 t = fma2(u[m], r2, nmr2);
-      u[m] = fma2(t, add2(bf16x2_to_f2(sc[m]), one2), bf16x2_to_f2(sh[m]));
+      u[m] = fma2(t, bf16x2_to_f2(sc[m]), add2(t, bf16x2_to_f2(sh[m])));
     }
     if (kForm == 1) {
       plain_apply(u, pf);
