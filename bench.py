@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "kq_quantize GB/s (bf16 in→MXFP4 out) and % of B200 HBM peak"
 UNIT = "GB/s"
+GEMM_METRIC = "W4A4 MXFP4 GEMM TFLOP/s on the transformed layer (M x d x d)"
 WORKLOAD = "stress"
 FALLBACK_HBM_GBS = 6650.0
 CPU_SAMPLE_ROWS = 4096
@@ -325,7 +326,7 @@ def run_gpu(args):
 
     # CPU baseline pool first (spawned, rank 0 at N=1 only).
     pool = None
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and args.op == "kron":
         pool = oracle_pool(_cpu_workers())
 
     torch.cuda.set_device(local)
@@ -356,7 +357,22 @@ def run_gpu(args):
     tokens = w.TOKENS_PER_SAMPLE[WORKLOAD]
     ada_shift, ada_scale = (t.to(dev) for t in w.draw_adaln(-(-M // tokens), d, case.seed))
 
-    if args.op == "kron":
+    gemm_flops = 2.0 * M * d * d
+    if args.op == "gemm":
+        # The layer the codes feed, as the timed step: C = Q(x T) Q(W T^-T)^T
+        # with a square synthetic weight (d x d), bf16 output.
+        Wg = w.device_randn_bf16((d, d), case.seed + 7, dev)
+        qw = torch.empty((d, d // 2), dtype=torch.uint8, device=dev)
+        sw = torch.empty((d, d // 32), dtype=torch.uint8, device=dev)
+        kq.quantize_weight(Wg, params, qw, sw)
+        del Wg
+        kq.quantize(x, params, q, s)
+        cg = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+
+    if args.op == "gemm":
+        def step():
+            kq.gemm_mxfp4(q, s, qw, sw, out=cg, out_dtype=torch.bfloat16)
+    elif args.op == "kron":
         def step():
             kq.quantize(x, params, q, s)
     elif args.op == "kron_mma":
@@ -399,6 +415,8 @@ def run_gpu(args):
     ms_max = max_over_ranks(ms, dev)
     eager_max = max_over_ranks(eager_ms, dev)
     value = aggregate_gbs(alg_bytes, world, args.steps, ms_max * args.steps)
+    if args.op == "gemm":
+        value = gemm_flops * world / (ms_max * 1e-3) / 1e12
 
     # Comparators and the copy ceiling on the same input (context, same GPU).
     variants = {}
@@ -462,7 +480,7 @@ def run_gpu(args):
     # End to end through the public API: pinned host x in, pinned host codes
     # and scales out, streamed through a device workspace (kq_quantize_host).
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.op == "kron":
         x_host = case.x.pin_memory()
         p_host = torch.from_numpy(case.params).pin_memory()
         q_host = torch.empty((M, d // 2), dtype=torch.uint8).pin_memory()
@@ -491,12 +509,20 @@ def run_gpu(args):
     peak, peak_src = measured_peak()
     per_launch_gbs = alg_bytes / (ms * 1e-3) / 1e9
     khash = kernel_source_hash()
+    if args.op == "gemm":
+        fp4_peak, fp4_src = measured_fp4_peak()
+        tf = gemm_flops / (ms * 1e-3) / 1e12
+        roof_gemm = {"bound": "tensor", "achieved": tf, "peak": fp4_peak, "unit": "TFLOP/s",
+                     "frac": tf / fp4_peak, "peak_source": fp4_src, "traffic": None,
+                     "algorithmic_flops_per_launch": gemm_flops,
+                     "kernel": "gemm_mxf4_kernel (tcgen05.mma kind::mxf4)"}
     roof = {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
             "frac": per_launch_gbs / peak, "peak_source": peak_src,
             "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.md")
                         if args.op == "kron" else None),
             "algorithmic_bytes_per_launch": alg_bytes,
             "kernel": {"kron": "panel_kernel<kron, mx4>", "kron16": "panel_kernel<kron16, mx4>",
+                       "gemm": "gemm_mxf4_kernel",
                        "kron_mma": "mma_kernel", "adaln": "adaln_kernel<mx4>",
                        "hadamard": "panel_kernel<hadamard, mx4>",
                        "smooth": "panel_kernel<smooth, mx4>"}[args.op],
@@ -513,22 +539,26 @@ def run_gpu(args):
                          f"oracle in {_cpu_workers()} spawned processes, 1 BLAS thread each, "
                          f"{sec:.2f} s wall"}
 
+    if args.op == "gemm":
+        roof = roof_gemm
     if world > 1:
         dist.barrier()
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "metric": METRIC if args.op != "gemm" else GEMM_METRIC, "value": value,
+            "unit": UNIT if args.op != "gemm" else "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
-            "config": dict(_config(d, M, {"kron": "panel", "kron16": "panel", "hadamard": "panel",
+            "dtype": "f32" if args.op != "gemm" else "mxfp4 x mxfp4, f32 accumulate",
+            "data": "synthetic",
+            "config": dict(_config(d, M, {"kron": "panel", "gemm": "tcgen05 kind::mxf4", "kron16": "panel", "hadamard": "panel",
                                           "smooth": "panel", "kron_mma": "tcgen05 dense K",
                                           "adaln": "fused rows"}[args.op],
                                    16 if args.op == "kron16" else 32), op=args.op,
                            launch=("cuda_graph: the K steps captured once, replayed once"
                                    if args.launch == "graph" else "eager: one call per step"), global_batch_rows=M * world,
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3),
-            "hbm_frac": value / world / peak,
+            "hbm_frac": value / world / peak if args.op != "gemm" else None,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": args.steps, "variants": variants,
         }
@@ -549,7 +579,7 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the comparator timings")
     ap.add_argument("--launch", default="eager", choices=["graph", "eager"],
                     help="time the K steps as K calls (default) or as one CUDA graph replay")
-    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "kron16", "adaln", "hadamard", "smooth"],
+    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "kron16", "adaln", "gemm", "hadamard", "smooth"],
                     help="quantizer timed as the step (kron = kq_quantize, the metric; "
                          "the comparators are for profiling)")
     ap.add_argument("--rows", type=int, default=0,

@@ -168,7 +168,7 @@ enum {
  *   c:  [M][N] row-major, float32 (c_dtype KQ_OUT_F32) or bf16
  *       (KQ_OUT_BF16, rounded to nearest even once from the float32 sum).
  * K must be a positive multiple of 32; M and N any size up to about 2^31
- * (M at most 128 * 65535).  qa, qb and c 16-byte aligned.  Each output is
+ * (each below 2^31 - 256).  qa, qb and c 16-byte aligned.  Each output is
  * the float32 accumulation of the exact products A[m][k] B[n][k]; scale byte
  * 0xFF (NaN) gives NaN. */
 int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,

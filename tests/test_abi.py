@@ -90,7 +90,7 @@ def test_null_and_misaligned_pointers(lib):
     assert ada(FAKE, 4, 64, FAKE, FAKE, 4, float("nan"), FAKE, FAKE, FAKE, None) == 1
     assert ada(FAKE, 4, 32 * 385, FAKE, FAKE, 4, 1e-6, FAKE, FAKE, FAKE, None) == 1
     assert lib.kq_transform_adaln(FAKE, 4, 64, FAKE, FAKE, 4, 1e-6, FAKE, FAKE + 8, None) == 1
-    assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 128 * 65536, 4, 64, FAKE, 0, None) == 1
+    assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 1 << 31, 4, 64, FAKE, 0, None) == 1
 
 
 def test_empty_input_needs_no_device(lib):

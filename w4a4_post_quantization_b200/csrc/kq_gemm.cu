@@ -52,6 +52,7 @@ constexpr int kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 2) * 8 
 constexpr int kSfWarp0 = 6;                    // warps 6..9 load scales, one stage each
 constexpr int kSfWarps = kStages;
 constexpr int kGemmThreads = 32 * (kSfWarp0 + kSfWarps);
+constexpr int kBandN = 16;                     // column tiles per raster band
 // Scale words (4 bytes) per stage: 2 per row of A and of B.
 constexpr int kSfWordsPerStage = (kBM + kBN) * kChunksPerStage;
 constexpr int kSfWordsPerLane = kSfWordsPerStage / 32;
@@ -73,7 +74,7 @@ constexpr uint32_t kIdescMxf4 = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 
 
 struct GemmArgs {
   int32_t M, N, K;
-  int32_t k_tiles;
+  int32_t k_tiles, m_tiles, n_tiles;
   int32_t sf_stride;        // scale bytes per row: K / 32
   int32_t out_bf16;
   const uint8_t* sa;
@@ -142,8 +143,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n0 = blockIdx.x * kBN;
-  const int m0 = blockIdx.y * kBM;
+  // Tile order: bands of kBandN column tiles; inside a band the row tile
+  // changes every kBandN CTAs, so a band's slice of B stays in L2 while all
+  // row tiles pass over it and each A tile is read by neighbouring CTAs.
+  int m0, n0;
+  {
+    const int t = blockIdx.x;
+    const int band = t / (kBandN * a.m_tiles);
+    const int r = t - band * kBandN * a.m_tiles;
+    const int width = min(kBandN, a.n_tiles - band * kBandN);
+    m0 = (r / width) * kBM;
+    n0 = (band * kBandN + r % width) * kBN;
+  }
   const int nk = a.k_tiles;
 
   if (tid == 0) {
@@ -368,7 +379,7 @@ extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t
   if (M == 0 || N == 0) return KQ_OK;
   if (M > (int64_t(1) << 31) - kBM || N > (int64_t(1) << 31) - kBN || K > (int64_t(1) << 31) - kBK)
     return KQ_ERR_INVALID;
-  if ((M + kBM - 1) / kBM > 65535) return KQ_ERR_INVALID;
+  if (((M + kBM - 1) / kBM) * ((N + kBN - 1) / kBN) > (int64_t(1) << 31) - 1) return KQ_ERR_INVALID;
   if (!qa || !sa || !qb || !sb || !c) return KQ_ERR_INVALID;
   auto al = [](const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; };
   if (!al(qa, 16) || !al(qb, 16) || !al(c, 16)) return KQ_ERR_INVALID;
@@ -383,6 +394,8 @@ extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t
   a.N = static_cast<int32_t>(N);
   a.K = static_cast<int32_t>(K);
   a.k_tiles = static_cast<int32_t>((K + kBK - 1) / kBK);
+  a.m_tiles = static_cast<int32_t>((M + kBM - 1) / kBM);
+  a.n_tiles = static_cast<int32_t>((N + kBN - 1) / kBN);
   a.sf_stride = static_cast<int32_t>(K / 32);
   a.out_bf16 = c_dtype == KQ_OUT_BF16;
   a.sa = sa;
@@ -392,8 +405,7 @@ extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t
   if (!encode_codes_map(&amap, qa, M, K, kBM) || !encode_codes_map(&bmap, qb, N, K, kBN))
     return record_cuda_error(cudaErrorInvalidValue);
   const bool aligned4 = (a.sf_stride % 4 == 0) && al(sa, 4) && al(sb, 4);
-  const dim3 grid(static_cast<unsigned>((N + kBN - 1) / kBN),
-                  static_cast<unsigned>((M + kBM - 1) / kBM));
+  const dim3 grid(static_cast<unsigned>(a.m_tiles * a.n_tiles));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (aligned4) {
     rc = allow_smem<gemm_mxf4_kernel<true>>(kSmemBytes, dev);
