@@ -174,6 +174,43 @@ enum {
 int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
                   int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream);
 
+/* Calibration of the transform on one linear layer (review, "What carries
+ * the argument" and the free-parameter ledger: per-layer minimization of the
+ * quantized output error plus per-operand regularization, Adam with a
+ * straight-through estimator through the quantizer).
+ *
+ * kq_transform_params_grad: for Z = X K(theta) per 32-block (K = T, or
+ * K = T^-T with inverse_transpose != 0, the weight side), the gradient of
+ * L with respect to the [d/32][5][3] parameters given
+ *   dL/dZ = g + 2 lambda (Z - Zq)   (g = dL_out/dZq, straight-through),
+ * written to dparams (float32 [d/32][5][3], overwritten), and
+ * reg = sum (Zq - Z)^2 (one float).  z, zq, g: float32 [M][d], 16-byte
+ * aligned; z must be the transform of the layer's operand at `params`
+ * (the stage inputs are recovered from it).  workspace: device memory of at
+ * least kq_transform_params_grad_workspace_bytes(M, d) bytes, 256-byte
+ * aligned, zero before its first use (each call leaves it reusable); calls
+ * sharing a workspace must be ordered.  The result is deterministic. */
+size_t kq_transform_params_grad_workspace_bytes(int64_t M, int64_t d);
+int kq_transform_params_grad(const float* z, const float* zq, const float* g, int64_t M,
+                             int64_t d, const float* params, int inverse_transpose,
+                             float lambda, float* dparams, float* reg, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* out[i] = scale (y[i] - y_ref[i]) and *sumsq = sum (y - y_ref)^2 (double,
+ * deterministic); out may alias y.  workspace as above, of
+ * kq_residual_workspace_bytes() bytes, zero before first use. */
+size_t kq_residual_workspace_bytes(void);
+int kq_residual(const float* y, const float* y_ref, int64_t n, float scale, float* out,
+                double* sumsq, void* workspace, size_t workspace_bytes, void* stream);
+
+/* One Adam step (bias-corrected; step counts from 1) on n float32
+ * parameters with gradient grad0 + grad1 (grad1 may be NULL); m and v are
+ * the float32 moment buffers, updated in place.  The hyperparameters are
+ * double so that 1 - beta is formed exactly before the float32 update. */
+int kq_adam_step(float* params, const float* grad0, const float* grad1, float* m, float* v,
+                 int64_t n, int step, double lr, double beta1, double beta2, double eps,
+                 void* stream);
+
 /* x = y T^-1 in float32 with T^-1 = diag(G1^-1 (x) ... (x) G5^-1) (review,
  * axiom ledger: the inverse of a Kronecker product factorizes). */
 int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,

@@ -36,6 +36,13 @@ SIGNATURES = {
     "kq_quantize_weight": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_fold_weight": [_p, _i64, _i64, _p, _p, _p],
     "kq_gemm_mxfp4": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p],
+    "kq_transform_params_grad_workspace_bytes": [_i64, _i64],
+    "kq_transform_params_grad": [_p, _p, _p, _i64, _i64, _p, _int, ctypes.c_float, _p, _p, _p,
+                                 ctypes.c_size_t, _p],
+    "kq_residual_workspace_bytes": [],
+    "kq_residual": [_p, _p, _i64, ctypes.c_float, _p, _p, _p, ctypes.c_size_t, _p],
+    "kq_adam_step": [_p, _p, _p, _p, _p, _i64, _int, ctypes.c_double, ctypes.c_double,
+                     ctypes.c_double, ctypes.c_double, _p],
     "kq_quantize_adaln": [_p, _i64, _i64, _p, _p, _i64, ctypes.c_float, _p, _p, _p, _p],
     "kq_transform_adaln": [_p, _i64, _i64, _p, _p, _i64, ctypes.c_float, _p, _p, _p],
     "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
@@ -50,7 +57,9 @@ SIGNATURES = {
     "kq_selftest_wait_timeout": [_p],
 }
 _RESTYPE = {"kq_status_string": ctypes.c_char_p,
-            "kq_quantize_host_workspace_bytes": ctypes.c_size_t}
+            "kq_quantize_host_workspace_bytes": ctypes.c_size_t,
+            "kq_transform_params_grad_workspace_bytes": ctypes.c_size_t,
+            "kq_residual_workspace_bytes": ctypes.c_size_t}
 
 
 class KQError(RuntimeError):
@@ -314,6 +323,73 @@ def transform_adaln(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
                                   y.data_ptr(), _stream(x.device))
     _check("kq_transform_adaln", st)
     return y
+
+
+def transform_params_grad(z: torch.Tensor, zq: torch.Tensor, g: torch.Tensor,
+                          params: torch.Tensor, inverse_transpose: bool, lam: float,
+                          workspace: torch.Tensor, dparams=None, reg=None):
+    """dL/dtheta of Z = X K(theta) (K = T, or T^-T for the weight side) with
+    dL/dZ = g + 2 lam (Z - Zq); returns (dparams [d/32, 5, 3], reg [1])."""
+    for t, n in ((z, "z"), (zq, "zq"), (g, "g")):
+        _dev_tensor(t, torch.float32, n)
+    M, d = _shape(z)
+    if zq.shape != z.shape or g.shape != z.shape:
+        raise ValueError("z, zq and g must have the same [M, d] shape")
+    _params(params, d)
+    if dparams is None:
+        dparams = torch.empty((d // 32, 5, 3), dtype=torch.float32, device=z.device)
+    if reg is None:
+        reg = torch.empty((1,), dtype=torch.float32, device=z.device)
+    _dev_tensor(workspace, torch.uint8, "workspace")
+    st = lib().kq_transform_params_grad(z.data_ptr(), zq.data_ptr(), g.data_ptr(), M, d,
+                                        params.data_ptr(), int(bool(inverse_transpose)),
+                                        float(lam), dparams.data_ptr(), reg.data_ptr(),
+                                        workspace.data_ptr(), workspace.numel(),
+                                        _stream(z.device))
+    _check("kq_transform_params_grad", st)
+    return dparams, reg
+
+
+def params_grad_workspace_bytes(M: int, d: int) -> int:
+    return int(lib().kq_transform_params_grad_workspace_bytes(M, d))
+
+
+def residual(y: torch.Tensor, y_ref: torch.Tensor, scale: float, workspace: torch.Tensor,
+             out=None, sumsq=None):
+    """(scale (y - y_ref), sum (y - y_ref)^2 as a float64 [1] tensor)."""
+    _dev_tensor(y, torch.float32, "y")
+    _dev_tensor(y_ref, torch.float32, "y_ref")
+    if y.shape != y_ref.shape:
+        raise ValueError("y and y_ref must have the same shape")
+    if out is None:
+        out = torch.empty_like(y)
+    if sumsq is None:
+        sumsq = torch.empty((1,), dtype=torch.float64, device=y.device)
+    _dev_tensor(workspace, torch.uint8, "workspace")
+    st = lib().kq_residual(y.data_ptr(), y_ref.data_ptr(), y.numel(), float(scale),
+                           out.data_ptr(), sumsq.data_ptr(), workspace.data_ptr(),
+                           workspace.numel(), _stream(y.device))
+    _check("kq_residual", st)
+    return out, sumsq
+
+
+def residual_workspace_bytes() -> int:
+    return int(lib().kq_residual_workspace_bytes())
+
+
+def adam_step(params: torch.Tensor, grad0: torch.Tensor, grad1, m: torch.Tensor,
+              v: torch.Tensor, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+              eps: float = 1e-8):
+    for t, n in ((params, "params"), (grad0, "grad0"), (m, "m"), (v, "v")):
+        _dev_tensor(t, torch.float32, n)
+    if grad1 is not None:
+        _dev_tensor(grad1, torch.float32, "grad1")
+    st = lib().kq_adam_step(params.data_ptr(), grad0.data_ptr(),
+                            grad1.data_ptr() if grad1 is not None else None, m.data_ptr(),
+                            v.data_ptr(), params.numel(), int(step), float(lr), float(beta1),
+                            float(beta2), float(eps), _stream(params.device))
+    _check("kq_adam_step", st)
+    return params
 
 
 def inverse_transform(y: torch.Tensor, params: torch.Tensor, x=None):
