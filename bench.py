@@ -568,6 +568,123 @@ def run_gpu(args):
     return 0
 
 
+# ---------------------------------------------------------- calibration leg
+CALIB_LAYER = dict(M=2048, d=1152, N=1152)   # a PixArt-Sigma-width projection
+
+
+def _calib_inputs(kind: str, seed: int):
+    """Synthetic calibration activations [M, d] (N(0, 1) rows) and an
+    N(0, 1/d) weight; ``kind`` places two outlier channels (x40 and x25) in
+    one 32-block ("inside") or 97 channels apart ("apart", the review's
+    falsifier: no 32x32 block can mix them)."""
+    import torch
+    import workloads as w
+    M, d, N = CALIB_LAYER["M"], CALIB_LAYER["d"], CALIB_LAYER["N"]
+    x = w.random_bf16((M, d), seed=seed).float()
+    chans = (37, 45) if kind == "inside" else (37, 134)
+    x[:, chans[0]] *= 40.0
+    x[:, chans[1]] *= 25.0
+    return x.to(torch.bfloat16), w.draw_weight(N, d, seed)
+
+
+def _output_loss_at(kc, x, wt, params):
+    cal = kc.LayerCalibrator(x, wt, params)
+    return cal.losses()[0]
+
+
+def _smooth_output_loss(kq, x, wt):
+    """SmoothQuant's output loss on the GPU: s_c = sqrt(max|x_c| / max|w_c|),
+    x diag(s)^-1 and W diag(s) through the per-channel quantizer, the W4A4
+    product on the tensor cores, the residual against x W^T."""
+    import torch
+    ax = x.float().abs().amax(dim=0)
+    aw = wt.float().abs().amax(dim=0)
+    s = torch.where((ax > 0) & (aw > 0), torch.sqrt(ax / aw.clamp_min(1e-30)),
+                    torch.ones_like(ax)).contiguous()
+    qa, sa = kq.quantize_smooth(x, (1.0 / s).contiguous())
+    qb, sb = kq.quantize_smooth(wt, s)
+    y = kq.gemm_mxfp4(qa, sa, qb, sb)
+    y_ref = torch.matmul(x.float(), wt.float().t())
+    ws = torch.zeros((kq.residual_workspace_bytes(),), dtype=torch.uint8, device=x.device)
+    _, ss = kq.residual(y, y_ref, 1.0, ws)
+    _, s0 = kq.residual(y_ref, torch.zeros_like(y_ref), 1.0, ws)
+    return float(ss.item()) / float(s0.item())
+
+
+def run_calibration(args):
+    """Calibration of the transform on one synthetic layer: time per Adam
+    step (the loss, its straight-through gradient and the update, all in the
+    library's kernels) and the output error it reaches, beside SmoothQuant,
+    the Hadamard initialization and no transform; with the review's two
+    falsifiers (outliers more than 32 channels apart; the learned transform
+    on jointly permuted channels)."""
+    import torch
+    import w4a4_post_quantization_b200 as kq
+    from w4a4_post_quantization_b200 import calibrate as kc
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--op calibrate runs on one GPU")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    steps = 100
+    quality = {}
+    ms_step = None
+    for kind in ("inside", "apart"):
+        x, wt = _calib_inputs(kind, seed=2026)
+        x, wt = x.to(dev), wt.to(dev)
+        nb = x.shape[1] // 32
+        ident = torch.zeros((nb, 5, 3), dtype=torch.float32, device=dev)
+        ident[:, :, 1] = 1.0
+        cal = kc.LayerCalibrator(x, wt)
+        l_init = cal.losses()[0]
+        cal.run(3)                                    # warm-up steps
+        cal = kc.LayerCalibrator(x, wt)
+        cal.losses()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        hist = cal.run(steps)
+        e1.record()
+        torch.cuda.synchronize()
+        if kind == "inside":
+            ms_step = e0.elapsed_time(e1) / steps
+        l_cal = cal.losses()[0]
+        perm = torch.randperm(x.shape[1], generator=torch.Generator().manual_seed(7)).to(dev)
+        l_perm = _output_loss_at(kc, x[:, perm].contiguous(), wt[:, perm].contiguous(),
+                                 cal.params)
+        quality[kind] = {
+            "output_mse_rel": {"no_transform": _output_loss_at(kc, x, wt, ident),
+                               "smoothquant": _smooth_output_loss(kq, x, wt),
+                               "hadamard_init": l_init, "kronecker_calibrated": l_cal,
+                               "calibrated_on_permuted_channels": l_perm},
+            "total_loss_first_last": [hist[0], hist[-1]]}
+    M, d, N = CALIB_LAYER["M"], CALIB_LAYER["d"], CALIB_LAYER["N"]
+    cpu = None
+    if not args.no_cpu_baseline:
+        import numpy as np
+        from oracle import kq_calibration as oc
+        from oracle import kq_oracle as oo
+        x, wt = _calib_inputs("inside", seed=2026)
+        bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+        x64, w64 = oo.bf16_bits_to_float64(bits(x)), oo.bf16_bits_to_float64(bits(wt))
+        t0 = time.perf_counter()
+        oc.calibrate(x64, w64, steps=2)
+        sec = (time.perf_counter() - t0) / 2
+        cpu = {"value": 1000.0 * sec, "unit": "ms per step", "cores": 1, "kind": "oracle",
+               "sample": f"2 Adam steps of the float64 oracle on the same {M}x{d}x{N} layer"}
+    line = {
+        "metric": "transform calibration: ms per Adam step (loss, straight-through "
+                  "gradient, update)", "value": ms_step, "unit": "ms", "n_gpus": 1,
+        "steps": steps, "warmup": 3, "higher_is_better": False, "data": "synthetic",
+        "config": {"workload": f"one linear layer M={M} tokens x d={d} -> N={N}, "
+                               "N(0,1) activations with two outlier channels (x40, x25), "
+                               "N(0,1/d) weight; Hadamard init, Adam lr 1e-2",
+                   **CALIB_LAYER},
+        "quality": quality, "cpu_baseline": cpu, "dtype": "f32", "vs_baseline": None}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -579,7 +696,8 @@ def main(argv=None):
     ap.add_argument("--quick", action="store_true", help="skip the comparator timings")
     ap.add_argument("--launch", default="eager", choices=["graph", "eager"],
                     help="time the K steps as K calls (default) or as one CUDA graph replay")
-    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "kron16", "adaln", "gemm", "hadamard", "smooth"],
+    ap.add_argument("--op", default="kron", choices=["kron", "kron_mma", "kron16", "adaln", "gemm", "calibrate", "hadamard",
+                             "smooth"],
                     help="quantizer timed as the step (kron = kq_quantize, the metric; "
                          "the comparators are for profiling)")
     ap.add_argument("--rows", type=int, default=0,
@@ -590,6 +708,8 @@ def main(argv=None):
         raise SystemExit("--warmup must be at least 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.op == "calibrate":
+        return run_calibration(args)
     return run_gpu(args)
 
 
