@@ -396,3 +396,36 @@ def abs_inverse_transform(y64: np.ndarray, params: np.ndarray) -> np.ndarray:
 
 
 PARAMS_PER_BLOCK = 3 * N_FACTORS          # three scalars per 2x2 factor
+
+
+# --------------------------------------------------------------------------
+# Scale layout the block-scaled tensor-core product reads (a data movement,
+# no arithmetic): 128-row x 4-scale tiles of 512 bytes, row-tile major then
+# K; inside a tile row r = r0 + 32 r1, scale i at byte 16 r0 + 4 r1 + i.
+# Rows are padded to 128 and scale columns to 4 with zero bytes.
+# --------------------------------------------------------------------------
+def scales_to_mma(scales: np.ndarray) -> np.ndarray:
+    """Row-major scale bytes ``[rows, K/32]`` -> the tiled layout (1-D)."""
+    scales = np.asarray(scales, dtype=np.uint8)
+    rows, ns = scales.shape
+    rt, ct = -(-rows // 128), -(-ns // 4)
+    out = np.zeros(rt * ct * 512, dtype=np.uint8)
+    for r in range(rows):
+        for k in range(ns):
+            tile = (r // 128) * ct + k // 4
+            rr = r % 128
+            out[tile * 512 + 16 * (rr % 32) + 4 * (rr // 32) + k % 4] = scales[r, k]
+    return out
+
+
+def scales_from_mma(tiled: np.ndarray, rows: int, ns: int) -> np.ndarray:
+    """Inverse of ``scales_to_mma`` for ``rows`` rows of ``ns`` scales."""
+    tiled = np.asarray(tiled, dtype=np.uint8)
+    ct = -(-ns // 4)
+    out = np.empty((rows, ns), dtype=np.uint8)
+    for r in range(rows):
+        for k in range(ns):
+            rr = r % 128
+            out[r, k] = tiled[((r // 128) * ct + k // 4) * 512 + 16 * (rr % 32) + 4 * (rr // 32) +
+                              k % 4]
+    return out

@@ -570,3 +570,25 @@ def test_adaln_terms_bound_the_modulated_values():
     h = o.adaln_modulate(x, shift, scale, 3, 1e-6)
     t = o.adaln_terms(x, shift, scale, 3, 1e-6)
     assert (np.abs(h) <= t * (1 + 1e-12)).all()
+
+
+# ------------------------------------------------ tensor-core scale layout
+def test_scales_to_mma_places_every_byte_once_and_pads_with_zero():
+    rows, ns = 130, 6                          # two row tiles, two scale tiles
+    s = (np.arange(rows * ns) % 251 + 1).astype(np.uint8).reshape(rows, ns)
+    t = o.scales_to_mma(s)
+    assert t.size == 2 * 2 * 512
+    assert np.count_nonzero(t) == rows * ns    # every (nonzero) byte once, padding zero
+    np.testing.assert_array_equal(o.scales_from_mma(t, rows, ns), s)
+
+
+def test_scales_to_mma_hand_positions():
+    """Row 33 (r0 = 1, r1 = 1), scale 5 (tile column 1, i = 1) of a 1-tile-
+    high array with 8 scale columns: tile 1, byte 16 + 4 + 1 = 21."""
+    s = np.zeros((40, 8), dtype=np.uint8)
+    s[33, 5] = 7
+    t = o.scales_to_mma(s)
+    assert np.flatnonzero(t).tolist() == [512 + 21]
+    s = np.zeros((300, 4), dtype=np.uint8)
+    s[256 + 100, 2] = 9                        # tile row 2: r0 = 4, r1 = 3
+    assert np.flatnonzero(o.scales_to_mma(s)).tolist() == [2 * 512 + 16 * 4 + 4 * 3 + 2]
