@@ -589,6 +589,6 @@ def test_scales_to_mma_hand_positions():
     s[33, 5] = 7
     t = o.scales_to_mma(s)
     assert np.flatnonzero(t).tolist() == [512 + 21]
-    s = np.zeros((300, 4), dtype=np.uint8)
+    s = np.zeros((400, 4), dtype=np.uint8)
     s[256 + 100, 2] = 9                        # tile row 2: r0 = 4, r1 = 3
     assert np.flatnonzero(o.scales_to_mma(s)).tolist() == [2 * 512 + 16 * 4 + 4 * 3 + 2]
