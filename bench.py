@@ -360,18 +360,17 @@ def run_gpu(args):
     gemm_flops = 2.0 * M * d * d
     if args.op == "gemm":
         # The layer the codes feed, as the timed step: C = Q(x T) Q(W T^-T)^T
-        # with a square synthetic weight (d x d), bf16 output.
+        # with a square synthetic weight (d x d), bf16 output; both
+        # quantizers write their scales in the tensor cores' tiled layout.
         Wg = w.device_randn_bf16((d, d), case.seed + 7, dev)
-        qw = torch.empty((d, d // 2), dtype=torch.uint8, device=dev)
-        sw = torch.empty((d, d // 32), dtype=torch.uint8, device=dev)
-        kq.quantize_weight(Wg, params, qw, sw)
+        qw, sw = kq.quantize_weight_tiled(Wg, params)
         del Wg
-        kq.quantize(x, params, q, s)
+        qt, st_ = kq.quantize_tiled(x, params)
         cg = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
 
     if args.op == "gemm":
         def step():
-            kq.gemm_mxfp4(q, s, qw, sw, out=cg, out_dtype=torch.bfloat16)
+            kq.gemm_mxfp4_tiled(qt, st_, qw, sw, out=cg, out_dtype=torch.bfloat16)
     elif args.op == "kron":
         def step():
             kq.quantize(x, params, q, s)
@@ -459,23 +458,23 @@ def run_gpu(args):
         # The layer the codes feed: C = Q(x T) Q(W T^-T)^T with a square
         # synthetic weight (d x d), bf16 output, block-scaled tcgen05 GEMM.
         W = w.device_randn_bf16((d, d), case.seed + 7, dev)
-        qw = torch.empty((d, d // 2), dtype=torch.uint8, device=dev)
-        sw = torch.empty((d, d // 32), dtype=torch.uint8, device=dev)
-        kq.quantize_weight(W, params, qw, sw)
+        qw, sw = kq.quantize_weight_tiled(W, params)
         del W
-        kq.quantize(x, params, q, s)
+        qt, st_ = kq.quantize_tiled(x, params)
         cg = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
         g_steps = max(3, min(args.steps, 40))
-        ms_g, _ = time_steps(lambda: kq.gemm_mxfp4(q, s, qw, sw, out=cg, out_dtype=torch.bfloat16),
-                             g_steps, 3, stream)
+        ms_g, _ = time_steps(
+            lambda: kq.gemm_mxfp4_tiled(qt, st_, qw, sw, out=cg, out_dtype=torch.bfloat16),
+            g_steps, 3, stream)
         ms_max_g = max_over_ranks(ms_g, dev)
         fp4_peak, fp4_src = measured_fp4_peak()
         tflops = 2.0 * M * d * d / (ms_max_g * 1e-3) / 1e12
         variants["w4a4_gemm"] = {
             "shape_mnk": [M, d, d], "out": "bf16", "steps": g_steps, "ms": ms_max_g,
             "tflops": tflops, "peak_tflops": fp4_peak, "peak_source": fp4_src,
-            "frac": tflops / fp4_peak, "kernel": "gemm_mxf4_kernel (tcgen05.mma kind::mxf4)"}
-        del qw, sw, cg
+            "frac": tflops / fp4_peak,
+            "kernel": "gemm_mxf4_kernel<tiled scales> (tcgen05.mma kind::mxf4)"}
+        del qw, sw, cg, qt, st_
 
     # End to end through the public API: pinned host x in, pinned host codes
     # and scales out, streamed through a device workspace (kq_quantize_host).
@@ -515,7 +514,7 @@ def run_gpu(args):
         roof_gemm = {"bound": "tensor", "achieved": tf, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": tf / fp4_peak, "peak_source": fp4_src, "traffic": None,
                      "algorithmic_flops_per_launch": gemm_flops,
-                     "kernel": "gemm_mxf4_kernel (tcgen05.mma kind::mxf4)"}
+                     "kernel": "gemm_mxf4_kernel<tiled scales> (tcgen05.mma kind::mxf4)"}
     roof = {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
             "frac": per_launch_gbs / peak, "peak_source": peak_src,
             "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.md")

@@ -211,6 +211,38 @@ int kq_adam_step(float* params, const float* grad0, const float* grad1, float* m
                  int64_t n, int step, double lr, double beta1, double beta2, double eps,
                  void* stream);
 
+/* The same product with both scale arrays in the tiled layout the tensor
+ * cores read: 128-row x 4-scale tiles of 512 bytes, row-tile major then
+ * along K; inside a tile row r = r0 + 32 r1 (r0 < 32, r1 < 4) and scale i
+ * (< 4) sit at byte 16 r0 + 4 r1 + i; rows are padded to a multiple of 128
+ * and the K/32 scales of a row to a multiple of 4 (zero bytes).  sa_tiled:
+ * kq_scales_tiled_bytes(M, K) bytes, sb_tiled: kq_scales_tiled_bytes(N, K),
+ * both 16-byte aligned.  The scale tiles reach the GEMM as whole bulk
+ * copies, which is faster than gathering row-major scale bytes. */
+int kq_gemm_mxfp4_tiled(const uint8_t* qa, const uint8_t* sa_tiled, const uint8_t* qb,
+                        const uint8_t* sb_tiled, int64_t M, int64_t N, int64_t K, void* c,
+                        int c_dtype, void* stream);
+
+/* Bytes of the tiled scale layout for `rows` rows of K/32 scales (0 for an
+ * invalid K or rows < 1). */
+size_t kq_scales_tiled_bytes(int64_t rows, int64_t K);
+
+/* kq_quantize and kq_quantize_weight with the scale bytes written straight
+ * into the tiled layout above (scales_tiled: kq_scales_tiled_bytes(M, d)
+ * bytes).  Every real entry and the padding of each row's last 4-scale
+ * column are written; the padding rows of the last 128-row tile are not
+ * (they only meet zero-filled code rows in the product).  Codes as for the
+ * row-major entry points. */
+int kq_quantize_tiled(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                      uint8_t* q_packed, uint8_t* scales_tiled, void* stream);
+int kq_quantize_weight_tiled(const uint16_t* w, int64_t N, int64_t d, const float* params,
+                             uint8_t* q_packed, uint8_t* scales_tiled, void* stream);
+
+/* Row-major scales [rows][K/32] -> the tiled layout above (tiled: 16-byte
+ * aligned, kq_scales_tiled_bytes(rows, K) bytes, padding written as 0). */
+int kq_scales_to_tiled(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* tiled,
+                       void* stream);
+
 /* x = y T^-1 in float32 with T^-1 = diag(G1^-1 (x) ... (x) G5^-1) (review,
  * axiom ledger: the inverse of a Kronecker product factorizes). */
 int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,

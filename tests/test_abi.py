@@ -83,6 +83,11 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.kq_gemm_mxfp4(FAKE + 8, FAKE, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1
     assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 4, 4, 64, FAKE + 4, 1, None) == 1
     assert lib.kq_gemm_mxfp4(FAKE, None, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1
+    assert lib.kq_gemm_mxfp4_tiled(FAKE, FAKE + 4, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1
+    assert lib.kq_gemm_mxfp4_tiled(FAKE, FAKE, FAKE, FAKE, 4, 4, 48, FAKE, 0, None) == 1
+    assert lib.kq_scales_to_tiled(FAKE, 4, 48, FAKE, None) == 1
+    assert lib.kq_scales_to_tiled(FAKE, 4, 64, FAKE + 4, None) == 1
+    assert lib.kq_scales_tiled_bytes(0, 64) == 0 and lib.kq_scales_tiled_bytes(130, 544) == 2 * 5 * 512
     ada = lambda *a: lib.kq_quantize_adaln(*a)
     assert ada(FAKE, 4, 64, FAKE, FAKE, 0, 1e-6, FAKE, FAKE, FAKE, None) == 1      # tokens
     assert ada(FAKE, 4, 64, FAKE, FAKE, 4, -1.0, FAKE, FAKE, FAKE, None) == 1      # eps

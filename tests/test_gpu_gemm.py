@@ -149,3 +149,53 @@ def test_gemm_empty_and_device_status():
     sb = torch.zeros((16, 2), dtype=torch.uint8, device=DEV)
     assert kq.gemm_mxfp4(qa, sa, qb, sb).shape == (0, 16)
     assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("rows,K", [(1, 32), (130, 544), (300, 2240), (256, 12288)])
+def test_scales_to_tiled_matches_the_oracle(rows, K):
+    s = np.random.default_rng(rows + K).integers(0, 255, (rows, K // 32), dtype=np.uint8)
+    t = kq.scales_to_tiled(_dev(s), K)
+    torch.cuda.synchronize()
+    assert np.array_equal(t.cpu().numpy(), o.scales_to_mma(s))
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (130, 300, 544), (1, 8, 32),
+                                   (257, 520, 1152), (64, 40, 2240), (300, 256, 96)])
+def test_tiled_scales_give_the_same_product(M, N, K):
+    """The tiled-scale kernel reads the same codes and scales and runs the
+    same MMAs: its output equals the row-major kernel's bit for bit, and the
+    oracle's product within the tolerance."""
+    qa, sa, qb, sb = random_operands(M, N, K, seed=M * 5 + N + K)
+    c_row = run(qa, sa, qb, sb)
+    c_tiled = kq.gemm_mxfp4_tiled(_dev(qa), kq.scales_to_tiled(_dev(sa), K), _dev(qb),
+                                  kq.scales_to_tiled(_dev(sb), K))
+    torch.cuda.synchronize()
+    assert torch.equal(c_row, c_tiled)
+    check_gemm(c_tiled.cpu().numpy(), qa, sa, qb, sb)
+    c16 = kq.gemm_mxfp4_tiled(_dev(qa), kq.scales_to_tiled(_dev(sa), K), _dev(qb),
+                              kq.scales_to_tiled(_dev(sb), K), out_dtype=torch.bfloat16)
+    assert torch.equal(c16, c_tiled.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("name,di,N", [("pixart_sigma", 0, 1152), ("sana", 0, 2240),
+                                       ("flux_schnell", 0, 3072)], ids=lambda v: str(v))
+def test_quantizers_write_the_tiled_layout(name, di, N):
+    """kq_quantize_tiled / kq_quantize_weight_tiled give the same codes as
+    the row-major quantizers and the tiled image of their scales (padding
+    of each row's last 4-scale column zero); the layer's product through
+    them equals the row-major product bit for bit."""
+    c = w.make_case(name, di, 0, M=192)
+    W = w.draw_weight(N, c.d, c.seed)
+    pd = _dev(c.params)
+    x, wd = c.x.to(DEV), W.to(DEV)
+    qa, sa = kq.quantize(x, pd)
+    qb, sb = kq.quantize_weight(wd, pd)
+    qa_t, ta = kq.quantize_tiled(x, pd)
+    qb_t, tb = kq.quantize_weight_tiled(wd, pd)
+    torch.cuda.synchronize()
+    assert torch.equal(qa, qa_t) and torch.equal(qb, qb_t)
+    assert np.array_equal(ta.cpu().numpy(), o.scales_to_mma(sa.cpu().numpy()))
+    assert np.array_equal(tb.cpu().numpy(), o.scales_to_mma(sb.cpu().numpy()))
+    c_row = kq.gemm_mxfp4(qa, sa, qb, sb)
+    c_tiled = kq.gemm_mxfp4_tiled(qa_t, ta, qb_t, tb)
+    assert torch.equal(c_row, c_tiled)

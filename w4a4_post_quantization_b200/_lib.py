@@ -36,6 +36,11 @@ SIGNATURES = {
     "kq_quantize_weight": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_fold_weight": [_p, _i64, _i64, _p, _p, _p],
     "kq_gemm_mxfp4": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p],
+    "kq_gemm_mxfp4_tiled": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p],
+    "kq_scales_tiled_bytes": [_i64, _i64],
+    "kq_quantize_tiled": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_quantize_weight_tiled": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_scales_to_tiled": [_p, _i64, _i64, _p, _p],
     "kq_transform_params_grad_workspace_bytes": [_i64, _i64],
     "kq_transform_params_grad": [_p, _p, _p, _i64, _i64, _p, _int, ctypes.c_float, _p, _p, _p,
                                  ctypes.c_size_t, _p],
@@ -59,7 +64,8 @@ SIGNATURES = {
 _RESTYPE = {"kq_status_string": ctypes.c_char_p,
             "kq_quantize_host_workspace_bytes": ctypes.c_size_t,
             "kq_transform_params_grad_workspace_bytes": ctypes.c_size_t,
-            "kq_residual_workspace_bytes": ctypes.c_size_t}
+            "kq_residual_workspace_bytes": ctypes.c_size_t,
+            "kq_scales_tiled_bytes": ctypes.c_size_t}
 
 
 class KQError(RuntimeError):
@@ -390,6 +396,77 @@ def adam_step(params: torch.Tensor, grad0: torch.Tensor, grad1, m: torch.Tensor,
                             float(beta2), float(eps), _stream(params.device))
     _check("kq_adam_step", st)
     return params
+
+
+def scales_to_tiled(scales: torch.Tensor, K: int, out=None):
+    """Row-major scale bytes [rows, K/32] -> the tiled layout the tensor-core
+    product reads (1-D uint8 of kq_scales_tiled_bytes(rows, K) bytes)."""
+    _dev_tensor(scales, torch.uint8, "scales")
+    rows = scales.shape[0]
+    if scales.dim() != 2 or scales.shape[1] != K // 32:
+        raise ValueError("scales must be [rows, K/32]")
+    n = int(lib().kq_scales_tiled_bytes(rows, K))
+    if out is None:
+        out = torch.empty((n,), dtype=torch.uint8, device=scales.device)
+    _dev_tensor(out, torch.uint8, "out")
+    if out.numel() < n:
+        raise ValueError("out is too small")
+    st = lib().kq_scales_to_tiled(scales.data_ptr(), rows, K, out.data_ptr(),
+                                  _stream(scales.device))
+    _check("kq_scales_to_tiled", st)
+    return out
+
+
+def _quantize_tiled(fn: str, x: torch.Tensor, params: torch.Tensor, q=None, scales=None):
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    _params(params, d)
+    if q is None:
+        q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
+    n = int(lib().kq_scales_tiled_bytes(M, d))
+    if scales is None:
+        scales = torch.zeros((n,), dtype=torch.uint8, device=x.device)
+    _dev_tensor(q, torch.uint8, "q")
+    _dev_tensor(scales, torch.uint8, "scales")
+    if tuple(q.shape) != (M, d // 2) or scales.numel() < n:
+        raise ValueError("q must be [M, d/2] and scales hold kq_scales_tiled_bytes(M, d) bytes")
+    st = getattr(lib(), fn)(x.data_ptr(), M, d, params.data_ptr(), q.data_ptr(),
+                            scales.data_ptr(), _stream(x.device))
+    _check(fn, st)
+    return q, scales
+
+
+def quantize_tiled(x: torch.Tensor, params: torch.Tensor, q=None, scales=None):
+    """MXFP4(x T) with the scales in the tiled layout of the tensor-core product."""
+    return _quantize_tiled("kq_quantize_tiled", x, params, q, scales)
+
+
+def quantize_weight_tiled(w: torch.Tensor, params: torch.Tensor, q=None, scales=None):
+    """MXFP4(W T^-T) with the scales in the tiled layout."""
+    return _quantize_tiled("kq_quantize_weight_tiled", w, params, q, scales)
+
+
+def gemm_mxfp4_tiled(qa: torch.Tensor, sa_tiled: torch.Tensor, qb: torch.Tensor,
+                     sb_tiled: torch.Tensor, out=None, out_dtype=torch.float32):
+    """C = A B^T with both operands' scales in the tiled layout."""
+    for t, n in ((qa, "qa"), (sa_tiled, "sa_tiled"), (qb, "qb"), (sb_tiled, "sb_tiled")):
+        _dev_tensor(t, torch.uint8, n)
+    M, K = qa.shape[0], 2 * qa.shape[1]
+    N = qb.shape[0]
+    if tuple(qb.shape) != (N, K // 2):
+        raise ValueError("qb must be [N, K/2]")
+    if sa_tiled.numel() < lib().kq_scales_tiled_bytes(M, K) or \
+            sb_tiled.numel() < lib().kq_scales_tiled_bytes(N, K):
+        raise ValueError("tiled scale arrays are too small")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    _dev_tensor(out, out_dtype, "out")
+    code = KQ_OUT_F32 if out_dtype == torch.float32 else KQ_OUT_BF16
+    st = lib().kq_gemm_mxfp4_tiled(qa.data_ptr(), sa_tiled.data_ptr(), qb.data_ptr(),
+                                   sb_tiled.data_ptr(), M, N, K, out.data_ptr(), code,
+                                   _stream(qa.device))
+    _check("kq_gemm_mxfp4_tiled", st)
+    return out
 
 
 def inverse_transform(y: torch.Tensor, params: torch.Tensor, x=None):

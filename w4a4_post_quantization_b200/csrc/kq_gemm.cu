@@ -13,7 +13,12 @@
 //   warps 6..9  scale loaders, one per stage: the tile's E8M0 bytes from the
 //               row-major scale arrays into shared memory in the tensor
 //               core's scale layout (128-row x 4-scale chunks of 512 bytes:
-//               row r, scale i at byte 16 (r mod 32) + 4 (r div 32) + i)
+//               row r, scale i at byte 16 (r mod 32) + 4 (r div 32) + i).
+//               With scales already in that tiled layout
+//               (kq_gemm_mxfp4_tiled) there are no scale warps: warp 0 adds
+//               one bulk copy per 512-byte chunk run to each stage's loads,
+//               since four-byte scale words scattered over rows cost as many
+//               L2 requests as the codes themselves.
 //   warp 1      allocates TMEM; one lane copies the stage's scales into TMEM
 //               (tcgen05.cp) and issues four block-scaled MMAs
 //               (tcgen05.mma kind::mxf4, K = 64 each) into a float32
@@ -75,6 +80,7 @@ constexpr uint32_t kIdescMxf4 = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 
 struct GemmArgs {
   int32_t M, N, K;
   int32_t k_tiles, m_tiles, n_tiles;
+  int32_t sf_tiles_k, sf_tiles_n;   // tiled scales: 4-scale columns, B row tiles
   int32_t sf_stride;        // scale bytes per row: K / 32
   int32_t out_bf16;
   const uint8_t* sa;
@@ -91,6 +97,17 @@ __device__ __forceinline__ void mma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64
       "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
       "\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Untiled bulk copy of `bytes` (a multiple of 16, 16-byte aligned ends)
+// from global memory into this CTA's shared memory, completing on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes),
+      "r"(smem_addr(bar))
       : "memory");
 }
 
@@ -130,7 +147,13 @@ __device__ __forceinline__ void load_sf_words(uint32_t (&v)[kSfWordsPerLane], co
   }
 }
 
-template <bool kSfAligned>
+// Scale modes: row-major scale bytes loaded by the scale warps (4-byte
+// words when every row's scales are 4-byte aligned, bytes otherwise), or
+// the tiled layout (128-row x 4-scale tiles of 512 bytes), which the
+// producer thread copies straight into the stage with bulk copies.
+enum SfMode { kSfRowWords = 0, kSfRowBytes = 1, kSfTiled = 2 };
+
+template <int kSfMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap,
                      const __grid_constant__ CUtensorMap bmap, const GemmArgs a) {
@@ -157,9 +180,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   const int nk = a.k_tiles;
 
+  if (kSfMode == kSfTiled) {
+    // Chunks past the end of K are not copied; their codes are zero, and
+    // the scales there must only be finite.
+    for (int s = 0; s < kStages; ++s)
+      for (int i = tid; i < (kSfaBytes + kSfbBytes) / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(base + s * kStageBytes + kATile + kBTile)[i] =
+            make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 2);                      // TMA bytes + the stage's scale warp
+      // TMA bytes, plus the stage's scale warp unless the scales come by
+      // bulk copy with the codes.
+      mbar_init(&full[s], kSfMode == kSfTiled ? 1 : 2);
       mbar_init(&empty[s], 1);                     // tcgen05.commit of the stage's MMAs
     }
     mbar_init(acc_full, 1);
@@ -186,7 +220,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         uint8_t* st = base + s * kStageBytes;
-        mbar_arrive_expect_tx(&full[s], kATile + kBTile);
+        if (kSfMode == kSfTiled) {
+          // This k-tile's scale columns 2 kt, 2 kt + 1 (those that exist) of
+          // the A row tile and of the (up to) two B row tiles.
+          const int avail = min(kChunksPerStage, a.sf_tiles_k - kChunksPerStage * kt);
+          const int b_tiles = min(kBN / 128, a.sf_tiles_n - n0 / 128);
+          const uint32_t sf_bytes = (uint32_t)(avail * (1 + b_tiles)) * kSfChunk;
+          mbar_arrive_expect_tx(&full[s], kATile + kBTile + sf_bytes);
+          uint8_t* sfa = st + kATile + kBTile;
+          bulk_load(sfa, a.sa + ((int64_t)(m0 / 128) * a.sf_tiles_k + kChunksPerStage * kt) *
+                                  kSfChunk, avail * kSfChunk, &full[s]);
+          for (int g = 0; g < b_tiles; ++g)
+            bulk_load(sfa + kSfaBytes + g * kChunksPerStage * kSfChunk,
+                      a.sb + ((int64_t)(n0 / 128 + g) * a.sf_tiles_k + kChunksPerStage * kt) *
+                                 kSfChunk, avail * kSfChunk, &full[s]);
+        } else {
+          mbar_arrive_expect_tx(&full[s], kATile + kBTile);
+        }
         tma_load_2d(st, &amap, kt * kBKBytes, m0, &full[s]);
         tma_load_2d(st + kATile, &bmap, kt * kBKBytes, n0, &full[s]);
         issued = kt + 1;
@@ -204,19 +254,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     return;
   }
 
-  if (warp >= kSfWarp0) {
+  if (kSfMode != kSfTiled && warp >= kSfWarp0) {
     // ---------------------------------------------------------- scale loader
-    // Loader warp sw owns stage sw (k-tiles sw, sw + 4, ...): it loads the
-    // scales of its next k-tile into registers while the current ones are
-    // stored, so that its global loads are always one owned stage ahead.
+    // Loader warp sw owns stage sw (k-tiles sw, sw + 4, ...), so a stage's
+    // scales have four k-tiles of MMA time to arrive; all of a stage's
+    // loads are in flight together before the stores.
     const int sw = warp - kSfWarp0;
     const int s = sw;
     uint8_t* sfa = base + s * kStageBytes + kATile + kBTile;
     uint8_t* sfb = sfa + kSfaBytes;
-    uint32_t cur[kSfWordsPerLane], nxt[kSfWordsPerLane];
-    if (sw < nk) load_sf_words<kSfAligned>(cur, a, m0, n0, sw, lane);
     for (int kt = sw, n = 0; kt < nk; kt += kStages, ++n) {
-      if (kt + kStages < nk) load_sf_words<kSfAligned>(nxt, a, m0, n0, kt + kStages, lane);
+      uint32_t cur[kSfWordsPerLane];
+      load_sf_words<kSfMode == kSfRowWords>(cur, a, m0, n0, kt, lane);
       if (n >= 1 && !__all_sync(0xFFFFFFFFu, mbar_wait(&empty[s], (n - 1) & 1))) {
         if (lane == 0) atomicOr(a.err, kErrProducerWait);
         break;
@@ -229,15 +278,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           *reinterpret_cast<uint32_t*>(sfa + c * kSfChunk + sf_chunk_offset(r)) = cur[i];
         } else {
           const int r = (w - kBM * kChunksPerStage) >> 1;
-          *reinterpret_cast<uint32_t*>(sfb + (2 * c + (r >> 7)) * kSfChunk +
+          *reinterpret_cast<uint32_t*>(sfb + (2 * (r >> 7) + c) * kSfChunk +
                                        sf_chunk_offset(r & 127)) = cur[i];
         }
       }
       fence_proxy_async_smem();      // generic stores -> tcgen05.cp reads
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[s]);
-#pragma unroll
-      for (int i = 0; i < kSfWordsPerLane; ++i) cur[i] = nxt[i];
     }
     return;
   }
@@ -265,7 +312,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int g = 0; g < kBN / 128; ++g)
             tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * g,
-                               smem_desc_rows16(smem_addr(sfb + (2 * c + g) * kSfChunk)));
+                               smem_desc_rows16(smem_addr(sfb + (2 * g + c) * kSfChunk)));
         }
         const uint64_t adesc = smem_desc_sw128(smem_addr(st));
         const uint64_t bdesc = smem_desc_sw128(smem_addr(st + kATile));
@@ -371,9 +418,12 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t 
 
 using namespace kq;
 
-extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb,
-                             const uint8_t* sb, int64_t M, int64_t N, int64_t K, void* c,
-                             int c_dtype, void* stream) {
+namespace kq {
+namespace {
+
+int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
+                int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream,
+                bool tiled) {
   if (M < 0 || N < 0 || K < 32 || K % 32 != 0) return KQ_ERR_INVALID;
   if (c_dtype != KQ_OUT_F32 && c_dtype != KQ_OUT_BF16) return KQ_ERR_INVALID;
   if (M == 0 || N == 0) return KQ_OK;
@@ -383,6 +433,7 @@ extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t
   if (!qa || !sa || !qb || !sb || !c) return KQ_ERR_INVALID;
   auto al = [](const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; };
   if (!al(qa, 16) || !al(qb, 16) || !al(c, 16)) return KQ_ERR_INVALID;
+  if (tiled && (!al(sa, 16) || !al(sb, 16))) return KQ_ERR_INVALID;
   const DeviceInfo* di = nullptr;
   int dev = 0;
   int rc = device_info(&di, &dev);
@@ -397,6 +448,8 @@ extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t
   a.m_tiles = static_cast<int32_t>((M + kBM - 1) / kBM);
   a.n_tiles = static_cast<int32_t>((N + kBN - 1) / kBN);
   a.sf_stride = static_cast<int32_t>(K / 32);
+  a.sf_tiles_k = static_cast<int32_t>((K / 32 + 3) / 4);
+  a.sf_tiles_n = static_cast<int32_t>((N + 127) / 128);
   a.out_bf16 = c_dtype == KQ_OUT_BF16;
   a.sa = sa;
   a.sb = sb;
@@ -404,18 +457,80 @@ extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t
   CUtensorMap amap, bmap;
   if (!encode_codes_map(&amap, qa, M, K, kBM) || !encode_codes_map(&bmap, qb, N, K, kBN))
     return record_cuda_error(cudaErrorInvalidValue);
-  const bool aligned4 = (a.sf_stride % 4 == 0) && al(sa, 4) && al(sb, 4);
   const dim3 grid(static_cast<unsigned>(a.m_tiles * a.n_tiles));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (aligned4) {
-    rc = allow_smem<gemm_mxf4_kernel<true>>(kSmemBytes, dev);
+  if (tiled) {
+    // No scale warps: six warps.
+    rc = allow_smem<gemm_mxf4_kernel<kSfTiled>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<true><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
+    gemm_mxf4_kernel<kSfTiled><<<grid, 32 * kSfWarp0, kSmemBytes, st>>>(amap, bmap, a);
+  } else if ((a.sf_stride % 4 == 0) && al(sa, 4) && al(sb, 4)) {
+    rc = allow_smem<gemm_mxf4_kernel<kSfRowWords>>(kSmemBytes, dev);
+    if (rc != KQ_OK) return rc;
+    gemm_mxf4_kernel<kSfRowWords><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
   } else {
-    rc = allow_smem<gemm_mxf4_kernel<false>>(kSmemBytes, dev);
+    rc = allow_smem<gemm_mxf4_kernel<kSfRowBytes>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<false><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
+    gemm_mxf4_kernel<kSfRowBytes><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
   }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return record_cuda_error(e);
+  return KQ_OK;
+}
+
+// One thread per 4-byte word of the tiled layout: word t of tile
+// (row tile, column) holds row 32 (t mod 4) + t / 4 of the tile, scales
+// 4 column .. 4 column + 3.
+__global__ void scales_tile_kernel(const uint8_t* s, int64_t rows, int64_t ns, int64_t col_tiles,
+                                   int64_t words, uint32_t* out) {
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < words;
+       w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t tile = w >> 7;
+    const int t = static_cast<int>(w & 127);
+    const int64_t row = (tile / col_tiles) * 128 + 32 * (t & 3) + (t >> 2);
+    const int64_t k0 = (tile % col_tiles) * 4;
+    uint32_t v = 0;
+    if (row < rows)
+      for (int i = 0; i < 4; ++i)
+        if (k0 + i < ns) v |= static_cast<uint32_t>(s[row * ns + k0 + i]) << (8 * i);
+    out[w] = v;
+  }
+}
+
+}  // namespace
+}  // namespace kq
+
+extern "C" int kq_gemm_mxfp4(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb,
+                             const uint8_t* sb, int64_t M, int64_t N, int64_t K, void* c,
+                             int c_dtype, void* stream) {
+  return launch_gemm(qa, sa, qb, sb, M, N, K, c, c_dtype, stream, false);
+}
+
+extern "C" int kq_gemm_mxfp4_tiled(const uint8_t* qa, const uint8_t* sa_tiled, const uint8_t* qb,
+                                   const uint8_t* sb_tiled, int64_t M, int64_t N, int64_t K,
+                                   void* c, int c_dtype, void* stream) {
+  return launch_gemm(qa, sa_tiled, qb, sb_tiled, M, N, K, c, c_dtype, stream, true);
+}
+
+extern "C" size_t kq_scales_tiled_bytes(int64_t rows, int64_t K) {
+  if (rows < 1 || K < 32 || K % 32 != 0) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K / 32 + 3) / 4) * 512;
+}
+
+extern "C" int kq_scales_to_tiled(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* tiled,
+                                  void* stream) {
+  if (rows < 0 || K < 32 || K % 32 != 0) return KQ_ERR_INVALID;
+  if (rows == 0) return KQ_OK;
+  if (rows > (int64_t(1) << 40) / K) return KQ_ERR_INVALID;
+  if (!scales || !tiled || reinterpret_cast<uintptr_t>(tiled) % 16 != 0) return KQ_ERR_INVALID;
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  const int64_t words = static_cast<int64_t>(kq_scales_tiled_bytes(rows, K) / 4);
+  const int grid = static_cast<int>(std::min<int64_t>((words + 255) / 256, di->sms * 8));
+  scales_tile_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      scales, rows, K / 32, (K / 32 + 3) / 4, words, reinterpret_cast<uint32_t*>(tiled));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_error(e);
   return KQ_OK;

@@ -230,7 +230,17 @@ struct PanelArgs {
   uint8_t* q;
   uint8_t* scales;
   float* y;
+  int32_t scale_tiles_k;  // 0: scales row-major; else the tiled layout with this
+                          // many 4-scale columns (128-row x 4-scale tiles)
 };
+
+// Offset of (row, scale column j) in the tiled scale layout: 128-row x
+// 4-scale tiles of 512 bytes, row r = r0 + 32 r1 and scale i at byte
+// 16 r0 + 4 r1 + i.
+__device__ __forceinline__ int64_t tiled_scale_offset(int64_t row, int j, int tiles_k) {
+  const int r = static_cast<int>(row & 127);
+  return ((row >> 7) * tiles_k + (j >> 2)) * 512 + 16 * (r & 31) + 4 * (r >> 5) + (j & 3);
+}
 
 // Launch shape of the panel kernel: consumer warps, rows per consumer thread
 // per tile, and CTAs per SM it is compiled for.
@@ -334,7 +344,16 @@ __device__ __forceinline__ void panel_consume(const PanelArgs& a, const uint8_t*
       } else if constexpr (kOut == kOutMx4) {
         const Mx4Block b = mxfp4_block(u);
         __stcs(reinterpret_cast<uint4*>(a.q + g * 16), b.codes);
-        a.scales[g] = static_cast<uint8_t>(b.scale);
+        if (a.scale_tiles_k == 0) {
+          a.scales[g] = static_cast<uint8_t>(b.scale);
+        } else {
+          const int64_t o = tiled_scale_offset(rr, j, a.scale_tiles_k);
+          a.scales[o] = static_cast<uint8_t>(b.scale);
+          // The last block of a row also zeroes the row's padding scales:
+          // they multiply zero codes in the product and must be finite.
+          if (j == a.nb - 1)
+            for (int t = (j & 3) + 1; t < 4; ++t) a.scales[o + t - (j & 3)] = 0;
+        }
       } else {
         float4* dst = reinterpret_cast<float4*>(a.y + g * kBlock);
 #pragma unroll
@@ -711,13 +730,15 @@ double panel_use(int nb, int sms, int* W, int* R) {
 
 template <int kXf, int kOut, class Cfg>
 int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q,
-                     uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev) {
+                     uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev,
+                     int32_t scale_tiles_k) {
   constexpr int kRpt = Cfg::kRpt;
   const int nb = static_cast<int>(d / kBlock);
   PanelArgs a{};
   // The 16-element variant and the weight fold have no other kernel, so
   // they take any shape.
-  const double min_use = (kXf == kXfKron16 || kXf == kXfKronInvT) ? 0.0 : 0.5;
+  const double min_use =
+      (kXf == kXfKron16 || kXf == kXfKronInvT || scale_tiles_k > 0) ? 0.0 : 0.5;
   if (panel_use<Cfg>(nb, di.sms, &a.W, &a.R) < min_use) return KQ_ERR_INVALID;
   a.M = M;
   a.nb = nb;
@@ -739,6 +760,7 @@ int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, 
   a.q = q;
   a.scales = scales;
   a.y = y;
+  a.scale_tiles_k = scale_tiles_k;
   const int smem = 1024 + a.stages * a.stage_bytes + 2 * a.stages * 8;
   int rc = allow_smem<panel_kernel<kXf, kOut, Cfg>>(smem, dev);
   if (rc != KQ_OK) return rc;
@@ -766,11 +788,18 @@ int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, 
 
 template <int kXf, int kOut>
 int launch_panel(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q,
-                 uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev) {
+                 uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev,
+                 int32_t scale_tiles_k = 0) {
   switch (panel_variant()) {
-    case 1: return launch_panel_cfg<kXf, kOut, PanelV1>(x, M, d, aux, q, scales, y, st, di, dev);
-    case 2: return launch_panel_cfg<kXf, kOut, PanelV2>(x, M, d, aux, q, scales, y, st, di, dev);
-    default: return launch_panel_cfg<kXf, kOut, PanelV0>(x, M, d, aux, q, scales, y, st, di, dev);
+    case 1:
+      return launch_panel_cfg<kXf, kOut, PanelV1>(x, M, d, aux, q, scales, y, st, di, dev,
+                                                  scale_tiles_k);
+    case 2:
+      return launch_panel_cfg<kXf, kOut, PanelV2>(x, M, d, aux, q, scales, y, st, di, dev,
+                                                  scale_tiles_k);
+    default:
+      return launch_panel_cfg<kXf, kOut, PanelV0>(x, M, d, aux, q, scales, y, st, di, dev,
+                                                  scale_tiles_k);
   }
 }
 
@@ -841,6 +870,21 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
     if (impl == KQ_IMPL_DIRECT) return launch_direct<kXf, kOut, false>(x, M, d, a, st, *di, dev);
     return KQ_ERR_INVALID;
   }
+}
+
+// The panel kernel with scales written in the tiled layout.
+template <int kXf>
+int run_tiled(const uint16_t* x, int64_t M, int64_t d, const float* params, uint8_t* q,
+              uint8_t* scales_tiled, void* stream) {
+  const DeviceInfo* di = nullptr;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != KQ_OK) return rc;
+  const int64_t nb = d / kBlock;
+  if (nb > 65535) return KQ_ERR_INVALID;
+  return launch_panel<kXf, kOutMx4>(x, M, d, params, q, scales_tiled, nullptr,
+                                    static_cast<cudaStream_t>(stream), *di, dev,
+                                    static_cast<int32_t>((nb + 3) / 4));
 }
 
 int check_quant_args(const uint16_t* x, int64_t M, int64_t d, const void* aux, bool need_aux,
@@ -933,6 +977,21 @@ extern "C" int kq_fold_weight(const uint16_t* w, int64_t N, int64_t d, const flo
     return KQ_ERR_INVALID;
   return run<kXfKronInvT, kOutF32>(w, N, d, params, nullptr, nullptr, w_folded, KQ_IMPL_PANEL,
                                    stream);
+}
+
+extern "C" int kq_quantize_tiled(const uint16_t* x, int64_t M, int64_t d, const float* params,
+                                 uint8_t* q_packed, uint8_t* scales_tiled, void* stream) {
+  int rc = check_quant_args(x, M, d, params, true, q_packed, scales_tiled);
+  if (rc != KQ_OK || M == 0) return rc;
+  return run_tiled<kXfKron>(x, M, d, params, q_packed, scales_tiled, stream);
+}
+
+extern "C" int kq_quantize_weight_tiled(const uint16_t* w, int64_t N, int64_t d,
+                                        const float* params, uint8_t* q_packed,
+                                        uint8_t* scales_tiled, void* stream) {
+  int rc = check_quant_args(w, N, d, params, true, q_packed, scales_tiled);
+  if (rc != KQ_OK || N == 0) return rc;
+  return run_tiled<kXfKronInvT>(w, N, d, params, q_packed, scales_tiled, stream);
 }
 
 extern "C" int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,
