@@ -53,6 +53,8 @@ constexpr int kSfbBytes = kChunksPerStage * (kBN / 128) * kSfChunk;
 constexpr int kStageBytes = kATile + kBTile + kSfaBytes + kSfbBytes;
 static_assert(kStageBytes % 1024 == 0, "stages must keep the 1024-byte swizzle alignment");
 constexpr int kSmemBytes = 1024 + kStages * kStageBytes + (2 * kStages + 2) * 8 + 16;
+constexpr int kOutBoxBytes = kBM * 128;        // one store box: 128 rows x 128 bytes
+static_assert(kBN * 4 / 128 * kOutBoxBytes <= kStages * kStageBytes, "output tile in the stages");
 
 constexpr int kSfWarp0 = 6;                    // warps 6..9 load scales, one stage each
 constexpr int kSfWarps = kStages;
@@ -81,6 +83,7 @@ struct GemmArgs {
   int32_t M, N, K;
   int32_t k_tiles, m_tiles, n_tiles;
   int32_t sf_tiles_k, sf_tiles_n;   // tiled scales: 4-scale columns, B row tiles
+  int32_t tma_store;                // the epilogue stages the tile and stores it by TMA
   int32_t sf_stride;        // scale bytes per row: K / 32
   int32_t out_bf16;
   const uint8_t* sa;
@@ -156,7 +159,8 @@ enum SfMode { kSfRowWords = 0, kSfRowBytes = 1, kSfTiled = 2 };
 template <int kSfMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap,
-                     const __grid_constant__ CUtensorMap bmap, const GemmArgs a) {
+                     const __grid_constant__ CUtensorMap bmap,
+                     const __grid_constant__ CUtensorMap cmap, const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
@@ -344,6 +348,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0));
     if (!ok) {
       if (lane == 0) atomicOr(a.err, kErrConsumerWait);
+    } else if (a.tma_store) {
+      // Every MMA has completed, so the stage buffers are free: the tile
+      // goes there as 128-byte-swizzled boxes of 128 rows x 128 bytes
+      // (row r's 16-byte chunk c at c ^ (r mod 8)), then out by TMA stores
+      // that clip at the matrix edges.
+      tmem_fence_after();
+      const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
+      const int r = quarter * 32 + lane;
+      const int cols_per_box = a.out_bf16 ? 64 : 32;
+#pragma unroll 1
+      for (int v = 0; v < kBN / 32; ++v) {
+        uint32_t x[32];
+        tmem_ld32(taddr + 32 * v, x);
+        tmem_wait_ld();
+        const int col = 32 * v;
+        uint8_t* box = base + (col / cols_per_box) * kOutBoxBytes + r * 128;
+        if (a.out_bf16) {
+          const int c0 = (col % 64) / 8;           // first 16-byte chunk of these 32 columns
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(x[8 * q + 2 * h]),
+                                                            __uint_as_float(x[8 * q + 2 * h + 1]));
+              wv[h] = *reinterpret_cast<const uint32_t*>(&p);
+            }
+            *reinterpret_cast<uint4*>(box + 16 * ((c0 + q) ^ (r & 7))) =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(box + 16 * (q ^ (r & 7))) =
+                make_uint4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();                    // generic stores -> TMA store reads
+      asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory");
+      if (warp == 2 && lane == 0) {
+        for (int b = 0; b < kBN / cols_per_box; ++b)
+          tma_store_2d(&cmap, base + b * kOutBoxBytes, n0 + b * cols_per_box, m0);
+        bulk_commit();
+        bulk_wait_all();
+      }
     } else {
       tmem_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
@@ -454,24 +503,41 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   a.sa = sa;
   a.sb = sb;
   a.c = c;
-  CUtensorMap amap, bmap;
+  CUtensorMap amap, bmap, cmap;
   if (!encode_codes_map(&amap, qa, M, K, kBM) || !encode_codes_map(&bmap, qb, N, K, kBN))
     return record_cuda_error(cudaErrorInvalidValue);
+  // TMA-store epilogue when the output row pitch is a multiple of 16 bytes.
+  const int esize = c_dtype == KQ_OUT_BF16 ? 2 : 4;
+  a.tma_store = (N * esize) % 16 == 0;
+  cmap = amap;
+  if (a.tma_store) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * esize};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), kBM};
+    const cuuint32_t estr[2] = {1, 1};
+    if (tensor_map_encoder()(&cmap,
+                             esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                             2, c, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return record_cuda_error(cudaErrorInvalidValue);
+  }
   const dim3 grid(static_cast<unsigned>(a.m_tiles * a.n_tiles));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (tiled) {
     // No scale warps: six warps.
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<kSfTiled><<<grid, 32 * kSfWarp0, kSmemBytes, st>>>(amap, bmap, a);
+    gemm_mxf4_kernel<kSfTiled><<<grid, 32 * kSfWarp0, kSmemBytes, st>>>(amap, bmap, cmap, a);
   } else if ((a.sf_stride % 4 == 0) && al(sa, 4) && al(sb, 4)) {
     rc = allow_smem<gemm_mxf4_kernel<kSfRowWords>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<kSfRowWords><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
+    gemm_mxf4_kernel<kSfRowWords><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, cmap, a);
   } else {
     rc = allow_smem<gemm_mxf4_kernel<kSfRowBytes>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<kSfRowBytes><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, a);
+    gemm_mxf4_kernel<kSfRowBytes><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, cmap, a);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_error(e);
