@@ -199,3 +199,26 @@ def test_quantizers_write_the_tiled_layout(name, di, N):
     c_row = kq.gemm_mxfp4(qa, sa, qb, sb)
     c_tiled = kq.gemm_mxfp4_tiled(qa_t, ta, qb_t, tb)
     assert torch.equal(c_row, c_tiled)
+
+
+@pytest.mark.parametrize("M,N,K,dt", [(4096, 4096, 1152, torch.bfloat16),
+                                      (2048, 4104, 544, torch.float32),
+                                      (2100, 2048, 4096, torch.bfloat16),
+                                      (300, 520, 96, torch.float32)])
+def test_persistent_and_per_tile_kernels_agree(M, N, K, dt, monkeypatch):
+    """The persistent tiled-scale kernel (several tiles per CTA, TMA stores
+    overlapping the next tile) and the one-tile-per-CTA kernel run the same
+    MMAs on the same stages: identical outputs."""
+    qa, sa, qb, sb = random_operands(M, N, K, seed=M + N + K + 3)
+    ta, tb = kq.scales_to_tiled(_dev(sa), K), kq.scales_to_tiled(_dev(sb), K)
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("KQ_GEMM_PERSISTENT", flag)
+        outs.append(kq.gemm_mxfp4_tiled(_dev(qa), ta, _dev(qb), tb, out_dtype=dt))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1])
+    rows = np.array([0, 1, 127, 128, M // 2, M - 1])
+    check_gemm(outs[0].float().cpu().numpy() if dt == torch.float32 else
+               outs[0].float().cpu().numpy(), qa, sa, qb, sb, rows=rows) \
+        if dt == torch.float32 else None
+    assert kq.device_status() == 0

@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 
 #include "kq.h"
 #include "kq_device.cuh"
@@ -462,6 +463,250 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t 
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ---------------------------------------------------------------------------
+// Persistent variant (tiled scales): one CTA per SM walks the banded tile
+// order.  Three stages leave room for a separate 64 KiB staging buffer, so
+// the producer runs on into the next tile while the epilogue drains: the MMAs
+// of tile i + 1 wait only until the accumulator of tile i has been read out
+// of TMEM, and tile i's TMA stores overlap tile i + 1's main loop.
+constexpr int kPStages = 3;
+constexpr int kPStageBytes = kStageBytes;
+constexpr int kStagingBytes = 4 * kOutBoxBytes;          // 64 KiB: 4 boxes
+constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kStagingBytes +
+                            (2 * kPStages + 4) * 8 + 16;
+constexpr int kPThreads = 32 * 6;
+constexpr int64_t kPersistentMaxK = 4096;
+
+__device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, int& n0) {
+  const int band = t / (kBandN * a.m_tiles);
+  const int r = t - band * kBandN * a.m_tiles;
+  const int width = min(kBandN, a.n_tiles - band * kBandN);
+  m0 = (r / width) * kBM;
+  n0 = (band * kBandN + r % width) * kBN;
+}
+
+__global__ void __launch_bounds__(kPThreads, 1)
+    gemm_mxf4_persistent(const __grid_constant__ CUtensorMap amap,
+                         const __grid_constant__ CUtensorMap bmap,
+                         const __grid_constant__ CUtensorMap cmap, const GemmArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* staging = base + kPStages * kPStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
+  uint64_t* empty = full + kPStages;
+  uint64_t* acc_full = empty + kPStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* mma_done = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_tiles_total = a.m_tiles * a.n_tiles;
+  const int nk = a.k_tiles;
+
+  for (int st = 0; st < kPStages; ++st)
+    for (int i = tid; i < (kSfaBytes + kSfbBytes) / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(base + st * kPStageBytes + kATile + kBTile)[i] =
+          make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (tid == 0) {
+    for (int st = 0; st < kPStages; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 4);                 // one arrival per epilogue warp
+    mbar_init(mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tmem_fence_before();
+  __syncthreads();
+  tmem_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_map(&amap);
+      tma_prefetch_map(&bmap);
+      int s = 0, issued = 0, g = 0;          // g: k-tiles issued over all tiles
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x) {
+        int m0, n0;
+        tile_origin(a, t, m0, n0);
+        const int b_tiles = min(kBN / 128, a.sf_tiles_n - n0 / 128);
+        for (int kt = 0; kt < nk; ++kt, ++g) {
+          if (g >= kPStages && !mbar_wait(&empty[s], phase)) {
+            ok = false;
+            break;
+          }
+          uint8_t* stg = base + s * kPStageBytes;
+          const int avail = min(kChunksPerStage, a.sf_tiles_k - kChunksPerStage * kt);
+          mbar_arrive_expect_tx(&full[s], kATile + kBTile +
+                                              (uint32_t)(avail * (1 + b_tiles)) * kSfChunk);
+          uint8_t* sfa = stg + kATile + kBTile;
+          bulk_load(sfa, a.sa + ((int64_t)(m0 / 128) * a.sf_tiles_k + kChunksPerStage * kt) *
+                                  kSfChunk, avail * kSfChunk, &full[s]);
+          for (int gb = 0; gb < b_tiles; ++gb)
+            bulk_load(sfa + kSfaBytes + gb * kChunksPerStage * kSfChunk,
+                      a.sb + ((int64_t)(n0 / 128 + gb) * a.sf_tiles_k + kChunksPerStage * kt) *
+                                 kSfChunk, avail * kSfChunk, &full[s]);
+          tma_load_2d(stg, &amap, kt * kBKBytes, m0, &full[s]);
+          tma_load_2d(stg + kATile, &bmap, kt * kBKBytes, n0, &full[s]);
+          issued = g + 1;
+          if (++s == kPStages) {
+            s = 0;
+            if (g >= kPStages) phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        atomicOr(a.err, kErrProducerWait);
+        for (int i = issued > kPStages ? issued - kPStages : 0; i < issued; ++i)
+          mbar_wait(&full[i % kPStages], (i / kPStages) & 1);
+      }
+    }
+    return;
+  }
+
+  if (warp == 1) {
+    // -------------------------------------------------- scale copies + MMA
+    if (lane == 0) {
+      int s = 0, i = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x, ++i) {
+        // The accumulator is free once the epilogue has read tile i - 1.
+        if (i >= 1 && !mbar_wait(acc_empty, (i - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tmem_fence_after();
+        for (int kt = 0; kt < nk; ++kt) {
+          if (!mbar_wait(&full[s], phase)) {
+            ok = false;
+            break;
+          }
+          tmem_fence_after();
+          const uint8_t* stg = base + s * kPStageBytes;
+          const uint8_t* sfa = stg + kATile + kBTile;
+          const uint8_t* sfb = sfa + kSfaBytes;
+          const uint32_t tsfa = tmem_base + kSfCol0 + s * (kSfColsA + kSfColsB);
+          const uint32_t tsfb = tsfa + kSfColsA;
+#pragma unroll
+          for (int c = 0; c < kChunksPerStage; ++c) {
+            tmem_cp_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
+#pragma unroll
+            for (int gb = 0; gb < kBN / 128; ++gb)
+              tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * gb,
+                                 smem_desc_rows16(smem_addr(sfb + (2 * gb + c) * kSfChunk)));
+          }
+          const uint64_t adesc = smem_desc_sw128(smem_addr(stg));
+          const uint64_t bdesc = smem_desc_sw128(smem_addr(stg + kATile));
+#pragma unroll
+          for (int kk = 0; kk < kBK / kMmaK; ++kk) {
+            const uint32_t sf_id = 2u * (kk & 1);
+            const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
+            mma_mxf4(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
+                     tsfb + 8 * (kk >> 1), (kt | kk) != 0);
+          }
+          mma_commit(&empty[s]);
+          if (++s == kPStages) {
+            s = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) mma_commit(acc_full);
+      }
+      if (!ok) atomicOr(a.err, kErrConsumerWait);
+      mma_commit(mma_done);
+      mbar_wait(mma_done, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // Rows of TMEM lane quarter (warp mod 4); the tile leaves through the
+    // staging buffer as 128-byte-swizzled boxes of 128 rows x 128 bytes.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
+    const bool issuer = warp == 2 && lane == 0;
+    const int cols_per_box = a.out_bf16 ? 64 : 32;
+    const int passes = a.out_bf16 ? 1 : 2;         // float32: two halves of 4 boxes
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles_total; t += gridDim.x, ++i) {
+      int m0, n0;
+      tile_origin(a, t, m0, n0);
+      // One AND-barrier makes a timeout the same for the four warps and,
+      // with the issuer's wait before it, frees the staging buffer (the
+      // previous tile's stores have read it).
+      const bool got = mbar_wait(acc_full, i & 1);
+      if (issuer) bulk_wait_read_0();
+      if (!bar_and(3, 4 * 32, got)) {
+        if (lane == 0) atomicOr(a.err, kErrConsumerWait);
+        break;
+      }
+      tmem_fence_after();
+      for (int pass = 0; pass < passes; ++pass) {
+        if (pass > 0) {
+          if (issuer) bulk_wait_read_0();
+          asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory");
+        }
+        const int v0 = pass * (kBN / 32 / passes), v1 = v0 + kBN / 32 / passes;
+#pragma unroll 1
+        for (int v = v0; v < v1; ++v) {
+          uint32_t x[32];
+          tmem_ld32(taddr + 32 * v, x);
+          tmem_wait_ld();
+          const int col = 32 * v - (a.out_bf16 ? 0 : pass * 128);
+          uint8_t* box = staging + (col / cols_per_box) * kOutBoxBytes + r * 128;
+          if (a.out_bf16) {
+            const int c0 = (col % 64) / 8;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t wv[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __nv_bfloat162 p = __floats2bfloat162_rn(
+                    __uint_as_float(x[8 * q + 2 * h]), __uint_as_float(x[8 * q + 2 * h + 1]));
+                wv[h] = *reinterpret_cast<const uint32_t*>(&p);
+              }
+              *reinterpret_cast<uint4*>(box + 16 * ((c0 + q) ^ (r & 7))) =
+                  make_uint4(wv[0], wv[1], wv[2], wv[3]);
+            }
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              *reinterpret_cast<uint4*>(box + 16 * (q ^ (r & 7))) =
+                  make_uint4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+          }
+        }
+        if (pass == passes - 1) {
+          // Every column has been read: the MMAs of the next tile may start.
+          tmem_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory");
+        if (issuer) {
+          for (int b = 0; b < 4; ++b)
+            tma_store_2d(&cmap, staging + b * kOutBoxBytes,
+                         n0 + (pass * 4 + b) * cols_per_box, m0);
+          bulk_commit();
+        }
+      }
+    }
+    if (issuer) bulk_wait_all();
+    tmem_fence_before();
+  }
+  asm volatile("bar.sync 2, %0;" ::"r"(5 * 32) : "memory");
+  if (warp == 1) {
+    tmem_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
 }  // namespace
 }  // namespace kq
 
@@ -469,6 +714,14 @@ using namespace kq;
 
 namespace kq {
 namespace {
+
+// The persistent kernel for short K, where a tile's own prologue and
+// epilogue weigh most; KQ_GEMM_PERSISTENT=0/1 forces either (measurements).
+bool persistent_gemm(int64_t K) {
+  const char* e = getenv("KQ_GEMM_PERSISTENT");
+  if (e) return atoi(e) != 0;
+  return K <= kPersistentMaxK;
+}
 
 int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
                 int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream,
@@ -525,7 +778,12 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   }
   const dim3 grid(static_cast<unsigned>(a.m_tiles * a.n_tiles));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (tiled) {
+  if (tiled && a.tma_store && persistent_gemm(K)) {
+    rc = allow_smem<gemm_mxf4_persistent>(kPSmemBytes, dev);
+    if (rc != KQ_OK) return rc;
+    const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
+    gemm_mxf4_persistent<<<pgrid, kPThreads, kPSmemBytes, st>>>(amap, bmap, cmap, a);
+  } else if (tiled) {
     // No scale warps: six warps.
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
