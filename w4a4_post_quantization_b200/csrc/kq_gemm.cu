@@ -475,7 +475,7 @@ constexpr int kStagingBytes = 4 * kOutBoxBytes;          // 64 KiB: 4 boxes
 constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kStagingBytes +
                             (2 * kPStages + 4) * 8 + 16;
 constexpr int kPThreads = 32 * 6;
-constexpr int64_t kPersistentMaxK = 4096;
+constexpr int64_t kPersistentMaxK = 8192;   // measured: K 6144 +22 %, 12288 even, 16384 -17 %
 
 __device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, int& n0) {
   const int band = t / (kBandN * a.m_tiles);
