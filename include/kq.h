@@ -134,6 +134,13 @@ int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const float* params1
 int kq_quantize_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
                       const uint16_t* scale, int64_t tokens_per_sample, float eps,
                       const float* params, uint8_t* q_packed, uint8_t* scales, void* stream);
+/* kq_quantize_adaln with the scales in the tiled layout of
+ * kq_gemm_mxfp4_tiled (scales_tiled: kq_scales_tiled_bytes(M, d) bytes; the
+ * padding of each row's last 4-scale column is written as 0). */
+int kq_quantize_adaln_tiled(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
+                            const uint16_t* scale, int64_t tokens_per_sample, float eps,
+                            const float* params, uint8_t* q_packed, uint8_t* scales_tiled,
+                            void* stream);
 int kq_transform_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
                        const uint16_t* scale, int64_t tokens_per_sample, float eps,
                        const float* params, float* y, void* stream);

@@ -137,3 +137,23 @@ def test_adaln_rejects_bad_arguments_and_no_wait_gave_up():
     assert lib.kq_quantize_adaln(x.data_ptr(), 4, 64, sh.data_ptr() + 2, sh.data_ptr(), 4, 1e-6,
                                  p.data_ptr(), q.data_ptr(), s.data_ptr(), st) == 1
     assert kq.device_status() == 0
+
+
+def test_adaln_tiled_scales_feed_the_tiled_gemm():
+    """kq_quantize_adaln_tiled writes the same codes and the tiled image of
+    the row-major scales; the normalized layer's product through the tiled
+    GEMM equals the row-major one bit for bit."""
+    c = w.make_case("pixart_sigma", 0, 0, M=300)
+    T = 128
+    shift, scale = w.draw_adaln(-(-c.M // T), c.d, c.seed)
+    xd, sd, cd = c.x.to(DEV), shift.to(DEV), scale.to(DEV)
+    pd = torch.from_numpy(c.params).to(DEV)
+    q, s = kq.quantize_adaln(xd, sd, cd, T, pd)
+    qt, st = kq.quantize_adaln_tiled(xd, sd, cd, T, pd)
+    torch.cuda.synchronize()
+    assert torch.equal(q, qt)
+    assert np.array_equal(st.cpu().numpy(), o.scales_to_mma(s.cpu().numpy()))
+    W = w.draw_weight(512, c.d, c.seed).to(DEV)
+    qb, sb = kq.quantize_weight(W, pd)
+    qbt, sbt = kq.quantize_weight_tiled(W, pd)
+    assert torch.equal(kq.gemm_mxfp4(q, s, qb, sb), kq.gemm_mxfp4_tiled(qt, st, qbt, sbt))

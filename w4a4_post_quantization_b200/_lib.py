@@ -49,6 +49,7 @@ SIGNATURES = {
     "kq_adam_step": [_p, _p, _p, _p, _p, _i64, _int, ctypes.c_double, ctypes.c_double,
                      ctypes.c_double, ctypes.c_double, _p],
     "kq_quantize_adaln": [_p, _i64, _i64, _p, _p, _i64, ctypes.c_float, _p, _p, _p, _p],
+    "kq_quantize_adaln_tiled": [_p, _i64, _i64, _p, _p, _i64, ctypes.c_float, _p, _p, _p, _p],
     "kq_transform_adaln": [_p, _i64, _i64, _p, _p, _i64, ctypes.c_float, _p, _p, _p],
     "kq_inverse_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_dequantize": [_p, _p, _i64, _i64, _p, _p],
@@ -313,6 +314,28 @@ def quantize_adaln(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
                                  int(tokens_per_sample), float(eps), params.data_ptr(),
                                  q.data_ptr(), scales.data_ptr(), _stream(x.device))
     _check("kq_quantize_adaln", st)
+    return q, scales
+
+
+def quantize_adaln_tiled(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor,
+                         tokens_per_sample: int, params: torch.Tensor, eps: float = 1e-6,
+                         q=None, scales=None):
+    """quantize_adaln with the scales in the tiled layout of gemm_mxfp4_tiled."""
+    M, d = _adaln_args(x, shift, scale, tokens_per_sample)
+    _params(params, d)
+    if q is None:
+        q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
+    n = int(lib().kq_scales_tiled_bytes(M, d))
+    if scales is None:
+        scales = torch.zeros((n,), dtype=torch.uint8, device=x.device)
+    _dev_tensor(q, torch.uint8, "q")
+    _dev_tensor(scales, torch.uint8, "scales")
+    if tuple(q.shape) != (M, d // 2) or scales.numel() < n:
+        raise ValueError("q must be [M, d/2] and scales hold kq_scales_tiled_bytes(M, d) bytes")
+    st = lib().kq_quantize_adaln_tiled(x.data_ptr(), M, d, shift.data_ptr(), scale.data_ptr(),
+                                       int(tokens_per_sample), float(eps), params.data_ptr(),
+                                       q.data_ptr(), scales.data_ptr(), _stream(x.device))
+    _check("kq_quantize_adaln_tiled", st)
     return q, scales
 
 

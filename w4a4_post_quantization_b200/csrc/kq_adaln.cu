@@ -56,6 +56,7 @@ struct AdaArgs {
   const uint32_t* scale;
   uint8_t* q;
   uint8_t* scales;
+  int32_t scale_tiles_k;     // 0: row-major scales; else the tiled layout (4-scale columns)
   float* y;
   int* err;
 };
@@ -306,7 +307,19 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
     if (kOut == 0) {
       const Mx4Block blk = mxfp4_block(u);
       __stcs(reinterpret_cast<uint4*>(a.q + gi * 16), blk.codes);
-      a.scales[gi] = static_cast<uint8_t>(blk.scale);
+      if (a.scale_tiles_k == 0) {
+        a.scales[gi] = static_cast<uint8_t>(blk.scale);
+      } else {
+        // Tiled layout: 128-row x 4-scale tiles, row r = r0 + 32 r1 and
+        // scale i at byte 16 r0 + 4 r1 + i; the row's last block also
+        // zeroes the padding of its 4-scale column.
+        const int rl = static_cast<int>(row & 127);
+        const int64_t o = ((row >> 7) * a.scale_tiles_k + (j >> 2)) * 512 + 16 * (rl & 31) +
+                          4 * (rl >> 5) + (j & 3);
+        a.scales[o] = static_cast<uint8_t>(blk.scale);
+        if (j == nb - 1)
+          for (int t = (j & 3) + 1; t < 4; ++t) a.scales[o + t - (j & 3)] = 0;
+      }
     } else {
       float4* dst = reinterpret_cast<float4*>(a.y + gi * 32);
 #pragma unroll
@@ -386,7 +399,7 @@ __global__ void __launch_bounds__(kAdaCons, 1)
 // Launches the fused kernel; the shapes were checked by the caller.
 int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
                  const uint16_t* scale, int64_t tokens, float eps, const float* params,
-                 uint8_t* q, uint8_t* scales, float* y, cudaStream_t st) {
+                 uint8_t* q, uint8_t* scales, float* y, cudaStream_t st, bool tiled = false) {
   const DeviceInfo* di = nullptr;
   int dev = 0;
   int rc = device_info(&di, &dev);
@@ -417,6 +430,7 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   a.scale = reinterpret_cast<const uint32_t*>(scale);
   a.q = q;
   a.scales = scales;
+  a.scale_tiles_k = tiled ? (nb + 3) / 4 : 0;
   a.y = y;
   // Barriers, four slot buffers and the diagonal table (128 bytes a block).
   const int fixed = 1024 + (kAdaMaxStages + 2) * 8 + kAdaSlotBufs * kAdaSlots * 16 + nb * 128;
@@ -480,6 +494,18 @@ extern "C" int kq_quantize_adaln(const uint16_t* x, int64_t M, int64_t d, const 
     return KQ_ERR_INVALID;
   return launch_adaln(x, M, d, shift, scale, tokens_per_sample, eps, params, q_packed, scales,
                       nullptr, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int kq_quantize_adaln_tiled(const uint16_t* x, int64_t M, int64_t d,
+                                       const uint16_t* shift, const uint16_t* scale,
+                                       int64_t tokens_per_sample, float eps, const float* params,
+                                       uint8_t* q_packed, uint8_t* scales_tiled, void* stream) {
+  int rc = check_adaln(x, M, d, shift, scale, tokens_per_sample, eps, params);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!q_packed || !scales_tiled || reinterpret_cast<uintptr_t>(q_packed) % 16 != 0)
+    return KQ_ERR_INVALID;
+  return launch_adaln(x, M, d, shift, scale, tokens_per_sample, eps, params, q_packed,
+                      scales_tiled, nullptr, static_cast<cudaStream_t>(stream), true);
 }
 
 extern "C" int kq_transform_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
