@@ -281,6 +281,26 @@ def abs_transform16(x64: np.ndarray, params16: np.ndarray) -> np.ndarray:
     return _apply_blocks(np.abs(x64), lambda j: np.abs(kron_block(params16[j])), BLOCK16)
 
 
+def fold_weight16(w64: np.ndarray, params16: np.ndarray) -> np.ndarray:
+    """``W' = W T16^-T``: each 16-column block of a weight row times
+    ``(K16^(j))^-T`` (Eq. 1 with 16-element blocks)."""
+    params16 = np.asarray(params16)
+    return _apply_blocks(w64, lambda j: inverse_block(params16[j]).T, BLOCK16)
+
+
+def abs_fold_weight16(w64: np.ndarray, params16: np.ndarray) -> np.ndarray:
+    params16 = np.asarray(params16)
+    return _apply_blocks(np.abs(w64), lambda j: np.abs(inverse_block(params16[j]).T), BLOCK16)
+
+
+def quantize_weight16(w_bits: np.ndarray, params16: np.ndarray):
+    """MXFP4 with 16-element blocks of ``W T16^-T``: (packed codes, scales
+    ``[N, d/16]``)."""
+    codes, scales = mxfp4_quantize(fold_weight16(bf16_bits_to_float64(w_bits), params16),
+                                   BLOCK16)
+    return pack_codes(codes), scales
+
+
 def quantize16(x_bits: np.ndarray, params16: np.ndarray):
     """bf16 bits ``[M, d]`` -> (packed codes ``[M, d/2]``, scales ``[M, d/16]``)."""
     codes, scales = mxfp4_quantize(transform16(bf16_bits_to_float64(x_bits), params16), BLOCK16)

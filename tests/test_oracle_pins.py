@@ -592,3 +592,34 @@ def test_scales_to_mma_hand_positions():
     s = np.zeros((400, 4), dtype=np.uint8)
     s[256 + 100, 2] = 9                        # tile row 2: r0 = 4, r1 = 3
     assert np.flatnonzero(o.scales_to_mma(s)).tolist() == [2 * 512 + 16 * 4 + 4 * 3 + 2]
+
+
+def test_fold_weight16_keeps_the_layer_output_eq1():
+    rng = np.random.default_rng(41)
+    p16 = w.draw_params16(64, seed=42)
+    x = rng.standard_normal((5, 64))
+    W = rng.standard_normal((7, 64))
+    lhs = o.transform16(x, p16) @ o.fold_weight16(W, p16).T
+    np.testing.assert_allclose(lhs, x @ W.T, rtol=1e-10, atol=1e-10)
+
+
+def test_block16_product_brute_force():
+    """mxfp4_gemm with 16-element scale blocks against a triple loop over
+    hand-decoded values."""
+    rng = np.random.default_rng(43)
+    M, N, K = 2, 3, 64
+    ca = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    cb = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    sa = rng.integers(120, 135, (M, K // 16), dtype=np.uint8)
+    sb = rng.integers(120, 135, (N, K // 16), dtype=np.uint8)
+    table = [0, 0.5, 1, 1.5, 2, 3, 4, 6]
+
+    def val(code, s):
+        v = table[int(code) & 7] * 2.0 ** (int(s) - 127)
+        return -v if code & 8 else v
+
+    C = o.mxfp4_gemm(_pack_hand(ca), sa, _pack_hand(cb), sb, block=16)
+    for m in range(M):
+        for n in range(N):
+            assert C[m, n] == sum(val(ca[m, k], sa[m, k // 16]) * val(cb[n, k], sb[n, k // 16])
+                                  for k in range(K))
