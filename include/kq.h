@@ -113,6 +113,27 @@ int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float* params,
 int kq_quantize16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
                   uint8_t* q_packed, uint8_t* scales16, void* stream);
 
+/* The block-16 weight side and W4A4 product (Eq. 1 with 16-element
+ * blocks): kq_quantize_weight16 writes MXFP4 of W T16^-T with a scale per 16
+ * (codes [N][d/2], scales16 [N][d/16], 2-byte aligned), kq_fold_weight16
+ * writes W T16^-T in float32.  The _tiled variants (and kq_quantize16_tiled)
+ * write the scales in the tiled layout of kq_gemm_mxfp4_tiled with d/16
+ * scales a row (kq_scales16_tiled_bytes(rows, d) bytes, 16-byte aligned).
+ * kq_gemm_mxfp4_16_tiled is C = A B^T for such operands on the tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, block16 scaling with E8M0 scales). */
+int kq_quantize_weight16(const uint16_t* w, int64_t N, int64_t d, const float* params16,
+                         uint8_t* q_packed, uint8_t* scales16, void* stream);
+int kq_fold_weight16(const uint16_t* w, int64_t N, int64_t d, const float* params16,
+                     float* w_folded, void* stream);
+int kq_quantize16_tiled(const uint16_t* x, int64_t M, int64_t d, const float* params16,
+                        uint8_t* q_packed, uint8_t* scales16_tiled, void* stream);
+int kq_quantize_weight16_tiled(const uint16_t* w, int64_t N, int64_t d, const float* params16,
+                               uint8_t* q_packed, uint8_t* scales16_tiled, void* stream);
+size_t kq_scales16_tiled_bytes(int64_t rows, int64_t K);
+int kq_gemm_mxfp4_16_tiled(const uint8_t* qa, const uint8_t* sa16_tiled, const uint8_t* qb,
+                           const uint8_t* sb16_tiled, int64_t M, int64_t N, int64_t K, void* c,
+                           int c_dtype, void* stream);
+
 /* y = x T16 in float32 (the kq_quantize16 transform without quantization). */
 int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
                    float* y, void* stream);

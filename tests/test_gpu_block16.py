@@ -146,3 +146,66 @@ def test_block16_empty_and_invalid():
                             torch.cuda.current_stream().cuda_stream)
     assert st == 1
     assert kq.device_status() == 0
+
+
+# ----------------------------------------------- block-16 W4A4 layer path
+def test_block16_weight_fold_and_quantizer():
+    c = w.make_case("flux_schnell", 0, 0, M=16)
+    p16 = w.draw_params16(c.d, c.seed)
+    W = w.draw_weight(150, c.d, c.seed)
+    pd = _dev(p16)
+    q, s = kq.quantize_weight16(W.to(DEV), pd)
+    f = kq.fold_weight16(W.to(DEV), pd)
+    torch.cuda.synchronize()
+    w64 = o.bf16_bits_to_float64(_bits(W))
+    f64 = o.fold_weight16(w64, p16)
+    cond = o.abs_fold_weight16(w64, p16)
+    check_transform(f.cpu().numpy(), f64, cond)
+    st = check_mx4(q.cpu().numpy(), s.cpu().numpy(), f64, cond, block=16)
+    assert st["scale_exempt"] <= 2 and st["code_exempt"] <= 8
+
+
+@pytest.mark.parametrize("name,di,N", [("pixart_sigma", 0, 1152), ("sana", 0, 2240),
+                                       ("stress", 0, 520)], ids=lambda v: str(v))
+def test_block16_layer_product(name, di, N):
+    """Block-16 quantizers with tiled scales feed the block16 tensor-core
+    product; the codes match the row-major quantizers, the tiled scales the
+    oracle's tiled image, and the product the oracle's exact product of the
+    GPU's operands within the float32-accumulation bound."""
+    c = w.make_case(name, di, 0, M=200)
+    p16 = w.draw_params16(c.d, c.seed)
+    W = w.draw_weight(N, c.d, c.seed)
+    pd, xd, wd = _dev(p16), c.x.to(DEV), W.to(DEV)
+    qa, sa = kq.quantize16(xd, pd)
+    qb, sb = kq.quantize_weight16(wd, pd)
+    qat, sat = kq.quantize16_tiled(xd, pd)
+    qbt, sbt = kq.quantize_weight16_tiled(wd, pd)
+    C = kq.gemm_mxfp4_16_tiled(qat, sat, qbt, sbt)
+    C16 = kq.gemm_mxfp4_16_tiled(qat, sat, qbt, sbt, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(qa, qat) and torch.equal(qb, qbt)
+    assert np.array_equal(sat.cpu().numpy(), o.scales_to_mma(sa.cpu().numpy()))
+    assert np.array_equal(sbt.cpu().numpy(), o.scales_to_mma(sb.cpu().numpy()))
+    assert torch.equal(C16, C.to(torch.bfloat16))
+    qa_, sa_, qb_, sb_ = (t.cpu().numpy() for t in (qa, sa, qb, sb))
+    ref = o.mxfp4_gemm(qa_, sa_, qb_, sb_, block=16)
+    mag = o.abs_mxfp4_gemm(qa_, sa_, qb_, sb_, block=16)
+    K = c.d
+    assert (np.abs(C.cpu().numpy() - ref) <= (K / 64 + 1) * 2.0 ** -22 * mag).all()
+
+
+def test_block16_product_random_operands_and_exact_sums():
+    rng = np.random.default_rng(77)
+    for (M, N, K) in [(130, 300, 544), (128, 256, 64), (257, 520, 2240)]:
+        ca = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+        cb = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+        lo, hi = (127, 128) if K == 64 else (120, 135)
+        sa = rng.integers(lo, hi, (M, K // 16), dtype=np.uint8)
+        sb = rng.integers(lo, hi, (N, K // 16), dtype=np.uint8)
+        C = kq.gemm_mxfp4_16_tiled(_dev(ca), _dev(o.scales_to_mma(sa)), _dev(cb),
+                                   _dev(o.scales_to_mma(sb))).cpu().numpy()
+        ref = o.mxfp4_gemm(ca, sa, cb, sb, block=16)
+        if K == 64:
+            assert np.array_equal(C.astype(np.float64), ref)   # small exact sums
+        mag = o.abs_mxfp4_gemm(ca, sa, cb, sb, block=16)
+        assert (np.abs(C - ref) <= (K / 64 + 1) * 2.0 ** -22 * mag).all(), (M, N, K)

@@ -32,6 +32,12 @@ SIGNATURES = {
     "kq_quantize_smooth": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_transform": [_p, _i64, _i64, _p, _p, _p],
     "kq_quantize16": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_quantize_weight16": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_fold_weight16": [_p, _i64, _i64, _p, _p, _p],
+    "kq_quantize16_tiled": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_quantize_weight16_tiled": [_p, _i64, _i64, _p, _p, _p, _p],
+    "kq_scales16_tiled_bytes": [_i64, _i64],
+    "kq_gemm_mxfp4_16_tiled": [_p, _p, _p, _p, _i64, _i64, _i64, _p, _int, _p],
     "kq_transform16": [_p, _i64, _i64, _p, _p, _p],
     "kq_quantize_weight": [_p, _i64, _i64, _p, _p, _p, _p],
     "kq_fold_weight": [_p, _i64, _i64, _p, _p, _p],
@@ -66,7 +72,8 @@ _RESTYPE = {"kq_status_string": ctypes.c_char_p,
             "kq_quantize_host_workspace_bytes": ctypes.c_size_t,
             "kq_transform_params_grad_workspace_bytes": ctypes.c_size_t,
             "kq_residual_workspace_bytes": ctypes.c_size_t,
-            "kq_scales_tiled_bytes": ctypes.c_size_t}
+            "kq_scales_tiled_bytes": ctypes.c_size_t,
+            "kq_scales16_tiled_bytes": ctypes.c_size_t}
 
 
 class KQError(RuntimeError):
@@ -222,6 +229,80 @@ def quantize16(x: torch.Tensor, params16: torch.Tensor, q=None, scales16=None):
                              scales16.data_ptr(), _stream(x.device))
     _check("kq_quantize16", st)
     return q, scales16
+
+
+def quantize_weight16(w: torch.Tensor, params16: torch.Tensor, q=None, scales16=None):
+    """MXFP4 with 16-element blocks of W T16^-T: (codes [N, d/2], scales [N, d/16])."""
+    _dev_tensor(w, torch.bfloat16, "w")
+    N, d = _shape(w)
+    _params16(params16, d)
+    if q is None:
+        q = torch.empty((N, d // 2), dtype=torch.uint8, device=w.device)
+    if scales16 is None:
+        scales16 = torch.empty((N, d // 16), dtype=torch.uint8, device=w.device)
+    st = lib().kq_quantize_weight16(w.data_ptr(), N, d, params16.data_ptr(), q.data_ptr(),
+                                    scales16.data_ptr(), _stream(w.device))
+    _check("kq_quantize_weight16", st)
+    return q, scales16
+
+
+def fold_weight16(w: torch.Tensor, params16: torch.Tensor, out=None):
+    """W T16^-T in float32."""
+    _dev_tensor(w, torch.bfloat16, "w")
+    N, d = _shape(w)
+    _params16(params16, d)
+    if out is None:
+        out = torch.empty((N, d), dtype=torch.float32, device=w.device)
+    st = lib().kq_fold_weight16(w.data_ptr(), N, d, params16.data_ptr(), out.data_ptr(),
+                                _stream(w.device))
+    _check("kq_fold_weight16", st)
+    return out
+
+
+def _quantize16_tiled(fn, x, params16, q=None, scales=None):
+    _dev_tensor(x, torch.bfloat16, "x")
+    M, d = _shape(x)
+    _params16(params16, d)
+    if q is None:
+        q = torch.empty((M, d // 2), dtype=torch.uint8, device=x.device)
+    n = int(lib().kq_scales16_tiled_bytes(M, d))
+    if scales is None:
+        scales = torch.zeros((n,), dtype=torch.uint8, device=x.device)
+    if scales.numel() < n:
+        raise ValueError("scales must hold kq_scales16_tiled_bytes(M, d) bytes")
+    st = getattr(lib(), fn)(x.data_ptr(), M, d, params16.data_ptr(), q.data_ptr(),
+                            scales.data_ptr(), _stream(x.device))
+    _check(fn, st)
+    return q, scales
+
+
+def quantize16_tiled(x, params16, q=None, scales=None):
+    return _quantize16_tiled("kq_quantize16_tiled", x, params16, q, scales)
+
+
+def quantize_weight16_tiled(w, params16, q=None, scales=None):
+    return _quantize16_tiled("kq_quantize_weight16_tiled", w, params16, q, scales)
+
+
+def gemm_mxfp4_16_tiled(qa, sa16_tiled, qb, sb16_tiled, out=None, out_dtype=torch.float32):
+    """C = A B^T for block-16 operands with tiled scales."""
+    for t, n in ((qa, "qa"), (sa16_tiled, "sa16_tiled"), (qb, "qb"), (sb16_tiled, "sb16_tiled")):
+        _dev_tensor(t, torch.uint8, n)
+    M, K = qa.shape[0], 2 * qa.shape[1]
+    N = qb.shape[0]
+    if tuple(qb.shape) != (N, K // 2):
+        raise ValueError("qb must be [N, K/2]")
+    if sa16_tiled.numel() < lib().kq_scales16_tiled_bytes(M, K) or \
+            sb16_tiled.numel() < lib().kq_scales16_tiled_bytes(N, K):
+        raise ValueError("tiled scale arrays are too small")
+    if out is None:
+        out = torch.empty((M, N), dtype=out_dtype, device=qa.device)
+    code = KQ_OUT_F32 if out_dtype == torch.float32 else KQ_OUT_BF16
+    st = lib().kq_gemm_mxfp4_16_tiled(qa.data_ptr(), sa16_tiled.data_ptr(), qb.data_ptr(),
+                                      sb16_tiled.data_ptr(), M, N, K, out.data_ptr(), code,
+                                      _stream(qa.device))
+    _check("kq_gemm_mxfp4_16_tiled", st)
+    return out
 
 
 def transform16(x: torch.Tensor, params16: torch.Tensor, y=None):

@@ -412,7 +412,9 @@ struct PlainFactors16 {
 
 constexpr int kFactors16 = 4;
 
-// p: the 2 x 4 x 3 parameters of the unit's two blocks.
+// p: the 2 x 4 x 3 parameters of the unit's two blocks; kInvT as for
+// load_shear_diag.
+template <bool kInvT = false>
 __device__ __forceinline__ bool load_shear_diag16(ShearDiag16& f, const float* p) {
   bool ok = true;
 #pragma unroll
@@ -424,10 +426,11 @@ __device__ __forceinline__ bool load_shear_diag16(ShearDiag16& f, const float* p
 #pragma unroll
     for (int k = 0; k < kFactors16; ++k) {
       double a00, a01, a10, a11;
-      factor_entries(ph, k, a00, a01, a10, a11);
+      factor_entries<kInvT>(ph, k, a00, a01, a10, a11);
       g00[k] = a00;
       g11[k] = a11;
-      const double ra = ph[3 * k + 0], rb = a01 / a11;
+      const double ra = kInvT ? a10 / a00 : static_cast<double>(ph[3 * k + 0]);
+      const double rb = a01 / a11;
       ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
       growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
       r10[k] = (float)ra;
@@ -452,13 +455,14 @@ __device__ __forceinline__ bool load_shear_diag16(ShearDiag16& f, const float* p
   return ok;
 }
 
+template <bool kInvT = false>
 __device__ __forceinline__ void load_plain16(PlainFactors16& f, const float* p) {
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
 #pragma unroll
     for (int k = 0; k < kFactors16; ++k) {
       double g00, g01, g10, g11;
-      factor_entries(p + 12 * h, k, g00, g01, g10, g11);
+      factor_entries<kInvT>(p + 12 * h, k, g00, g01, g10, g11);
       const float f00 = (float)g00, f01 = (float)g01, f10 = (float)g10, f11 = (float)g11;
       if (k < 3) {
         f.g00[h][k] = pack2(f00, f00);

@@ -155,16 +155,49 @@ __device__ __forceinline__ void load_sf_words(uint32_t (&v)[kSfWordsPerLane], co
 // words when every row's scales are 4-byte aligned, bytes otherwise), or
 // the tiled layout (128-row x 4-scale tiles of 512 bytes), which the
 // producer thread copies straight into the stage with bulk copies.
-enum SfMode { kSfRowWords = 0, kSfRowBytes = 1, kSfTiled = 2 };
+// kSfTiled16: tiled scales with one scale per 16 elements along K (the
+// 16-element variant), MMAs of kind::mxf4nvf4 with block16 scaling.
+enum SfMode { kSfRowWords = 0, kSfRowBytes = 1, kSfTiled = 2, kSfTiled16 = 3 };
+
+// Per-stage scale geometry: 4-scale chunks of 128 rows per stage (two for
+// scales per 32, four for scales per 16), their bytes and TMEM columns.
+template <int kSfMode>
+struct StageGeom {
+  static constexpr int kChunks = kSfMode == kSfTiled16 ? 4 : kChunksPerStage;
+  static constexpr int kSfa = kChunks * kSfChunk;
+  static constexpr int kSfb = kChunks * (kBN / 128) * kSfChunk;
+  static constexpr int kStage = kATile + kBTile + kSfa + kSfb;
+  static constexpr int kColsA = 4 * kChunks;
+  static constexpr int kColsB = 8 * kChunks;
+  static constexpr int kSmem = 1024 + kStages * kStage + (2 * kStages + 2) * 8 + 16;
+  static_assert(kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+  static_assert(kSfCol0 + kStages * (kColsA + kColsB) <= kTmemCols, "TMEM columns");
+  static_assert(kSmem <= 232448, "shared memory");
+};
+
+// Block-scaled MMA with a scale per 16 elements: four E8M0 scales of each
+// row per K = 64 (the whole 32-bit TMEM word, scale-factor id 0).
+__device__ __forceinline__ void mma_mxf4_b16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                             uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;"
+      "\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
 
 template <int kSfMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap,
                      const __grid_constant__ CUtensorMap bmap,
                      const __grid_constant__ CUtensorMap cmap, const GemmArgs a) {
+  using Geo = StageGeom<kSfMode>;
+  constexpr bool kTiledSf = kSfMode == kSfTiled || kSfMode == kSfTiled16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(base + kStages * Geo::kStage);
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* mma_done = acc_full + 1;
@@ -185,12 +218,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
   const int nk = a.k_tiles;
 
-  if (kSfMode == kSfTiled) {
+  if (kTiledSf) {
     // Chunks past the end of K are not copied; their codes are zero, and
     // the scales there must only be finite.
     for (int s = 0; s < kStages; ++s)
-      for (int i = tid; i < (kSfaBytes + kSfbBytes) / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(base + s * kStageBytes + kATile + kBTile)[i] =
+      for (int i = tid; i < (Geo::kSfa + Geo::kSfb) / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(base + s * Geo::kStage + kATile + kBTile)[i] =
             make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
   }
@@ -198,7 +231,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       // TMA bytes, plus the stage's scale warp unless the scales come by
       // bulk copy with the codes.
-      mbar_init(&full[s], kSfMode == kSfTiled ? 1 : 2);
+      mbar_init(&full[s], kTiledSf ? 1 : 2);
       mbar_init(&empty[s], 1);                     // tcgen05.commit of the stage's MMAs
     }
     mbar_init(acc_full, 1);
@@ -224,20 +257,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ok = false;
           break;
         }
-        uint8_t* st = base + s * kStageBytes;
-        if (kSfMode == kSfTiled) {
+        uint8_t* st = base + s * Geo::kStage;
+        if (kTiledSf) {
           // This k-tile's scale columns 2 kt, 2 kt + 1 (those that exist) of
           // the A row tile and of the (up to) two B row tiles.
-          const int avail = min(kChunksPerStage, a.sf_tiles_k - kChunksPerStage * kt);
+          const int avail = min(Geo::kChunks, a.sf_tiles_k - Geo::kChunks * kt);
           const int b_tiles = min(kBN / 128, a.sf_tiles_n - n0 / 128);
           const uint32_t sf_bytes = (uint32_t)(avail * (1 + b_tiles)) * kSfChunk;
           mbar_arrive_expect_tx(&full[s], kATile + kBTile + sf_bytes);
           uint8_t* sfa = st + kATile + kBTile;
-          bulk_load(sfa, a.sa + ((int64_t)(m0 / 128) * a.sf_tiles_k + kChunksPerStage * kt) *
+          bulk_load(sfa, a.sa + ((int64_t)(m0 / 128) * a.sf_tiles_k + Geo::kChunks * kt) *
                                   kSfChunk, avail * kSfChunk, &full[s]);
           for (int g = 0; g < b_tiles; ++g)
-            bulk_load(sfa + kSfaBytes + g * kChunksPerStage * kSfChunk,
-                      a.sb + ((int64_t)(n0 / 128 + g) * a.sf_tiles_k + kChunksPerStage * kt) *
+            bulk_load(sfa + Geo::kSfa + g * Geo::kChunks * kSfChunk,
+                      a.sb + ((int64_t)(n0 / 128 + g) * a.sf_tiles_k + Geo::kChunks * kt) *
                                  kSfChunk, avail * kSfChunk, &full[s]);
         } else {
           mbar_arrive_expect_tx(&full[s], kATile + kBTile);
@@ -259,15 +292,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     return;
   }
 
-  if (kSfMode != kSfTiled && warp >= kSfWarp0) {
+  if (!kTiledSf && warp >= kSfWarp0) {
     // ---------------------------------------------------------- scale loader
     // Loader warp sw owns stage sw (k-tiles sw, sw + 4, ...), so a stage's
     // scales have four k-tiles of MMA time to arrive; all of a stage's
     // loads are in flight together before the stores.
     const int sw = warp - kSfWarp0;
     const int s = sw;
-    uint8_t* sfa = base + s * kStageBytes + kATile + kBTile;
-    uint8_t* sfb = sfa + kSfaBytes;
+    uint8_t* sfa = base + s * Geo::kStage + kATile + kBTile;
+    uint8_t* sfb = sfa + Geo::kSfa;
     for (int kt = sw, n = 0; kt < nk; kt += kStages, ++n) {
       uint32_t cur[kSfWordsPerLane];
       load_sf_words<kSfMode == kSfRowWords>(cur, a, m0, n0, kt, lane);
@@ -306,28 +339,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           break;
         }
         tmem_fence_after();
-        const uint8_t* st = base + s * kStageBytes;
+        const uint8_t* st = base + s * Geo::kStage;
         const uint8_t* sfa = st + kATile + kBTile;
-        const uint8_t* sfb = sfa + kSfaBytes;
-        const uint32_t tsfa = tmem_base + kSfCol0 + s * (kSfColsA + kSfColsB);
-        const uint32_t tsfb = tsfa + kSfColsA;
+        const uint8_t* sfb = sfa + Geo::kSfa;
+        const uint32_t tsfa = tmem_base + kSfCol0 + s * (Geo::kColsA + Geo::kColsB);
+        const uint32_t tsfb = tsfa + Geo::kColsA;
 #pragma unroll
-        for (int c = 0; c < kChunksPerStage; ++c) {
+        for (int c = 0; c < Geo::kChunks; ++c) {
           tmem_cp_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
 #pragma unroll
           for (int g = 0; g < kBN / 128; ++g)
             tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * g,
-                               smem_desc_rows16(smem_addr(sfb + (2 * g + c) * kSfChunk)));
+                               smem_desc_rows16(smem_addr(sfb + (Geo::kChunks * g + c) * kSfChunk)));
         }
         const uint64_t adesc = smem_desc_sw128(smem_addr(st));
         const uint64_t bdesc = smem_desc_sw128(smem_addr(st + kATile));
 #pragma unroll
         for (int kk = 0; kk < kBK / kMmaK; ++kk) {
           // 64 codes = 32 bytes per MMA: the start address steps by 2 (x16 B).
-          const uint32_t sf_id = 2u * (kk & 1);
-          const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
-          mma_mxf4(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
-                   tsfb + 8 * (kk >> 1), (kt | kk) != 0);
+          if constexpr (kSfMode == kSfTiled16) {
+            // Four scales per row and MMA: chunk kk, the whole word.
+            mma_mxf4_b16(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, kIdescMxf4, tsfa + 4 * kk,
+                         tsfb + 8 * kk, (kt | kk) != 0);
+          } else {
+            const uint32_t sf_id = 2u * (kk & 1);
+            const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
+            mma_mxf4(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
+                     tsfb + 8 * (kk >> 1), (kt | kk) != 0);
+          }
         }
         mma_commit(&empty[s]);         // stage (codes and scales) free once read
         if (++s == kStages) {
@@ -725,7 +764,7 @@ bool persistent_gemm(int64_t K) {
 
 int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
                 int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream,
-                bool tiled) {
+                bool tiled, int scale_block = 32) {
   if (M < 0 || N < 0 || K < 32 || K % 32 != 0) return KQ_ERR_INVALID;
   if (c_dtype != KQ_OUT_F32 && c_dtype != KQ_OUT_BF16) return KQ_ERR_INVALID;
   if (M == 0 || N == 0) return KQ_OK;
@@ -750,7 +789,7 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   a.m_tiles = static_cast<int32_t>((M + kBM - 1) / kBM);
   a.n_tiles = static_cast<int32_t>((N + kBN - 1) / kBN);
   a.sf_stride = static_cast<int32_t>(K / 32);
-  a.sf_tiles_k = static_cast<int32_t>((K / 32 + 3) / 4);
+  a.sf_tiles_k = static_cast<int32_t>((K / scale_block + 3) / 4);
   a.sf_tiles_n = static_cast<int32_t>((N + 127) / 128);
   a.out_bf16 = c_dtype == KQ_OUT_BF16;
   a.sa = sa;
@@ -778,7 +817,12 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   }
   const dim3 grid(static_cast<unsigned>(a.m_tiles * a.n_tiles));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (tiled && a.tma_store && persistent_gemm(K)) {
+  if (scale_block == 16) {
+    using G = StageGeom<kSfTiled16>;
+    rc = allow_smem<gemm_mxf4_kernel<kSfTiled16>>(G::kSmem, dev);
+    if (rc != KQ_OK) return rc;
+    gemm_mxf4_kernel<kSfTiled16><<<grid, 32 * kSfWarp0, G::kSmem, st>>>(amap, bmap, cmap, a);
+  } else if (tiled && a.tma_store && persistent_gemm(K)) {
     rc = allow_smem<gemm_mxf4_persistent>(kPSmemBytes, dev);
     if (rc != KQ_OK) return rc;
     const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
@@ -834,6 +878,17 @@ extern "C" int kq_gemm_mxfp4_tiled(const uint8_t* qa, const uint8_t* sa_tiled, c
                                    const uint8_t* sb_tiled, int64_t M, int64_t N, int64_t K,
                                    void* c, int c_dtype, void* stream) {
   return launch_gemm(qa, sa_tiled, qb, sb_tiled, M, N, K, c, c_dtype, stream, true);
+}
+
+extern "C" int kq_gemm_mxfp4_16_tiled(const uint8_t* qa, const uint8_t* sa16_tiled,
+                                      const uint8_t* qb, const uint8_t* sb16_tiled, int64_t M,
+                                      int64_t N, int64_t K, void* c, int c_dtype, void* stream) {
+  return launch_gemm(qa, sa16_tiled, qb, sb16_tiled, M, N, K, c, c_dtype, stream, true, 16);
+}
+
+extern "C" size_t kq_scales16_tiled_bytes(int64_t rows, int64_t K) {
+  if (rows < 1 || K < 32 || K % 32 != 0) return 0;
+  return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((K / 16 + 3) / 4) * 512;
 }
 
 extern "C" size_t kq_scales_tiled_bytes(int64_t rows, int64_t K) {

@@ -37,10 +37,14 @@ int record_cuda_error(cudaError_t e) {
 // kXfKron16: 16-element Kronecker blocks (four factors each) with a scale
 // per 16 elements; a thread owns a unit of two adjacent 16-blocks.
 // kXfKronInvT: the weight-side fold W T^-T, factors (G_k^-1)^T.
-enum Xform { kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2, kXfKron16 = 3, kXfKronInvT = 4 };
+// kXfKron16InvT: the weight-side fold with 16-element blocks.
+enum Xform {
+  kXfKron = 0, kXfHadamard = 1, kXfSmooth = 2, kXfKron16 = 3, kXfKronInvT = 4, kXfKron16InvT = 5
+};
 
-// Transforms made of five 2x2 factors per 32-block.
+// Transforms made of five 2x2 factors per 32-block, and of four per 16-block.
 __host__ __device__ constexpr bool kron5(int xf) { return xf == kXfKron || xf == kXfKronInvT; }
+__host__ __device__ constexpr bool kron4(int xf) { return xf == kXfKron16 || xf == kXfKron16InvT; }
 enum Out { kOutMx4 = 0, kOutF32 = 1 };
 
 constexpr int kConsumerWarps = 8;
@@ -320,7 +324,7 @@ __device__ __forceinline__ void panel_consume(const PanelArgs& a, const uint8_t*
         u[4 * q + 2] = bf16x2_to_f2(c[r][q].z);
         u[4 * q + 3] = bf16x2_to_f2(c[r][q].w);
       }
-      if constexpr (kXf == kXfKron16) {
+      if constexpr (kron4(kXf)) {
         if constexpr (kForm == 1) {
           plain_apply16(u, pf);
         } else {
@@ -336,11 +340,20 @@ __device__ __forceinline__ void panel_consume(const PanelArgs& a, const uint8_t*
         diag_mul(u, sd.delta);
       }
       const int64_t g = rr * a.nb + j;
-      if constexpr (kOut == kOutMx4 && kXf == kXfKron16) {
+      if constexpr (kOut == kOutMx4 && kron4(kXf)) {
         // Two scale bytes per unit, block 0 at the lower address.
         const Mx4Block b = mxfp4_block16x2(u);
         __stcs(reinterpret_cast<uint4*>(a.q + g * 16), b.codes);
-        reinterpret_cast<uint16_t*>(a.scales)[g] = static_cast<uint16_t>(b.scale);
+        if (a.scale_tiles_k == 0) {
+          reinterpret_cast<uint16_t*>(a.scales)[g] = static_cast<uint16_t>(b.scale);
+        } else {
+          // Tiled layout, scale columns 2 j and 2 j + 1 (one 4-byte word
+          // half); an odd count of units leaves half a 4-scale column of
+          // padding, zeroed by the row's last unit.
+          const int64_t o = tiled_scale_offset(rr, 2 * j, a.scale_tiles_k);
+          *reinterpret_cast<uint16_t*>(a.scales + o) = static_cast<uint16_t>(b.scale);
+          if (j == a.nb - 1 && (j & 1) == 0) *reinterpret_cast<uint16_t*>(a.scales + o + 2) = 0;
+        }
       } else if constexpr (kOut == kOutMx4) {
         const Mx4Block b = mxfp4_block(u);
         __stcs(reinterpret_cast<uint4*>(a.q + g * 16), b.codes);
@@ -429,12 +442,12 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   const bool active = tid < a.W * a.R;
   const int rho = tid / a.W;
   const int j = panel * a.W + (tid % a.W);
-  using SD = std::conditional_t<kXf == kXfKron16, ShearDiag16, ShearDiag>;
-  using PF = std::conditional_t<kXf == kXfKron16, PlainFactors16, PlainFactors>;
+  using SD = std::conditional_t<kron4(kXf), ShearDiag16, ShearDiag>;
+  using PF = std::conditional_t<kron4(kXf), PlainFactors16, PlainFactors>;
   SD sd;
   PF pf;
   int plain = 0;
-  if constexpr (kron5(kXf) || kXf == kXfKron16) {
+  if constexpr (kron5(kXf) || kron4(kXf)) {
     // Parameters per thread unit: 5 x 3 for a 32-block, 2 x 4 x 3 for a pair
     // of 16-blocks.
     constexpr int kUnitParams = kron5(kXf) ? 15 : 24;
@@ -442,7 +455,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     if constexpr (kron5(kXf)) {
       if (active) plain = load_shear_diag<kXf == kXfKronInvT>(sd, p) ? 0 : 1;
     } else {
-      if (active) plain = load_shear_diag16(sd, p) ? 0 : 1;
+      if (active) plain = load_shear_diag16<kXf == kXfKron16InvT>(sd, p) ? 0 : 1;
     }
     // One form for the whole CTA: the plain one if any of its blocks needs it.
     asm volatile(
@@ -453,7 +466,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
         : "memory");
     if (plain && active) {
       if constexpr (kron5(kXf)) load_plain<kXf == kXfKronInvT>(pf, p);
-      else load_plain16(pf, p);
+      else load_plain16<kXf == kXfKron16InvT>(pf, p);
     }
   } else if constexpr (kXf == kXfSmooth) {
     if (active) {
@@ -738,7 +751,7 @@ int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, 
   // The 16-element variant and the weight fold have no other kernel, so
   // they take any shape.
   const double min_use =
-      (kXf == kXfKron16 || kXf == kXfKronInvT || scale_tiles_k > 0) ? 0.0 : 0.5;
+      (kron4(kXf) || kXf == kXfKronInvT || scale_tiles_k > 0) ? 0.0 : 0.5;
   if (panel_use<Cfg>(nb, di.sms, &a.W, &a.R) < min_use) return KQ_ERR_INVALID;
   a.M = M;
   a.nb = nb;
@@ -846,7 +859,7 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
   a.inverse = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nb = d / kBlock;
-  if constexpr (kXf == kXfKron16 || kXf == kXfKronInvT) {
+  if constexpr (kron4(kXf) || kXf == kXfKronInvT) {
     // Only the panel kernel carries the 16-element variant and the fold.
     if (impl != KQ_IMPL_PANEL || nb > 65535) return KQ_ERR_INVALID;
     return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
@@ -872,7 +885,8 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
   }
 }
 
-// The panel kernel with scales written in the tiled layout.
+// The panel kernel with scales written in the tiled layout (4-scale
+// columns: d/32 scales a row, or d/16 for the 16-element variants).
 template <int kXf>
 int run_tiled(const uint16_t* x, int64_t M, int64_t d, const float* params, uint8_t* q,
               uint8_t* scales_tiled, void* stream) {
@@ -882,9 +896,10 @@ int run_tiled(const uint16_t* x, int64_t M, int64_t d, const float* params, uint
   if (rc != KQ_OK) return rc;
   const int64_t nb = d / kBlock;
   if (nb > 65535) return KQ_ERR_INVALID;
+  const int64_t ns = kron4(kXf) ? 2 * nb : nb;
   return launch_panel<kXf, kOutMx4>(x, M, d, params, q, scales_tiled, nullptr,
                                     static_cast<cudaStream_t>(stream), *di, dev,
-                                    static_cast<int32_t>((nb + 3) / 4));
+                                    static_cast<int32_t>((ns + 3) / 4));
 }
 
 int check_quant_args(const uint16_t* x, int64_t M, int64_t d, const void* aux, bool need_aux,
@@ -957,6 +972,45 @@ extern "C" int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const flo
       d / kBlock > 65535)
     return KQ_ERR_INVALID;
   return run<kXfKron16, kOutF32>(x, M, d, params16, nullptr, nullptr, y, KQ_IMPL_PANEL, stream);
+}
+
+extern "C" int kq_quantize16_tiled(const uint16_t* x, int64_t M, int64_t d,
+                                   const float* params16, uint8_t* q_packed,
+                                   uint8_t* scales16_tiled, void* stream) {
+  int rc = check_quant_args(x, M, d, params16, true, q_packed, scales16_tiled);
+  if (rc != KQ_OK || M == 0) return rc;
+  if (!aligned(scales16_tiled, 16)) return KQ_ERR_INVALID;
+  return run_tiled<kXfKron16>(x, M, d, params16, q_packed, scales16_tiled, stream);
+}
+
+extern "C" int kq_quantize_weight16(const uint16_t* w, int64_t N, int64_t d,
+                                    const float* params16, uint8_t* q_packed, uint8_t* scales16,
+                                    void* stream) {
+  int rc = check_quant_args(w, N, d, params16, true, q_packed, scales16);
+  if (rc != KQ_OK || N == 0) return rc;
+  if (!aligned(scales16, 2) || d / kBlock > 65535) return KQ_ERR_INVALID;
+  return run<kXfKron16InvT, kOutMx4>(w, N, d, params16, q_packed, scales16, nullptr,
+                                     KQ_IMPL_PANEL, stream);
+}
+
+extern "C" int kq_quantize_weight16_tiled(const uint16_t* w, int64_t N, int64_t d,
+                                          const float* params16, uint8_t* q_packed,
+                                          uint8_t* scales16_tiled, void* stream) {
+  int rc = check_quant_args(w, N, d, params16, true, q_packed, scales16_tiled);
+  if (rc != KQ_OK || N == 0) return rc;
+  if (!aligned(scales16_tiled, 16)) return KQ_ERR_INVALID;
+  return run_tiled<kXfKron16InvT>(w, N, d, params16, q_packed, scales16_tiled, stream);
+}
+
+extern "C" int kq_fold_weight16(const uint16_t* w, int64_t N, int64_t d, const float* params16,
+                                float* w_folded, void* stream) {
+  int rc = check_shape(N, d);
+  if (rc != KQ_OK || N == 0) return rc;
+  if (!w || !params16 || !w_folded || !aligned(w, 16) || !aligned(w_folded, 16) ||
+      !aligned(params16, 4) || d / kBlock > 65535)
+    return KQ_ERR_INVALID;
+  return run<kXfKron16InvT, kOutF32>(w, N, d, params16, nullptr, nullptr, w_folded,
+                                     KQ_IMPL_PANEL, stream);
 }
 
 extern "C" int kq_quantize_weight(const uint16_t* w, int64_t N, int64_t d, const float* params,
