@@ -23,8 +23,15 @@
 // M2 = sum M2_i + n_i (m_i - m)^2, with no divisions); the segment's first
 // lane writes a slot, and after one named barrier every thread combines its
 // row's slots in a fixed order, so the result does not depend on timing.
-// Each thread keeps its block's factors and its sample's 32 shift and 32
-// scale values (bf16 pairs) in registers.
+//
+// The transform is taken with its diagonal first: every factor is
+// G = diag(g00, g11) [[1, g01/g00], [g10/g11, 1]], so K = D S with
+// D = (x) diag(g00, g11) and S the product of five unit-diagonal shears.  D
+// then merges with the modulation: h D = t alpha + beta with t = (x - mean)
+// rstd, alpha = (1 + scale[b]) D and beta = shift[b] D, per sample and
+// channel, followed by the shear stages.  A thread keeps column block j for
+// the whole kernel, so it recomputes its block's alpha and beta only when its
+// rows enter a new sample, into a slice of shared memory that only it reads.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -98,6 +105,115 @@ __device__ __forceinline__ float segment_sum(float v, uint32_t inside) {
   return v;
 }
 
+// The shear form with its diagonal first: per factor
+// G = diag(g00, g11) [[1, r01], [r10, 1]] with r01 = g01 / g00 and
+// r10 = g10 / g11, applied to a row vector v as
+// (v_lo + r10 v_hi, v_hi + r01 v_lo) after v has been scaled by the diagonal.
+// |diag| |S| = |G| entrywise, so each stage keeps the float32 error within a
+// few ulp of the magnitudes of the terms of the plain product.
+struct ShearIn {
+  f2 r10[4], r01[4];     // stages on index bits 4..1, both halves equal
+  float r10b, r01b;      // stage on bit 0
+  float g00[kFactors], g11[kFactors];
+};
+
+// Fills the form for the block with parameters p[15]; false if the block
+// must take the plain four-term stages instead (a vanishing diagonal entry,
+// or intermediate growth above the bound of the output-side shear form).
+__device__ __forceinline__ bool load_shear_in(ShearIn& f, const float* p) {
+  double growth = 1.0;
+  bool ok = true;
+  float r10[kFactors], r01[kFactors];
+#pragma unroll
+  for (int k = 0; k < kFactors; ++k) {
+    double g00, g01, g10, g11;
+    factor_entries<false>(p, k, g00, g01, g10, g11);
+    const double ra = g10 / g11, rb = g01 / g00;
+    ok = ok && (g00 != 0.0) && (g11 != 0.0) && isfinite(ra) && isfinite(rb);
+    growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
+    r10[k] = (float)ra;
+    r01[k] = (float)rb;
+    f.g00[k] = (float)g00;
+    f.g11[k] = (float)g11;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    f.r10[k] = pack2(r10[k], r10[k]);
+    f.r01[k] = pack2(r01[k], r01[k]);
+  }
+  f.r10b = r10[4];
+  f.r01b = r01[4];
+  return ok && growth <= kShearGrowthMax;
+}
+
+__device__ __forceinline__ void shear_in_apply(f2 (&u)[16], const ShearIn& f) {
+  shear_stage<8>(u, f.r10[0], f.r01[0]);
+  shear_stage<4>(u, f.r10[1], f.r01[1]);
+  shear_stage<2>(u, f.r10[2], f.r01[2]);
+  shear_stage<1>(u, f.r10[3], f.r01[3]);
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    float lo, hi;
+    unpack2(u[m], lo, hi);
+    u[m] = pack2(__fmaf_rn(f.r10b, hi, lo), __fmaf_rn(f.r01b, lo, hi));
+  }
+}
+
+// Entries 2m and 2m + 1 of the diagonal (x) diag(g00_k, g11_k), factor k on
+// index bit 4 - k, as products in float32 (at most four roundings).
+__device__ __forceinline__ void diag_pairs(const ShearIn& f, f2 (&dl)[16]) {
+  float hi2[4], lo2[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    hi2[q] = ((q & 2) ? f.g11[0] : f.g00[0]) * ((q & 1) ? f.g11[1] : f.g00[1]);
+    lo2[q] = ((q & 2) ? f.g11[2] : f.g00[2]) * ((q & 1) ? f.g11[3] : f.g00[3]);
+  }
+#pragma unroll
+  for (int m = 0; m < 16; ++m) {
+    const float t = hi2[m >> 2] * lo2[m & 3];
+    dl[m] = pack2(t * f.g00[4], t * f.g11[4]);
+  }
+}
+
+// Writes alpha = (1 + scale) delta and beta = shift delta of this thread's
+// block for sample b into its slice of the modulation table: chunk c (four
+// channels) of alpha at tab[c * kAdaCons + tid], of beta at
+// tab[(8 + c) * kAdaCons + tid], so that a warp's 16-byte reads of one chunk
+// are consecutive.  delta = 1 for the plain form.
+template <int kForm>
+__device__ __forceinline__ void load_modulation(const AdaArgs& a, int64_t b, int j, int tid,
+                                                const ShearIn& si, float4* tab) {
+  f2 dl[16];
+  if (kForm == 0) {
+    diag_pairs(si, dl);
+  } else {
+#pragma unroll
+    for (int m = 0; m < 16; ++m) dl[m] = pack2(1.0f, 1.0f);
+  }
+  const uint4* ps = reinterpret_cast<const uint4*>(a.shift + (b * a.nb + j) * 16);
+  const uint4* pc = reinterpret_cast<const uint4*>(a.scale + (b * a.nb + j) * 16);
+  const f2 one2 = pack2(1.0f, 1.0f);
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint4 vs = __ldg(ps + t), vc = __ldg(pc + t);
+    const uint32_t ws[4] = {vs.x, vs.y, vs.z, vs.w};
+    const uint32_t wc[4] = {vc.x, vc.y, vc.z, vc.w};
+    float al[8], be[8];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const f2 dd = dl[4 * t + w];
+      const f2 av = mul2(add2(bf16x2_to_f2(wc[w]), one2), dd);
+      const f2 bv = mul2(bf16x2_to_f2(ws[w]), dd);
+      unpack2(av, al[2 * w], al[2 * w + 1]);
+      unpack2(bv, be[2 * w], be[2 * w + 1]);
+    }
+    tab[(2 * t) * kAdaCons + tid] = make_float4(al[0], al[1], al[2], al[3]);
+    tab[(2 * t + 1) * kAdaCons + tid] = make_float4(al[4], al[5], al[6], al[7]);
+    tab[(8 + 2 * t) * kAdaCons + tid] = make_float4(be[0], be[1], be[2], be[3]);
+    tab[(8 + 2 * t + 1) * kAdaCons + tid] = make_float4(be[4], be[5], be[6], be[7]);
+  }
+}
+
 // Thread 0 issues the TMA load of a group into a stage.
 __device__ __forceinline__ void adaln_issue(const AdaArgs& a, const CUtensorMap* xmap,
                                             uint8_t* stage, uint64_t* bar, int g) {
@@ -115,8 +231,8 @@ __device__ __forceinline__ void adaln_issue(const AdaArgs& a, const CUtensorMap*
 template <int kOut, int kForm>
 __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMap* xmap,
                                               uint8_t* stages, uint64_t* full, uint64_t* statbar,
-                                              float4* slots, const float* delta_tab, int tid,
-                                              const ShearDiag& sd, const PlainFactors& pf) {
+                                              float4* slots, float4* modtab, int tid,
+                                              const ShearIn& si, const PlainFactors& pf) {
   const int lane = tid & 31, warp = tid >> 5;
   const int nb = a.nb, R = a.R;
   const bool active = tid < R * nb;
@@ -194,8 +310,7 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
     if (lane == 0) mbar_arrive(&statbar[k & 1]);
   };
 
-  int64_t cur_b = -1;
-  uint32_t sh[16], sc[16];                        // shift / scale of block j, bf16 pairs
+  int64_t b_end = 0;                              // first row past this thread's sample
   uint4 cn[4];
   bool ok = n_local > 0;
   int read = 0;                                   // groups whose data arrived
@@ -261,47 +376,35 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
     }
     const int64_t row = ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * R + rr;
     if (!active || row >= a.M) continue;
-    const int64_t b = row / a.tokens;
-    if (b != cur_b) {
-      cur_b = b;
-      const uint4* ps = reinterpret_cast<const uint4*>(a.shift + (b * nb + j) * 16);
-      const uint4* pc = reinterpret_cast<const uint4*>(a.scale + (b * nb + j) * 16);
-#pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        const uint4 vs = __ldg(ps + t), vc = __ldg(pc + t);
-        sh[4 * t] = vs.x; sh[4 * t + 1] = vs.y; sh[4 * t + 2] = vs.z; sh[4 * t + 3] = vs.w;
-        sc[4 * t] = vc.x; sc[4 * t + 1] = vc.y; sc[4 * t + 2] = vc.z; sc[4 * t + 3] = vc.w;
-      }
+    if (row >= b_end) {                           // rows only grow: a new sample
+      const int64_t b = row / a.tokens;
+      b_end = (b + 1) * a.tokens;
+      load_modulation<kForm>(a, b, j, tid, si, modtab);
     }
-    const float rstd = 1.0f / sqrtf(__fmaf_rn(m2, inv_d, a.eps));
-    // h = (x - mean) rstd (1 + scale) + shift, as t = x rstd - mean rstd,
-    // then h = t scale + (t + shift).
+    // rsqrtf: within 2 ulp, far inside the 1e-5 band of the modulated value.
+    const float rstd = rsqrtf(__fmaf_rn(m2, inv_d, a.eps));
+    // h D = t alpha + beta with t = x rstd - mean rstd.
     const f2 r2 = pack2(rstd, rstd), nmr2 = pack2(-mean * rstd, -mean * rstd);
     f2 u[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      u[4 * q + 0] = bf16x2_to_f2(cc[q].x);
-      u[4 * q + 1] = bf16x2_to_f2(cc[q].y);
-      u[4 * q + 2] = bf16x2_to_f2(cc[q].z);
-      u[4 * q + 3] = bf16x2_to_f2(cc[q].w);
-    }
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const f2 t = fma2(u[m], r2, nmr2);
-      u[m] = fma2(t, bf16x2_to_f2(sc[m]), add2(t, bf16x2_to_f2(sh[m])));
+      const float4 al0 = modtab[(2 * q) * kAdaCons + tid];
+      const float4 al1 = modtab[(2 * q + 1) * kAdaCons + tid];
+      const float4 be0 = modtab[(8 + 2 * q) * kAdaCons + tid];
+      const float4 be1 = modtab[(8 + 2 * q + 1) * kAdaCons + tid];
+      u[4 * q + 0] = fma2(fma2(bf16x2_to_f2(cc[q].x), r2, nmr2), pack2(al0.x, al0.y),
+                          pack2(be0.x, be0.y));
+      u[4 * q + 1] = fma2(fma2(bf16x2_to_f2(cc[q].y), r2, nmr2), pack2(al0.z, al0.w),
+                          pack2(be0.z, be0.w));
+      u[4 * q + 2] = fma2(fma2(bf16x2_to_f2(cc[q].z), r2, nmr2), pack2(al1.x, al1.y),
+                          pack2(be1.x, be1.y));
+      u[4 * q + 3] = fma2(fma2(bf16x2_to_f2(cc[q].w), r2, nmr2), pack2(al1.z, al1.w),
+                          pack2(be1.z, be1.w));
     }
     if (kForm == 1) {
       plain_apply(u, pf);
     } else {
-      shear_apply(u, sd);
-      // The diagonal of the shear form, from the block's row of the table.
-      const float* dt = delta_tab + j * 32;
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const float4 v = *reinterpret_cast<const float4*>(dt + 4 * (c8 ^ (j & 7)));
-        u[2 * c8] = mul2(u[2 * c8], pack2(v.x, v.y));
-        u[2 * c8 + 1] = mul2(u[2 * c8 + 1], pack2(v.z, v.w));
-      }
+      shear_in_apply(u, si);
     }
     const int64_t gi = row * nb + j;
     if (kOut == 0) {
@@ -348,7 +451,7 @@ __global__ void __launch_bounds__(kAdaCons, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(base + a.stages * a.stage_bytes);
   uint64_t* statbar = full + kAdaMaxStages;
   float4* slots = reinterpret_cast<float4*>(statbar + 2);            // 16-byte aligned
-  float* delta_tab = reinterpret_cast<float*>(slots + kAdaSlotBufs * kAdaSlots);
+  float4* modtab = slots + kAdaSlotBufs * kAdaSlots;               // [16][kAdaCons]
   const int tid = threadIdx.x;
   const int S = a.stages;
   if (tid == 0) {
@@ -366,22 +469,10 @@ __global__ void __launch_bounds__(kAdaCons, 1)
 
   const bool active = tid < a.R * a.nb;
   const int j = active ? tid % a.nb : 0;
-  ShearDiag sd;
+  ShearIn si;
   PlainFactors pf;
   int plain = 0;
-  if (active) plain = load_shear_diag(sd, a.params + (int64_t)j * 15) ? 0 : 1;
-  // The shear form's diagonal goes to a shared table (row j, 16-byte chunk
-  // c at c ^ (j mod 8), conflict-free for eight consecutive blocks).
-  if (active && tid < a.nb) {
-#pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-      float d0, d1, d2, d3;
-      unpack2(sd.delta[2 * c8], d0, d1);
-      unpack2(sd.delta[2 * c8 + 1], d2, d3);
-      *reinterpret_cast<float4*>(delta_tab + j * 32 + 4 * (c8 ^ (j & 7))) =
-          make_float4(d0, d1, d2, d3);
-    }
-  }
+  if (active) plain = load_shear_in(si, a.params + (int64_t)j * 15) ? 0 : 1;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
       "bar.red.or.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
@@ -390,9 +481,9 @@ __global__ void __launch_bounds__(kAdaCons, 1)
       : "memory");
   if (plain) {
     if (active) load_plain(pf, a.params + (int64_t)j * 15);
-    adaln_consume<kOut, 1>(a, &xmap, stages, full, statbar, slots, delta_tab, tid, sd, pf);
+    adaln_consume<kOut, 1>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf);
   } else {
-    adaln_consume<kOut, 0>(a, &xmap, stages, full, statbar, slots, delta_tab, tid, sd, pf);
+    adaln_consume<kOut, 0>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf);
   }
 }
 
@@ -432,8 +523,10 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   a.scales = scales;
   a.scale_tiles_k = tiled ? (nb + 3) / 4 : 0;
   a.y = y;
-  // Barriers, four slot buffers and the diagonal table (128 bytes a block).
-  const int fixed = 1024 + (kAdaMaxStages + 2) * 8 + kAdaSlotBufs * kAdaSlots * 16 + nb * 128;
+  // Barriers, four slot buffers and the modulation table (alpha and beta,
+  // 256 bytes a thread).
+  const int fixed =
+      1024 + (kAdaMaxStages + 2) * 8 + kAdaSlotBufs * kAdaSlots * 16 + 16 * kAdaCons * 16;
   a.stages = std::min(kAdaMaxStages, (di->smem_optin - fixed) / a.stage_bytes);
   if (a.stages < 2) return KQ_ERR_INVALID;
   const int smem = a.stages * a.stage_bytes + fixed;
