@@ -358,7 +358,20 @@ def run_gpu(args):
     ada_shift, ada_scale = (t.to(dev) for t in w.draw_adaln(-(-M // tokens), d, case.seed))
 
     gemm_flops = 2.0 * M * d * d
-    if args.op == "gemm":
+    gemm_mnk = [M, d, d]
+    if args.op == "gemm" and args.gemm_shape:
+        # Another layer shape M x N x K (profiling): N(0, 1) activations and
+        # weights drawn on the device, parameters of the stress distribution.
+        gm, gn, gk = gemm_mnk = args.gemm_shape
+        pg = torch.from_numpy(w.draw_params(gk, case.seed)).to(dev)
+        Wg = w.device_randn_bf16((gn, gk), case.seed + 7, dev)
+        qw, sw = kq.quantize_weight_tiled(Wg, pg)
+        xg = w.device_randn_bf16((gm, gk), case.seed + 11, dev)
+        qt, st_ = kq.quantize_tiled(xg, pg)
+        del Wg, xg
+        cg = torch.empty((gm, gn), dtype=torch.bfloat16, device=dev)
+        gemm_flops = 2.0 * gm * gn * gk
+    elif args.op == "gemm":
         # The layer the codes feed, as the timed step: C = Q(x T) Q(W T^-T)^T
         # with a square synthetic weight (d x d), bf16 output; both
         # quantizers write their scales in the tensor cores' tiled layout.
@@ -556,7 +569,8 @@ def run_gpu(args):
                                    16 if args.op == "kron16" else 32), op=args.op,
                            launch=("cuda_graph: the K steps captured once, replayed once"
                                    if args.launch == "graph" else "eager: one call per step"), global_batch_rows=M * world,
-                           parallelism=f"row shards x{world}", clock_ramp_s=0.3),
+                           parallelism=f"row shards x{world}", clock_ramp_s=0.3,
+                           **({"gemm_shape_mnk": gemm_mnk} if args.op == "gemm" else {})),
             "hbm_frac": value / world / peak if args.op != "gemm" else None,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": args.steps, "variants": variants,
@@ -699,6 +713,10 @@ def main(argv=None):
                              "smooth"],
                     help="quantizer timed as the step (kron = kq_quantize, the metric; "
                          "the comparators are for profiling)")
+    ap.add_argument("--gemm-shape", type=lambda v: [int(t) for t in v.split(",")], default=None,
+                    metavar="M,N,K",
+                    help="with --op gemm: time this layer shape instead of the stress "
+                         "input's square layer (profiling)")
     ap.add_argument("--rows", type=int, default=0,
                     help="rows of the stress input per GPU (default: its 16384); "
                          "smaller values are for profiling captures only")

@@ -204,7 +204,8 @@ def test_quantizers_write_the_tiled_layout(name, di, N):
 @pytest.mark.parametrize("M,N,K,dt", [(4096, 4096, 1152, torch.bfloat16),
                                       (2048, 4104, 544, torch.float32),
                                       (2100, 2048, 4096, torch.bfloat16),
-                                      (300, 520, 96, torch.float32)])
+                                      (300, 520, 96, torch.float32),
+                                      (384, 768, 12320, torch.bfloat16)])
 def test_persistent_and_per_tile_kernels_agree(M, N, K, dt, monkeypatch):
     """The persistent tiled-scale kernel (several tiles per CTA, TMA stores
     overlapping the next tile) and the one-tile-per-CTA kernel run the same

@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <cstdlib>
 
 #include "kq.h"
@@ -188,6 +189,43 @@ __device__ __forceinline__ void mma_mxf4_b16(uint32_t tmem_d, uint64_t adesc, ui
       : "memory");
 }
 
+// The kN MMAs (K = 64 each) of one k-tile: 64 codes = 32 bytes per MMA, so
+// the descriptors' start address steps by 2 (x16 B).  Scales per 32: two per
+// row and MMA, bytes 0-1 or 2-3 of the chunk's 32-bit word (scale-factor
+// id); scales per 16: four per row and MMA, chunk kk, the whole word.
+template <int kSfMode, int kN>
+__device__ __forceinline__ void ktile_mmas(uint32_t tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t tsfa, uint32_t tsfb, int kt) {
+#pragma unroll
+  for (int kk = 0; kk < kN; ++kk) {
+    if constexpr (kSfMode == kSfTiled16) {
+      mma_mxf4_b16(tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdescMxf4, tsfa + 4 * kk,
+                   tsfb + 8 * kk, (kt | kk) != 0);
+    } else {
+      const uint32_t sf_id = 2u * (kk & 1);
+      const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
+      mma_mxf4(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
+               tsfb + 8 * (kk >> 1), (kt | kk) != 0);
+    }
+  }
+}
+
+// A k-tile's MMAs; a last k-tile that ends inside the stage issues none
+// over its zero fill (K elements left: rem).
+template <int kSfMode>
+__device__ __forceinline__ void issue_ktile(uint32_t tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t tsfa, uint32_t tsfb, int kt, int rem) {
+  static_assert(kBK / kMmaK == 4, "four MMAs per k-tile");
+  if (rem > 3 * kMmaK)
+    ktile_mmas<kSfMode, 4>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+  else if (rem > 2 * kMmaK)
+    ktile_mmas<kSfMode, 3>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+  else if (rem > kMmaK)
+    ktile_mmas<kSfMode, 2>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+  else
+    ktile_mmas<kSfMode, 1>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+}
+
 template <int kSfMode>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_mxf4_kernel(const __grid_constant__ CUtensorMap amap,
@@ -332,12 +370,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int s = 0;
       uint32_t phase = 0;
-      bool ok = true;
-      for (int kt = 0; kt < nk; ++kt) {
-        if (!mbar_wait(&full[s], phase)) {
-          ok = false;
-          break;
-        }
+      // One k-tile: its stage's scales into TMEM, its MMAs (all four in a
+      // full k-tile, so that path has no branch; a last k-tile that ends
+      // inside the stage issues none over its zero fill), the stage freed.
+      auto ktile = [&](int kt, auto full_tile) -> bool {
+        if (!mbar_wait(&full[s], phase)) return false;
         tmem_fence_after();
         const uint8_t* st = base + s * Geo::kStage;
         const uint8_t* sfa = st + kATile + kBTile;
@@ -354,26 +391,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         const uint64_t adesc = smem_desc_sw128(smem_addr(st));
         const uint64_t bdesc = smem_desc_sw128(smem_addr(st + kATile));
-#pragma unroll
-        for (int kk = 0; kk < kBK / kMmaK; ++kk) {
-          // 64 codes = 32 bytes per MMA: the start address steps by 2 (x16 B).
-          if constexpr (kSfMode == kSfTiled16) {
-            // Four scales per row and MMA: chunk kk, the whole word.
-            mma_mxf4_b16(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, kIdescMxf4, tsfa + 4 * kk,
-                         tsfb + 8 * kk, (kt | kk) != 0);
-          } else {
-            const uint32_t sf_id = 2u * (kk & 1);
-            const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
-            mma_mxf4(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
-                     tsfb + 8 * (kk >> 1), (kt | kk) != 0);
-          }
-        }
+        if constexpr (decltype(full_tile)::value)
+          ktile_mmas<kSfMode, kBK / kMmaK>(tmem_base, adesc, bdesc, tsfa, tsfb, kt);
+        else
+          issue_ktile<kSfMode>(tmem_base, adesc, bdesc, tsfa, tsfb, kt, a.K - kt * kBK);
         mma_commit(&empty[s]);         // stage (codes and scales) free once read
         if (++s == kStages) {
           s = 0;
           phase ^= 1;
         }
-      }
+        return true;
+      };
+      const int nk_full = a.K % kBK == 0 ? nk : nk - 1;
+      bool ok = true;
+      int kt = 0;
+      for (; ok && kt < nk_full; ++kt) ok = ktile(kt, std::true_type{});
+      if (ok && kt < nk) ok = ktile(kt, std::false_type{});
       if (!ok) atomicOr(a.err, kErrConsumerWait);
       mma_commit(acc_full);
       // Every issued MMA completes before the columns are released.
@@ -504,17 +537,17 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t 
 
 // ---------------------------------------------------------------------------
 // Persistent variant (tiled scales): one CTA per SM walks the banded tile
-// order.  Three stages leave room for a separate 64 KiB staging buffer, so
-// the producer runs on into the next tile while the epilogue drains: the MMAs
-// of tile i + 1 wait only until the accumulator of tile i has been read out
-// of TMEM, and tile i's TMA stores overlap tile i + 1's main loop.
-constexpr int kPStages = 3;
+// order with four stages and a separate 16 KiB staging box, so the producer
+// runs on into the next tile while the epilogue drains.  With bf16 output an
+// epilogue thread holds its row's 256 outputs as 128 registers of bf16
+// pairs, so the accumulator is released as soon as it has been read and the
+// MMAs of tile i + 1 start while tile i's four boxes still leave by TMA.
+constexpr int kPStages = 4;
 constexpr int kPStageBytes = kStageBytes;
-constexpr int kStagingBytes = 4 * kOutBoxBytes;          // 64 KiB: 4 boxes
+constexpr int kStagingBytes = kOutBoxBytes;              // 16 KiB: one box
 constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kStagingBytes +
                             (2 * kPStages + 4) * 8 + 16;
 constexpr int kPThreads = 32 * 6;
-constexpr int64_t kPersistentMaxK = 8192;   // measured: K 6144 +22 %, 12288 even, 16384 -17 %
 
 __device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, int& n0) {
   const int band = t / (kBandN * a.m_tiles);
@@ -614,6 +647,38 @@ __global__ void __launch_bounds__(kPThreads, 1)
       int s = 0, i = 0;
       uint32_t phase = 0;
       bool ok = true;
+      // One k-tile: its stage's scales into TMEM, its MMAs (all four in a
+      // full k-tile, so that path has no branch; a last k-tile that ends
+      // inside the stage issues none over its zero fill), the stage freed.
+      auto ktile = [&](int kt, auto full_tile) -> bool {
+        if (!mbar_wait(&full[s], phase)) return false;
+        tmem_fence_after();
+        const uint8_t* stg = base + s * kPStageBytes;
+        const uint8_t* sfa = stg + kATile + kBTile;
+        const uint8_t* sfb = sfa + kSfaBytes;
+        const uint32_t tsfa = tmem_base + kSfCol0 + s * (kSfColsA + kSfColsB);
+        const uint32_t tsfb = tsfa + kSfColsA;
+#pragma unroll
+        for (int c = 0; c < kChunksPerStage; ++c) {
+          tmem_cp_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
+#pragma unroll
+          for (int gb = 0; gb < kBN / 128; ++gb)
+            tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * gb,
+                               smem_desc_rows16(smem_addr(sfb + (2 * gb + c) * kSfChunk)));
+        }
+        const uint64_t adesc = smem_desc_sw128(smem_addr(stg));
+        const uint64_t bdesc = smem_desc_sw128(smem_addr(stg + kATile));
+        if constexpr (decltype(full_tile)::value)
+          ktile_mmas<kSfTiled, kBK / kMmaK>(tmem_base, adesc, bdesc, tsfa, tsfb, kt);
+        else
+          issue_ktile<kSfTiled>(tmem_base, adesc, bdesc, tsfa, tsfb, kt, a.K - kt * kBK);
+        mma_commit(&empty[s]);
+        if (++s == kPStages) {
+          s = 0;
+          phase ^= 1;
+        }
+        return true;
+      };
       for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x, ++i) {
         // The accumulator is free once the epilogue has read tile i - 1.
         if (i >= 1 && !mbar_wait(acc_empty, (i - 1) & 1)) {
@@ -621,40 +686,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
           break;
         }
         tmem_fence_after();
-        for (int kt = 0; kt < nk; ++kt) {
-          if (!mbar_wait(&full[s], phase)) {
-            ok = false;
-            break;
-          }
-          tmem_fence_after();
-          const uint8_t* stg = base + s * kPStageBytes;
-          const uint8_t* sfa = stg + kATile + kBTile;
-          const uint8_t* sfb = sfa + kSfaBytes;
-          const uint32_t tsfa = tmem_base + kSfCol0 + s * (kSfColsA + kSfColsB);
-          const uint32_t tsfb = tsfa + kSfColsA;
-#pragma unroll
-          for (int c = 0; c < kChunksPerStage; ++c) {
-            tmem_cp_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
-#pragma unroll
-            for (int gb = 0; gb < kBN / 128; ++gb)
-              tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * gb,
-                                 smem_desc_rows16(smem_addr(sfb + (2 * gb + c) * kSfChunk)));
-          }
-          const uint64_t adesc = smem_desc_sw128(smem_addr(stg));
-          const uint64_t bdesc = smem_desc_sw128(smem_addr(stg + kATile));
-#pragma unroll
-          for (int kk = 0; kk < kBK / kMmaK; ++kk) {
-            const uint32_t sf_id = 2u * (kk & 1);
-            const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
-            mma_mxf4(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
-                     tsfb + 8 * (kk >> 1), (kt | kk) != 0);
-          }
-          mma_commit(&empty[s]);
-          if (++s == kPStages) {
-            s = 0;
-            phase ^= 1;
-          }
-        }
+        const int nk_full = a.K % kBK == 0 ? nk : nk - 1;
+        int kt = 0;
+        for (; ok && kt < nk_full; ++kt) ok = ktile(kt, std::true_type{});
+        if (ok && kt < nk) ok = ktile(kt, std::false_type{});
         if (ok) mma_commit(acc_full);
       }
       if (!ok) atomicOr(a.err, kErrConsumerWait);
@@ -665,74 +700,80 @@ __global__ void __launch_bounds__(kPThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     // Rows of TMEM lane quarter (warp mod 4); the tile leaves through the
-    // staging buffer as 128-byte-swizzled boxes of 128 rows x 128 bytes.
+    // staging box as 128-byte-swizzled boxes of 128 rows x 128 bytes (row
+    // r's 16-byte chunk c at c ^ (r mod 8)), one box at a time.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
     const bool issuer = warp == 2 && lane == 0;
-    const int cols_per_box = a.out_bf16 ? 64 : 32;
-    const int passes = a.out_bf16 ? 1 : 2;         // float32: two halves of 4 boxes
+    uint8_t* srow = staging + r * 128;
+    auto epi_sync = [] { asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory"); };
+    // Box `col` of the tile from the staging box: wait until the previous
+    // store has read it, fill it, store it.
+    auto store_box = [&](int m0, int col, const uint32_t (&wv)[32]) {
+      if (issuer) bulk_wait_read_0();
+      epi_sync();
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(srow + 16 * (c ^ (r & 7))) =
+            make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+      fence_proxy_async_smem();
+      epi_sync();
+      if (issuer) {
+        tma_store_2d(&cmap, staging, col, m0);
+        bulk_commit();
+      }
+    };
     int i = 0;
     for (int t = blockIdx.x; t < n_tiles_total; t += gridDim.x, ++i) {
       int m0, n0;
       tile_origin(a, t, m0, n0);
-      // One AND-barrier makes a timeout the same for the four warps and,
-      // with the issuer's wait before it, frees the staging buffer (the
-      // previous tile's stores have read it).
+      // One AND-barrier makes a timeout the same for the four warps.
       const bool got = mbar_wait(acc_full, i & 1);
-      if (issuer) bulk_wait_read_0();
       if (!bar_and(3, 4 * 32, got)) {
         if (lane == 0) atomicOr(a.err, kErrConsumerWait);
         break;
       }
       tmem_fence_after();
-      for (int pass = 0; pass < passes; ++pass) {
-        if (pass > 0) {
-          if (issuer) bulk_wait_read_0();
-          asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory");
-        }
-        const int v0 = pass * (kBN / 32 / passes), v1 = v0 + kBN / 32 / passes;
-#pragma unroll 1
-        for (int v = v0; v < v1; ++v) {
+      if (a.out_bf16) {
+        uint32_t h[kBN / 2];                      // the row as bf16 pairs
+#pragma unroll
+        for (int v = 0; v < kBN / 32; ++v) {
           uint32_t x[32];
           tmem_ld32(taddr + 32 * v, x);
           tmem_wait_ld();
-          const int col = 32 * v - (a.out_bf16 ? 0 : pass * 128);
-          uint8_t* box = staging + (col / cols_per_box) * kOutBoxBytes + r * 128;
-          if (a.out_bf16) {
-            const int c0 = (col % 64) / 8;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t wv[4];
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const __nv_bfloat162 p = __floats2bfloat162_rn(
-                    __uint_as_float(x[8 * q + 2 * h]), __uint_as_float(x[8 * q + 2 * h + 1]));
-                wv[h] = *reinterpret_cast<const uint32_t*>(&p);
-              }
-              *reinterpret_cast<uint4*>(box + 16 * ((c0 + q) ^ (r & 7))) =
-                  make_uint4(wv[0], wv[1], wv[2], wv[3]);
-            }
-          } else {
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-              *reinterpret_cast<uint4*>(box + 16 * (q ^ (r & 7))) =
-                  make_uint4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+          for (int q = 0; q < 16; ++q) {
+            const __nv_bfloat162 p =
+                __floats2bfloat162_rn(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1]));
+            h[16 * v + q] = *reinterpret_cast<const uint32_t*>(&p);
           }
         }
-        if (pass == passes - 1) {
-          // Every column has been read: the MMAs of the next tile may start.
-          tmem_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(acc_empty);
+        // Every column has been read: the MMAs of the next tile may start.
+        tmem_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          uint32_t wv[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) wv[k] = h[32 * b + k];
+          store_box(m0, n0 + 64 * b, wv);
         }
-        fence_proxy_async_smem();
-        asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory");
-        if (issuer) {
-          for (int b = 0; b < 4; ++b)
-            tma_store_2d(&cmap, staging + b * kOutBoxBytes,
-                         n0 + (pass * 4 + b) * cols_per_box, m0);
-          bulk_commit();
+      } else {
+        // float32: eight boxes of 32 columns, each read out of TMEM as it
+        // goes; the accumulator is released after the last read.
+#pragma unroll 1
+        for (int b = 0; b < kBN / 32; ++b) {
+          uint32_t x[32];
+          tmem_ld32(taddr + 32 * b, x);
+          tmem_wait_ld();
+          if (b == kBN / 32 - 1) {
+            tmem_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty);
+          }
+          store_box(m0, n0 + 32 * b, x);
         }
       }
     }
@@ -754,12 +795,12 @@ using namespace kq;
 namespace kq {
 namespace {
 
-// The persistent kernel for short K, where a tile's own prologue and
-// epilogue weigh most; KQ_GEMM_PERSISTENT=0/1 forces either (measurements).
-bool persistent_gemm(int64_t K) {
+// The persistent kernel for the tiled layout with TMA stores (measured
+// ahead of the one-tile-per-CTA kernel at every K from 1152 to 16384);
+// KQ_GEMM_PERSISTENT=0/1 forces either (measurements, tests).
+bool persistent_gemm() {
   const char* e = getenv("KQ_GEMM_PERSISTENT");
-  if (e) return atoi(e) != 0;
-  return K <= kPersistentMaxK;
+  return e ? atoi(e) != 0 : true;
 }
 
 int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
@@ -822,7 +863,7 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled16>>(G::kSmem, dev);
     if (rc != KQ_OK) return rc;
     gemm_mxf4_kernel<kSfTiled16><<<grid, 32 * kSfWarp0, G::kSmem, st>>>(amap, bmap, cmap, a);
-  } else if (tiled && a.tma_store && persistent_gemm(K)) {
+  } else if (tiled && a.tma_store && persistent_gemm()) {
     rc = allow_smem<gemm_mxf4_persistent>(kPSmemBytes, dev);
     if (rc != KQ_OK) return rc;
     const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
