@@ -209,3 +209,31 @@ def test_block16_product_random_operands_and_exact_sums():
             assert np.array_equal(C.astype(np.float64), ref)   # small exact sums
         mag = o.abs_mxfp4_gemm(ca, sa, cb, sb, block=16)
         assert (np.abs(C - ref) <= (K / 64 + 1) * 2.0 ** -22 * mag).all(), (M, N, K)
+
+
+@pytest.mark.parametrize("M,N,K,dt", [(2048, 4096, 1152, torch.bfloat16),
+                                      (300, 520, 96, torch.float32),
+                                      (384, 768, 4128, torch.bfloat16)])
+def test_block16_persistent_and_per_tile_kernels_agree(M, N, K, dt, monkeypatch):
+    """The persistent kernel with scales per 16 (several tiles per CTA, three
+    stages) and the one-tile-per-CTA kernel run the same MMAs: identical
+    outputs, within the tolerance of the exact product on sampled rows."""
+    rng = np.random.default_rng(M + N + K)
+    ca = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    cb = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = rng.integers(120, 135, (M, K // 16), dtype=np.uint8)
+    sb = rng.integers(120, 135, (N, K // 16), dtype=np.uint8)
+    args = (_dev(ca), _dev(o.scales_to_mma(sa)), _dev(cb), _dev(o.scales_to_mma(sb)))
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("KQ_GEMM16_PERSISTENT", flag)
+        outs.append(kq.gemm_mxfp4_16_tiled(*args, out_dtype=dt))
+    torch.cuda.synchronize()
+    assert torch.equal(outs[0], outs[1])
+    rows = np.array([0, 1, 127, 128, M // 2, M - 1])
+    ref = o.mxfp4_gemm(ca[rows], sa[rows], cb, sb, block=16)
+    mag = o.abs_mxfp4_gemm(ca[rows], sa[rows], cb, sb, block=16)
+    got = outs[0].float().cpu().numpy()[rows].astype(np.float64)
+    tol = (K / 64 + 1) * 2.0 ** -22 * mag + (np.abs(ref) * 2.0 ** -8 if dt == torch.bfloat16 else 0)
+    assert (np.abs(got - ref) <= tol).all()
+    assert kq.device_status() == 0

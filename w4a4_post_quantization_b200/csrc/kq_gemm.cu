@@ -542,12 +542,21 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t 
 // epilogue thread holds its row's 256 outputs as 128 registers of bf16
 // pairs, so the accumulator is released as soon as it has been read and the
 // MMAs of tile i + 1 start while tile i's four boxes still leave by TMA.
-constexpr int kPStages = 4;
-constexpr int kPStageBytes = kStageBytes;
 constexpr int kStagingBytes = kOutBoxBytes;              // 16 KiB: one box
-constexpr int kPSmemBytes = 1024 + kPStages * kPStageBytes + kStagingBytes +
-                            (2 * kPStages + 4) * 8 + 16;
 constexpr int kPThreads = 32 * 6;
+
+// Stages of the persistent kernel per scale mode: four of 51 KiB with scales
+// per 32, three of 54 KiB with scales per 16 (four do not fit beside the
+// staging box).
+template <int kSfMode>
+struct PGeom : StageGeom<kSfMode> {
+  static constexpr int kStages = kSfMode == kSfTiled16 ? 3 : 4;
+  static constexpr int kSmem = 1024 + kStages * StageGeom<kSfMode>::kStage + kStagingBytes +
+                               (2 * kStages + 4) * 8 + 16;
+  static_assert(kSmem <= 232448, "shared memory");
+  static_assert(kSfCol0 + kStages * (StageGeom<kSfMode>::kColsA + StageGeom<kSfMode>::kColsB) <=
+                    kTmemCols, "TMEM columns");
+};
 
 __device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, int& n0) {
   const int band = t / (kBandN * a.m_tiles);
@@ -557,16 +566,18 @@ __device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, i
   n0 = (band * kBandN + r % width) * kBN;
 }
 
+template <int kSfMode>
 __global__ void __launch_bounds__(kPThreads, 1)
     gemm_mxf4_persistent(const __grid_constant__ CUtensorMap amap,
                          const __grid_constant__ CUtensorMap bmap,
                          const __grid_constant__ CUtensorMap cmap, const GemmArgs a) {
+  using P = PGeom<kSfMode>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
-  uint8_t* staging = base + kPStages * kPStageBytes;
+  uint8_t* staging = base + P::kStages * P::kStage;
   uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
-  uint64_t* empty = full + kPStages;
-  uint64_t* acc_full = empty + kPStages;
+  uint64_t* empty = full + P::kStages;
+  uint64_t* acc_full = empty + P::kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_done = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -574,13 +585,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int n_tiles_total = a.m_tiles * a.n_tiles;
   const int nk = a.k_tiles;
 
-  for (int st = 0; st < kPStages; ++st)
-    for (int i = tid; i < (kSfaBytes + kSfbBytes) / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(base + st * kPStageBytes + kATile + kBTile)[i] =
+  for (int st = 0; st < P::kStages; ++st)
+    for (int i = tid; i < (P::kSfa + P::kSfb) / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(base + st * P::kStage + kATile + kBTile)[i] =
           make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (tid == 0) {
-    for (int st = 0; st < kPStages; ++st) {
+    for (int st = 0; st < P::kStages; ++st) {
       mbar_init(&full[st], 1);
       mbar_init(&empty[st], 1);
     }
@@ -608,34 +619,34 @@ __global__ void __launch_bounds__(kPThreads, 1)
         tile_origin(a, t, m0, n0);
         const int b_tiles = min(kBN / 128, a.sf_tiles_n - n0 / 128);
         for (int kt = 0; kt < nk; ++kt, ++g) {
-          if (g >= kPStages && !mbar_wait(&empty[s], phase)) {
+          if (g >= P::kStages && !mbar_wait(&empty[s], phase)) {
             ok = false;
             break;
           }
-          uint8_t* stg = base + s * kPStageBytes;
-          const int avail = min(kChunksPerStage, a.sf_tiles_k - kChunksPerStage * kt);
+          uint8_t* stg = base + s * P::kStage;
+          const int avail = min(P::kChunks, a.sf_tiles_k - P::kChunks * kt);
           mbar_arrive_expect_tx(&full[s], kATile + kBTile +
                                               (uint32_t)(avail * (1 + b_tiles)) * kSfChunk);
           uint8_t* sfa = stg + kATile + kBTile;
-          bulk_load(sfa, a.sa + ((int64_t)(m0 / 128) * a.sf_tiles_k + kChunksPerStage * kt) *
+          bulk_load(sfa, a.sa + ((int64_t)(m0 / 128) * a.sf_tiles_k + P::kChunks * kt) *
                                   kSfChunk, avail * kSfChunk, &full[s]);
           for (int gb = 0; gb < b_tiles; ++gb)
-            bulk_load(sfa + kSfaBytes + gb * kChunksPerStage * kSfChunk,
-                      a.sb + ((int64_t)(n0 / 128 + gb) * a.sf_tiles_k + kChunksPerStage * kt) *
+            bulk_load(sfa + P::kSfa + gb * P::kChunks * kSfChunk,
+                      a.sb + ((int64_t)(n0 / 128 + gb) * a.sf_tiles_k + P::kChunks * kt) *
                                  kSfChunk, avail * kSfChunk, &full[s]);
           tma_load_2d(stg, &amap, kt * kBKBytes, m0, &full[s]);
           tma_load_2d(stg + kATile, &bmap, kt * kBKBytes, n0, &full[s]);
           issued = g + 1;
-          if (++s == kPStages) {
+          if (++s == P::kStages) {
             s = 0;
-            if (g >= kPStages) phase ^= 1;
+            if (g >= P::kStages) phase ^= 1;
           }
         }
       }
       if (!ok) {
         atomicOr(a.err, kErrProducerWait);
-        for (int i = issued > kPStages ? issued - kPStages : 0; i < issued; ++i)
-          mbar_wait(&full[i % kPStages], (i / kPStages) & 1);
+        for (int i = issued > P::kStages ? issued - P::kStages : 0; i < issued; ++i)
+          mbar_wait(&full[i % P::kStages], (i / P::kStages) & 1);
       }
     }
     return;
@@ -653,27 +664,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
       auto ktile = [&](int kt, auto full_tile) -> bool {
         if (!mbar_wait(&full[s], phase)) return false;
         tmem_fence_after();
-        const uint8_t* stg = base + s * kPStageBytes;
+        const uint8_t* stg = base + s * P::kStage;
         const uint8_t* sfa = stg + kATile + kBTile;
-        const uint8_t* sfb = sfa + kSfaBytes;
-        const uint32_t tsfa = tmem_base + kSfCol0 + s * (kSfColsA + kSfColsB);
-        const uint32_t tsfb = tsfa + kSfColsA;
+        const uint8_t* sfb = sfa + P::kSfa;
+        const uint32_t tsfa = tmem_base + kSfCol0 + s * (P::kColsA + P::kColsB);
+        const uint32_t tsfb = tsfa + P::kColsA;
 #pragma unroll
-        for (int c = 0; c < kChunksPerStage; ++c) {
+        for (int c = 0; c < P::kChunks; ++c) {
           tmem_cp_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
 #pragma unroll
           for (int gb = 0; gb < kBN / 128; ++gb)
             tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * gb,
-                               smem_desc_rows16(smem_addr(sfb + (2 * gb + c) * kSfChunk)));
+                               smem_desc_rows16(smem_addr(sfb + (P::kChunks * gb + c) * kSfChunk)));
         }
         const uint64_t adesc = smem_desc_sw128(smem_addr(stg));
         const uint64_t bdesc = smem_desc_sw128(smem_addr(stg + kATile));
         if constexpr (decltype(full_tile)::value)
-          ktile_mmas<kSfTiled, kBK / kMmaK>(tmem_base, adesc, bdesc, tsfa, tsfb, kt);
+          ktile_mmas<kSfMode, kBK / kMmaK>(tmem_base, adesc, bdesc, tsfa, tsfb, kt);
         else
-          issue_ktile<kSfTiled>(tmem_base, adesc, bdesc, tsfa, tsfb, kt, a.K - kt * kBK);
+          issue_ktile<kSfMode>(tmem_base, adesc, bdesc, tsfa, tsfb, kt, a.K - kt * kBK);
         mma_commit(&empty[s]);
-        if (++s == kPStages) {
+        if (++s == P::kStages) {
           s = 0;
           phase ^= 1;
         }
@@ -803,6 +814,13 @@ bool persistent_gemm() {
   return e ? atoi(e) != 0 : true;
 }
 
+// The same choice for scales per 16 (three persistent stages against the
+// one-tile-per-CTA kernel's four); KQ_GEMM16_PERSISTENT=0/1 forces either.
+bool persistent_gemm16() {
+  const char* e = getenv("KQ_GEMM16_PERSISTENT");
+  return e ? atoi(e) != 0 : true;
+}
+
 int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
                 int64_t M, int64_t N, int64_t K, void* c, int c_dtype, void* stream,
                 bool tiled, int scale_block = 32) {
@@ -858,16 +876,23 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   }
   const dim3 grid(static_cast<unsigned>(a.m_tiles * a.n_tiles));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (scale_block == 16) {
+  if (scale_block == 16 && a.tma_store && persistent_gemm16()) {
+    rc = allow_smem<gemm_mxf4_persistent<kSfTiled16>>(PGeom<kSfTiled16>::kSmem, dev);
+    if (rc != KQ_OK) return rc;
+    const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
+    gemm_mxf4_persistent<kSfTiled16>
+        <<<pgrid, kPThreads, PGeom<kSfTiled16>::kSmem, st>>>(amap, bmap, cmap, a);
+  } else if (scale_block == 16) {
     using G = StageGeom<kSfTiled16>;
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled16>>(G::kSmem, dev);
     if (rc != KQ_OK) return rc;
     gemm_mxf4_kernel<kSfTiled16><<<grid, 32 * kSfWarp0, G::kSmem, st>>>(amap, bmap, cmap, a);
   } else if (tiled && a.tma_store && persistent_gemm()) {
-    rc = allow_smem<gemm_mxf4_persistent>(kPSmemBytes, dev);
+    rc = allow_smem<gemm_mxf4_persistent<kSfTiled>>(PGeom<kSfTiled>::kSmem, dev);
     if (rc != KQ_OK) return rc;
     const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
-    gemm_mxf4_persistent<<<pgrid, kPThreads, kPSmemBytes, st>>>(amap, bmap, cmap, a);
+    gemm_mxf4_persistent<kSfTiled>
+        <<<pgrid, kPThreads, PGeom<kSfTiled>::kSmem, st>>>(amap, bmap, cmap, a);
   } else if (tiled) {
     // No scale warps: six warps.
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled>>(kSmemBytes, dev);
