@@ -214,10 +214,23 @@ def _cpu_workers() -> int:
     return max(1, min(32, n))
 
 
+def _worker_ready(pause: float):
+    """Imports the oracle in a spawned worker, then holds it briefly so that
+    every worker of the pool takes one of these tasks."""
+    from oracle import kq_oracle  # noqa: F401
+    time.sleep(pause)
+    return os.getpid()
+
+
 def oracle_pool(workers: int):
+    """A spawned pool whose workers have all started and imported the
+    oracle before it is returned, so that their start-up does not compete
+    with the timed GPU launches for the host cores."""
     for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
         os.environ[var] = "1"
-    return mp.get_context("spawn").Pool(workers)
+    pool = mp.get_context("spawn").Pool(workers)
+    pool.map(_worker_ready, [0.2] * workers, chunksize=1)
+    return pool
 
 
 def time_oracle(pool, case, rows: int, chunk: int = 128):
