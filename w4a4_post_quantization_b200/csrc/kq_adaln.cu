@@ -48,8 +48,10 @@ namespace {
 constexpr int kAdaWarps = 12;                     // 3 warps per scheduler: 168 registers
 constexpr int kAdaCons = 32 * kAdaWarps;          // threads, all consumers
 constexpr int kAdaMaxStages = 8;
-constexpr int kAdaMaxRows = 256;                  // TMA box limit on R
-constexpr int kAdaSlots = kAdaWarps + kAdaMaxRows;   // segment slots per buffer
+constexpr int kAdaHalves = 2;                     // rows of a group a thread takes
+constexpr int kAdaMaxRows = 256;                  // TMA box limit on a group's rows
+constexpr int kAdaMaxHalfRows = kAdaMaxRows / kAdaHalves;
+constexpr int kAdaSlots = kAdaWarps + kAdaMaxHalfRows;   // segment slots per half
 constexpr int kAdaSlotBufs = 4;
 
 struct AdaArgs {
@@ -93,16 +95,20 @@ __device__ __forceinline__ void block_sums(const f2 (&u)[16], float& sum, float&
   m2 = (a0 + a1) + (b0 + b1);
 }
 
-// Sum of v over this lane's segment (the lanes of the warp in the same row),
-// left in the segment's first lane: shuffle-down steps that stay inside the
-// segment (bit k of `inside` says whether lane + 2^k is in it).
-__device__ __forceinline__ float segment_sum(float v, uint32_t inside) {
+// Sums of two values over this lane's segment (the lanes of the warp in
+// the same row), left in the segment's first lane: shuffle-down steps that
+// stay inside the segment (bit k of `inside` says whether lane + 2^k is in
+// it), the two values side by side.
+__device__ __forceinline__ void segment_sum2(float& v0, float& v1, uint32_t inside) {
 #pragma unroll
   for (int k = 0; k < 5; ++k) {
-    const float o = __shfl_down_sync(0xFFFFFFFFu, v, 1 << k);
-    if (inside & (1u << k)) v += o;
+    const float o0 = __shfl_down_sync(0xFFFFFFFFu, v0, 1 << k);
+    const float o1 = __shfl_down_sync(0xFFFFFFFFu, v1, 1 << k);
+    if (inside & (1u << k)) {
+      v0 += o0;
+      v1 += o1;
+    }
   }
-  return v;
 }
 
 // The shear form with its diagonal first: per factor
@@ -114,7 +120,6 @@ __device__ __forceinline__ float segment_sum(float v, uint32_t inside) {
 struct ShearIn {
   f2 r10[4], r01[4];     // stages on index bits 4..1, both halves equal
   float r10b, r01b;      // stage on bit 0
-  float g00[kFactors], g11[kFactors];
 };
 
 // Fills the form for the block with parameters p[15]; false if the block
@@ -133,8 +138,6 @@ __device__ __forceinline__ bool load_shear_in(ShearIn& f, const float* p) {
     growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
     r10[k] = (float)ra;
     r01[k] = (float)rb;
-    f.g00[k] = (float)g00;
-    f.g11[k] = (float)g11;
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -159,19 +162,22 @@ __device__ __forceinline__ void shear_in_apply(f2 (&u)[16], const ShearIn& f) {
   }
 }
 
-// Entries 2m and 2m + 1 of the diagonal (x) diag(g00_k, g11_k), factor k on
-// index bit 4 - k, as products in float32 (at most four roundings).
-__device__ __forceinline__ void diag_pairs(const ShearIn& f, f2 (&dl)[16]) {
-  float hi2[4], lo2[4];
+// Entries 2m and 2m + 1 of the diagonal (x) diag(g00_k, g11_k) of the block
+// with parameters p[15], factor k on index bit 4 - k, formed in double and
+// rounded once.
+__device__ __forceinline__ void diag_pairs(const float* p, f2 (&dl)[16]) {
+  double g00[kFactors], g11[kFactors];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    hi2[q] = ((q & 2) ? f.g11[0] : f.g00[0]) * ((q & 1) ? f.g11[1] : f.g00[1]);
-    lo2[q] = ((q & 2) ? f.g11[2] : f.g00[2]) * ((q & 1) ? f.g11[3] : f.g00[3]);
+  for (int k = 0; k < kFactors; ++k) {
+    double e01, e10;
+    factor_entries<false>(p, k, g00[k], e01, e10, g11[k]);
   }
 #pragma unroll
   for (int m = 0; m < 16; ++m) {
-    const float t = hi2[m >> 2] * lo2[m & 3];
-    dl[m] = pack2(t * f.g00[4], t * f.g11[4]);
+    double t = 1.0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) t *= ((2 * m) >> (4 - k)) & 1 ? g11[k] : g00[k];
+    dl[m] = pack2((float)(t * g00[4]), (float)(t * g11[4]));
   }
 }
 
@@ -182,10 +188,10 @@ __device__ __forceinline__ void diag_pairs(const ShearIn& f, f2 (&dl)[16]) {
 // are consecutive.  delta = 1 for the plain form.
 template <int kForm>
 __device__ __forceinline__ void load_modulation(const AdaArgs& a, int64_t b, int j, int tid,
-                                                const ShearIn& si, float4* tab) {
+                                                float4* tab) {
   f2 dl[16];
   if (kForm == 0) {
-    diag_pairs(si, dl);
+    diag_pairs(a.params + (int64_t)j * 15, dl);
   } else {
 #pragma unroll
     for (int m = 0; m < 16; ++m) dl[m] = pack2(1.0f, 1.0f);
@@ -219,7 +225,7 @@ __device__ __forceinline__ void adaln_issue(const AdaArgs& a, const CUtensorMap*
                                             uint8_t* stage, uint64_t* bar, int g) {
   mbar_arrive_expect_tx(bar, a.tx_bytes);
   for (int b = 0; b < a.boxes; ++b)
-    tma_load_3d(stage + b * a.box_bytes, xmap, 0, b * a.Wb, g * a.R, bar);
+    tma_load_3d(stage + b * a.box_bytes, xmap, 0, b * a.Wb, g * kAdaHalves * a.R, bar);
 }
 
 // The loop of one thread over its CTA's groups, software-pipelined by one
@@ -227,7 +233,10 @@ __device__ __forceinline__ void adaln_issue(const AdaArgs& a, const CUtensorMap*
 // statistics mbarrier) are produced before group i is normalized, so no
 // warp waits for the whole CTA inside a group.  Slots rotate through four
 // buffers, enough that a warp writing group i + 3's slots can only have got
-// there after every warp finished reading group i - 1's.
+// there after every warp finished reading group i - 1's.  A group is 2 R
+// rows and a thread takes block j of rows rr and R + rr, so the two rows'
+// reductions run side by side and a group's latency is paid once per 64
+// elements of each thread.
 template <int kOut, int kForm>
 __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMap* xmap,
                                               uint8_t* stages, uint64_t* full, uint64_t* statbar,
@@ -238,14 +247,16 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
   const bool active = tid < R * nb;
   const int rr = active ? tid / nb : R;         // inactive threads form their own "row"
   const int j = tid - rr * nb;
-  // Byte offsets of this thread's four 16-byte chunks inside a stage: box
-  // j / Wb, line rr Wb + j mod Wb, chunk q at q ^ ((line >> 1) & 3).
-  uint32_t off[4];
-  {
-    const int line = rr * a.Wb + (j % a.Wb);
+  // Byte offsets of this thread's four 16-byte chunks of row h R + rr inside
+  // a stage: box j / Wb, line (h R + rr) Wb + j mod Wb, chunk q at
+  // q ^ ((line >> 1) & 3).
+  uint32_t off[kAdaHalves][4];
+#pragma unroll
+  for (int h = 0; h < kAdaHalves; ++h) {
+    const int line = (h * R + rr) * a.Wb + (j % a.Wb);
     const uint32_t boff = (j / a.Wb) * a.box_bytes;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) off[q] = boff + line * 64 + 16 * (q ^ ((line >> 1) & 3));
+    for (int q = 0; q < 4; ++q) off[h][q] = boff + line * 64 + 16 * (q ^ ((line >> 1) & 3));
   }
   // Segments: the lanes of a warp that share a row.  Slot of (row, warp) is
   // warp + row, unique and increasing along the rows.
@@ -278,40 +289,55 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
 
   // Group k's data from its stage: waits for the TMA, reads, and orders the
   // reads before the stage's refill.
-  auto read_group = [&](int k, uint4 (&c)[4]) -> bool {
+  auto read_group = [&](int k, uint4 (&c)[kAdaHalves][4]) -> bool {
     const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(&full[k % S], (k / S) & 1));
     const uint8_t* st = stages + (k % S) * a.stage_bytes;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      c[q] = active ? *reinterpret_cast<const uint4*>(st + off[q]) : make_uint4(0, 0, 0, 0);
+    for (int h = 0; h < kAdaHalves; ++h)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        c[h][q] = active ? *reinterpret_cast<const uint4*>(st + off[h][q]) : make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     return got;
   };
   // Group k's slots: segment sums of the block sums give the segment mean,
   // then the block M2 plus 32 (block mean - segment mean)^2 summed over the
   // segment is the segment's M2.  Rows past M hold zeros (TMA fill).
-  auto post_stats = [&](int k, const uint4 (&c)[4]) {
-    f2 u[16];
+  auto post_stats = [&](int k, const uint4 (&c)[kAdaHalves][4]) {
+    float bsum[kAdaHalves], bm2[kAdaHalves];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      u[4 * q + 0] = bf16x2_to_f2(c[q].x);
-      u[4 * q + 1] = bf16x2_to_f2(c[q].y);
-      u[4 * q + 2] = bf16x2_to_f2(c[q].z);
-      u[4 * q + 3] = bf16x2_to_f2(c[q].w);
+    for (int h = 0; h < kAdaHalves; ++h) {
+      f2 u[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        u[4 * q + 0] = bf16x2_to_f2(c[h][q].x);
+        u[4 * q + 1] = bf16x2_to_f2(c[h][q].y);
+        u[4 * q + 2] = bf16x2_to_f2(c[h][q].z);
+        u[4 * q + 3] = bf16x2_to_f2(c[h][q].w);
+      }
+      bsum[h] = 0.f;
+      bm2[h] = 0.f;
+      if (active) block_sums(u, bsum[h], bm2[h]);
     }
-    float bsum = 0.f, bm2 = 0.f;
-    if (active) block_sums(u, bsum, bm2);
-    const float seg_sum = __shfl_sync(0xFFFFFFFFu, segment_sum(bsum, inside), head_lane);
-    const float seg_mean = seg_sum * inv_seg_n;
-    const float dm = __fmaf_rn(bsum, 1.0f / 32.0f, -seg_mean);
-    const float seg_m2 = segment_sum(__fmaf_rn(32.0f * dm, dm, bm2), inside);
-    if (head) slots[(k & 3) * kAdaSlots + warp + rr] = make_float4(seg_mean, seg_m2, seg_n, 0.f);
+    float s0 = bsum[0], s1 = bsum[1];
+    segment_sum2(s0, s1, inside);
+    const float m0 = __shfl_sync(0xFFFFFFFFu, s0, head_lane) * inv_seg_n;
+    const float m1 = __shfl_sync(0xFFFFFFFFu, s1, head_lane) * inv_seg_n;
+    const float d0 = __fmaf_rn(bsum[0], 1.0f / 32.0f, -m0);
+    const float d1 = __fmaf_rn(bsum[1], 1.0f / 32.0f, -m1);
+    float q0 = __fmaf_rn(32.0f * d0, d0, bm2[0]), q1 = __fmaf_rn(32.0f * d1, d1, bm2[1]);
+    segment_sum2(q0, q1, inside);
+    if (head) {
+      float4* sb = slots + (k & 3) * (kAdaHalves * kAdaSlots) + warp + rr;
+      sb[0] = make_float4(m0, q0, seg_n, 0.f);
+      sb[kAdaSlots] = make_float4(m1, q1, seg_n, 0.f);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&statbar[k & 1]);
   };
 
   int64_t b_end = 0;                              // first row past this thread's sample
-  uint4 cn[4];
+  uint4 cn[kAdaHalves][4];
   bool ok = n_local > 0;
   int read = 0;                                   // groups whose data arrived
   if (ok) {
@@ -320,9 +346,11 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
     post_stats(0, cn);
   }
   for (int i = 0; ok && i < n_local; ++i) {
-    uint4 cc[4];
+    uint4 cc[kAdaHalves][4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) cc[q] = cn[q];
+    for (int h = 0; h < kAdaHalves; ++h)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) cc[h][q] = cn[h][q];
     if (i + 1 < n_local) {
       ok = read_group(i + 1, cn);
       read += ok ? 1 : 0;
@@ -336,55 +364,68 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
                   (int)blockIdx.x + (i + S) * (int)gridDim.x);
       ++issued;
     }
-    // The row's segments in a fixed order: mean = sum n_k m_k / d, then
-    // M2 = sum M2_k + n_k (m_k - mean)^2.
-    const float4* sbuf = slots + (i & 3) * kAdaSlots;
-    float mean, m2;
+    // Each row's segments in a fixed order: mean = sum n_k m_k / d, then
+    // M2 = sum M2_k + n_k (m_k - mean)^2; the two halves side by side.
+    const float4* sbuf = slots + (i & 3) * (kAdaHalves * kAdaSlots);
+    float mean[kAdaHalves] = {0.f, 0.f}, m2[kAdaHalves] = {0.f, 0.f};
     if (lane_parallel) {
       // Lane k takes slot k of the warp's first (then last) row; xor sums
       // give every lane the same totals.
-      mean = 0.f;
-      m2 = 0.f;
       for (int t = 0; t < n_rows_here; ++t) {
         const int r = t == 0 ? row_lo : row_hi;
         const int base = ((r * nb) >> 5) + r, cnt = (((r + 1) * nb - 1) >> 5) - ((r * nb) >> 5) + 1;
-        const float4 v = lane < cnt ? sbuf[base + lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-        float ms = v.z * v.x;
+        const float4 z4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v0 = lane < cnt ? sbuf[base + lane] : z4;
+        const float4 v1 = lane < cnt ? sbuf[kAdaSlots + base + lane] : z4;
+        float ms0 = v0.z * v0.x, ms1 = v1.z * v1.x;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) ms += __shfl_xor_sync(0xFFFFFFFFu, ms, o);
-        const float mr = ms * inv_d;
-        const float dk = v.x - mr;
-        float q = __fmaf_rn(v.z * dk, dk, v.y);
+        for (int o = 16; o > 0; o >>= 1) {
+          ms0 += __shfl_xor_sync(0xFFFFFFFFu, ms0, o);
+          ms1 += __shfl_xor_sync(0xFFFFFFFFu, ms1, o);
+        }
+        const float mr0 = ms0 * inv_d, mr1 = ms1 * inv_d;
+        const float dk0 = v0.x - mr0, dk1 = v1.x - mr1;
+        float q0 = __fmaf_rn(v0.z * dk0, dk0, v0.y), q1 = __fmaf_rn(v1.z * dk1, dk1, v1.y);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xFFFFFFFFu, q, o);
+        for (int o = 16; o > 0; o >>= 1) {
+          q0 += __shfl_xor_sync(0xFFFFFFFFu, q0, o);
+          q1 += __shfl_xor_sync(0xFFFFFFFFu, q1, o);
+        }
         if (rr == r) {
-          mean = mr;
-          m2 = q;
+          mean[0] = mr0;
+          m2[0] = q0;
+          mean[1] = mr1;
+          m2[1] = q1;
         }
       }
     } else {
-      const float4* rs = sbuf + w_first + rr;
-      float msum = 0.f;
-      for (int k = 0; k < n_slots; ++k) msum = __fmaf_rn(rs[k].z, rs[k].x, msum);
-      mean = msum * inv_d;
-      m2 = 0.f;
-      for (int k = 0; k < n_slots; ++k) {
-        const float4 v = rs[k];
-        const float dk = v.x - mean;
-        m2 += __fmaf_rn(v.z * dk, dk, v.y);
+#pragma unroll
+      for (int h = 0; h < kAdaHalves; ++h) {
+        const float4* rs = sbuf + h * kAdaSlots + w_first + rr;
+        float msum = 0.f;
+        for (int k = 0; k < n_slots; ++k) msum = __fmaf_rn(rs[k].z, rs[k].x, msum);
+        mean[h] = msum * inv_d;
+        for (int k = 0; k < n_slots; ++k) {
+          const float4 v = rs[k];
+          const float dk = v.x - mean[h];
+          m2[h] += __fmaf_rn(v.z * dk, dk, v.y);
+        }
       }
     }
-    const int64_t row = ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * R + rr;
+#pragma unroll
+    for (int h = 0; h < kAdaHalves; ++h) {
+    const int64_t row =
+        ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * (kAdaHalves * R) + h * R + rr;
     if (!active || row >= a.M) continue;
     if (row >= b_end) {                           // rows only grow: a new sample
       const int64_t b = row / a.tokens;
       b_end = (b + 1) * a.tokens;
-      load_modulation<kForm>(a, b, j, tid, si, modtab);
+      load_modulation<kForm>(a, b, j, tid, modtab);
     }
     // rsqrtf: within 2 ulp, far inside the 1e-5 band of the modulated value.
-    const float rstd = rsqrtf(__fmaf_rn(m2, inv_d, a.eps));
+    const float rstd = rsqrtf(__fmaf_rn(m2[h], inv_d, a.eps));
     // h D = t alpha + beta with t = x rstd - mean rstd.
-    const f2 r2 = pack2(rstd, rstd), nmr2 = pack2(-mean * rstd, -mean * rstd);
+    const f2 r2 = pack2(rstd, rstd), nmr2 = pack2(-mean[h] * rstd, -mean[h] * rstd);
     f2 u[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -392,13 +433,13 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
       const float4 al1 = modtab[(2 * q + 1) * kAdaCons + tid];
       const float4 be0 = modtab[(8 + 2 * q) * kAdaCons + tid];
       const float4 be1 = modtab[(8 + 2 * q + 1) * kAdaCons + tid];
-      u[4 * q + 0] = fma2(fma2(bf16x2_to_f2(cc[q].x), r2, nmr2), pack2(al0.x, al0.y),
+      u[4 * q + 0] = fma2(fma2(bf16x2_to_f2(cc[h][q].x), r2, nmr2), pack2(al0.x, al0.y),
                           pack2(be0.x, be0.y));
-      u[4 * q + 1] = fma2(fma2(bf16x2_to_f2(cc[q].y), r2, nmr2), pack2(al0.z, al0.w),
+      u[4 * q + 1] = fma2(fma2(bf16x2_to_f2(cc[h][q].y), r2, nmr2), pack2(al0.z, al0.w),
                           pack2(be0.z, be0.w));
-      u[4 * q + 2] = fma2(fma2(bf16x2_to_f2(cc[q].z), r2, nmr2), pack2(al1.x, al1.y),
+      u[4 * q + 2] = fma2(fma2(bf16x2_to_f2(cc[h][q].z), r2, nmr2), pack2(al1.x, al1.y),
                           pack2(be1.x, be1.y));
-      u[4 * q + 3] = fma2(fma2(bf16x2_to_f2(cc[q].w), r2, nmr2), pack2(al1.z, al1.w),
+      u[4 * q + 3] = fma2(fma2(bf16x2_to_f2(cc[h][q].w), r2, nmr2), pack2(al1.z, al1.w),
                           pack2(be1.z, be1.w));
     }
     if (kForm == 1) {
@@ -433,6 +474,7 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
         __stcs(dst + t, make_float4(x0, x1, x2, x3));
       }
     }
+    }
   }
   if (!ok) {
     if (lane == 0) atomicOr(a.err, kErrConsumerWait);
@@ -451,7 +493,7 @@ __global__ void __launch_bounds__(kAdaCons, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(base + a.stages * a.stage_bytes);
   uint64_t* statbar = full + kAdaMaxStages;
   float4* slots = reinterpret_cast<float4*>(statbar + 2);            // 16-byte aligned
-  float4* modtab = slots + kAdaSlotBufs * kAdaSlots;               // [16][kAdaCons]
+  float4* modtab = slots + kAdaSlotBufs * kAdaHalves * kAdaSlots;  // [16][kAdaCons]
   const int tid = threadIdx.x;
   const int S = a.stages;
   if (tid == 0) {
@@ -503,17 +545,19 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   a.M = M;
   a.tokens = tokens;
   a.nb = nb;
-  a.R = std::min(kAdaCons / nb, kAdaMaxRows);
+  a.R = std::min(kAdaCons / nb, kAdaMaxHalfRows);   // rows per half of a group
   // Boxes of at most 256 blocks; the last may run past the row and is
   // zero-filled there.
   a.boxes = (nb + 255) / 256;
   a.Wb = (nb + a.boxes - 1) / a.boxes;
-  const int box_raw = a.R * a.Wb * kBlock * 2;
+  const int box_raw = kAdaHalves * a.R * a.Wb * kBlock * 2;
   a.box_bytes = (box_raw + 1023) / 1024 * 1024;
   a.stage_bytes = a.boxes * a.box_bytes;
   a.tx_bytes = a.boxes * box_raw;
-  const int64_t groups = (M + a.R - 1) / a.R;
-  if (M > (int64_t(1) << 31) - 1 - a.R || groups > (int64_t(1) << 30)) return KQ_ERR_INVALID;
+  const int group_rows = kAdaHalves * a.R;
+  const int64_t groups = (M + group_rows - 1) / group_rows;
+  if (M > (int64_t(1) << 31) - 1 - group_rows || groups > (int64_t(1) << 30))
+    return KQ_ERR_INVALID;
   a.groups = static_cast<int32_t>(groups);
   a.eps = eps;
   a.params = params;
@@ -526,7 +570,8 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   // Barriers, four slot buffers and the modulation table (alpha and beta,
   // 256 bytes a thread).
   const int fixed =
-      1024 + (kAdaMaxStages + 2) * 8 + kAdaSlotBufs * kAdaSlots * 16 + 16 * kAdaCons * 16;
+      1024 + (kAdaMaxStages + 2) * 8 + kAdaSlotBufs * kAdaHalves * kAdaSlots * 16 +
+      16 * kAdaCons * 16;
   a.stages = std::min(kAdaMaxStages, (di->smem_optin - fixed) / a.stage_bytes);
   if (a.stages < 2) return KQ_ERR_INVALID;
   const int smem = a.stages * a.stage_bytes + fixed;
@@ -534,7 +579,8 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBlock), static_cast<cuuint64_t>(nb),
                               static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[2] = {kBlock * 2, static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[3] = {kBlock, static_cast<cuuint32_t>(a.Wb), static_cast<cuuint32_t>(a.R)};
+  const cuuint32_t box[3] = {kBlock, static_cast<cuuint32_t>(a.Wb),
+                             static_cast<cuuint32_t>(kAdaHalves * a.R)};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult cr = tensor_map_encoder()(
       &map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims, strides, box,
