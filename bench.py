@@ -300,6 +300,71 @@ def _config(d, M, impl, block=32):
     }
 
 
+# Per-config table: the three quantizers at every config (C0..C4, first gain
+# input), per-launch CUDA events with L2 flushed before every launch.
+PER_CONFIG_REPS = 50
+PER_CONFIG_WARMUP = 10
+LATENCY_BOUND_US = 10.0     # roofline time below this: launch latency dominates
+
+
+def per_config_table(dev, peak, stress=None):
+    """Median, p10 and p90 per launch of kq_quantize, kq_quantize_hadamard and
+    kq_quantize_smooth at every config.  Before each launch a buffer of twice
+    the L2 size is overwritten, so every launch reads x from HBM; configs whose
+    roofline time is under LATENCY_BOUND_US are labelled latency-bound.
+    ``stress`` = (x, params, inv_s) already on the device reuses C4's input."""
+    import numpy as np
+    import torch
+    import workloads as w
+    import w4a4_post_quantization_b200 as kq
+    flush = torch.empty(int(2 * L2_BYTES) // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for name, cfg in w.CONFIGS.items():
+        for di in range(len(cfg["d"])):
+            if name == "stress" and stress is not None:
+                x, params, inv_s = stress
+            else:
+                c = w.make_case(name, di, 0)
+                x = c.x.to(dev)
+                params = torch.from_numpy(c.params).to(dev)
+                inv_s = torch.from_numpy(c.inv_s).to(dev)
+            M, d = x.shape
+            q = torch.empty((M, d // 2), dtype=torch.uint8, device=dev)
+            s = torch.empty((M, d // 32), dtype=torch.uint8, device=dev)
+            alg = w.algorithmic_bytes(M, d)
+            fns = {"kron": lambda: kq.quantize(x, params, q, s),
+                   "hadamard": lambda: kq.quantize_hadamard(x, q, s),
+                   "smooth": lambda: kq.quantize_smooth(x, inv_s, q, s)}
+            row = {"config": f"{name} d={d}", "M": M, "d": d, "algorithmic_bytes": alg,
+                   "regime": ("latency-bound" if alg / (peak * 1e9) * 1e6 < LATENCY_BOUND_US
+                              else "bandwidth")}
+            for vname, fn in fns.items():
+                for _ in range(PER_CONFIG_WARMUP):
+                    fn()
+                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                      for _ in range(PER_CONFIG_REPS)]
+                torch.cuda.synchronize()
+                for e0, e1 in ev:
+                    flush.zero_()
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                torch.cuda.synchronize()
+                us = np.array([e0.elapsed_time(e1) * 1e3 for e0, e1 in ev])
+                med = float(np.median(us))
+                row[vname] = {"median_us": med, "p10_us": float(np.percentile(us, 10)),
+                              "p90_us": float(np.percentile(us, 90)),
+                              "gbs": alg / (med * 1e-6) / 1e9,
+                              "frac": alg / (med * 1e-6) / 1e9 / peak}
+            rows.append(row)
+            del q, s
+    del flush
+    return {"reps": PER_CONFIG_REPS, "warmup": PER_CONFIG_WARMUP,
+            "l2": "a 2x L2 buffer overwritten before every launch",
+            "latency_bound_below_us": LATENCY_BOUND_US, "rows": rows}
+
+
 # --------------------------------------------------------------- GPU leg
 def time_steps(fn, steps: int, warmup: int, stream, sampler=None):
     """Average ms per step over exactly ``steps`` calls, CUDA events on
@@ -501,6 +566,9 @@ def run_gpu(args):
             "frac": tflops / fp4_peak,
             "kernel": "gemm_mxf4_kernel<tiled scales> (tcgen05.mma kind::mxf4)"}
         del qw, sw, cg, qt, st_
+        if world == 1 and args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"]:
+            variants["per_config"] = per_config_table(dev, measured_peak()[0],
+                                                      (x, params, inv_s))
 
     # End to end through the public API: pinned host x in, pinned host codes
     # and scales out, streamed through a device workspace (kq_quantize_host).
