@@ -233,13 +233,16 @@ def oracle_pool(workers: int):
     return pool
 
 
-def time_oracle(pool, case, rows: int, chunk: int = 128):
+def time_oracle(pool, case, rows: int, chunk: int = 128, per_chunk=None):
     """Wall time of the oracle over the first ``rows`` rows, split in chunks
-    over the pool's workers."""
+    over the pool's workers; ``per_chunk`` (a list) receives each chunk's own
+    compute time on its one core."""
     bits = case.x_bits()[:rows]
     jobs = [(bits[r:r + chunk], case.params) for r in range(0, rows, chunk)]
     t0 = time.perf_counter()
-    pool.map(_oracle_chunk, jobs)
+    times = pool.map(_oracle_chunk, jobs)
+    if per_chunk is not None:
+        per_chunk.extend(times)
     return time.perf_counter() - t0
 
 
@@ -624,13 +627,16 @@ def run_gpu(args):
     cpu = None
     if pool is not None and rank == 0:
         rows = CPU_SAMPLE_ROWS
-        sec = time_oracle(pool, case, rows)
+        chunk_s = []
+        sec = time_oracle(pool, case, rows, per_chunk=chunk_s)
         pool.close()
         cpu = {"value": w.algorithmic_bytes(rows, d) / sec / 1e9, "unit": UNIT,
                "cores": _cpu_workers(), "kind": "oracle",
                "sample": f"rows 0-{rows - 1} of the {M}x{d} stress input, float64 numpy "
                          f"oracle in {_cpu_workers()} spawned processes, 1 BLAS thread each, "
-                         f"{sec:.2f} s wall"}
+                         f"{sec:.2f} s wall",
+               # One core: the same chunks' compute times inside their workers.
+               "single_core_value": w.algorithmic_bytes(rows, d) / sum(chunk_s) / 1e9}
 
     if args.op == "gemm":
         roof = roof_gemm
