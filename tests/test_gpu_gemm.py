@@ -223,3 +223,27 @@ def test_persistent_and_per_tile_kernels_agree(M, N, K, dt, monkeypatch):
                outs[0].float().cpu().numpy(), qa, sa, qb, sb, rows=rows) \
         if dt == torch.float32 else None
     assert kq.device_status() == 0
+
+
+@pytest.mark.parametrize("M,N,K,dt", [(256, 256, 256, torch.float32),
+                                      (300, 520, 544, torch.float32),
+                                      (1, 8, 32, torch.float32),
+                                      (2048, 4096, 1152, torch.bfloat16),
+                                      (384, 768, 12320, torch.bfloat16)])
+def test_cta_pair_kernel_agrees(M, N, K, dt, monkeypatch):
+    """The CTA-pair kernel (clusters of two, tcgen05.mma.cta_group::2 on
+    256 x 256 tiles, each CTA loading half of B) gives the persistent
+    one-CTA kernel's output bit for bit, within the tolerance of the exact
+    product on sampled rows; tile edges in M and N, partial last k-tiles."""
+    qa, sa, qb, sb = random_operands(M, N, K, seed=M * 3 + N + K)
+    ta, tb = kq.scales_to_tiled(_dev(sa), K), kq.scales_to_tiled(_dev(sb), K)
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("KQ_GEMM_PAIR", flag)
+        outs.append(kq.gemm_mxfp4_tiled(_dev(qa), ta, _dev(qb), tb, out_dtype=dt))
+    torch.cuda.synchronize()
+    assert kq.device_status() == 0
+    assert torch.equal(outs[0], outs[1])
+    if dt == torch.float32:
+        rows = np.unique(np.array([0, min(1, M - 1), min(127, M - 1), min(128, M - 1), M // 2, M - 1]))
+        check_gemm(outs[0].cpu().numpy(), qa, sa, qb, sb, rows=rows)

@@ -105,6 +105,20 @@ __device__ __forceinline__ void mma_mxf4(uint32_t tmem_d, uint64_t adesc, uint64
       : "memory");
 }
 
+// The same MMA over a CTA pair (M = 256): issued by the even CTA, A rows and
+// accumulator rows 0..127 in it and 128..255 in the odd one, B's N rows split
+// 128 / 128 between their shared memories, each CTA's scales in its TMEM.
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                              uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
+      "\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
 // Untiled bulk copy of `bytes` (a multiple of 16, 16-byte aligned ends)
 // from global memory into this CTA's shared memory, completing on `bar`.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
@@ -798,6 +812,277 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// CTA-pair kernel (tiled scales per 32): clusters of two CTAs walk the banded
+// order of 256 x 256 output tiles with tcgen05.mma.cta_group::2 (M = 256).
+// Each CTA loads its 128 rows of A and its 128 rows of B, so B costs each SM
+// half the bytes per flop of a one-CTA tile, plus the scales of its A rows
+// and of all 256 B rows (the MMA reads B's scales from each CTA's own TMEM).
+// The even CTA (rank 0) issues the scale copies, the MMAs and the commits;
+// the commits arrive on the barriers of both CTAs, and every TMA load of the
+// pair counts its bytes on rank 0's stage barrier.  No load uses cluster
+// multicast.  Every cross-CTA wait is bounded; both CTAs always reach the
+// final TMEM release.
+constexpr int kQBN = 128;                                     // B rows per CTA
+constexpr int kQBTile = kQBN * kBKBytes;                      // 16 KiB
+constexpr int kQStage = kATile + kQBTile + kSfaBytes + kSfbBytes;   // 35 KiB
+constexpr int kQStages = 6;
+constexpr int kQBoxRows = 64;                                 // staging box: 64 rows x 128 B
+constexpr int kQStaging = kQBoxRows * 128;
+constexpr int kQSmem = 1024 + kQStages * kQStage + kQStaging + (2 * kQStages + 4) * 8 + 16;
+constexpr int kQTile = 2 * kBM;                               // 256 rows and columns a tile
+static_assert(kQStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+static_assert(kQSmem <= 232448, "shared memory");
+static_assert(kSfCol0 + kQStages * (kSfColsA + kSfColsB) <= kTmemCols, "TMEM columns");
+// M = 256 over the pair, N = 256.
+constexpr uint32_t kIdescMxf4Pair = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) |
+                                    (1u << 23) | (uint32_t(kQTile >> 4) << 24);
+// Bytes one k-tile brings into the pair: codes of 128 A rows and 128 B rows,
+// the A scales of 128 rows and the B scales of 256 rows, per CTA.
+constexpr uint32_t kQTxBytes = 2u * kQStage;
+
+struct PairArgs {
+  int32_t K, k_tiles, m_tiles, n_tiles;     // tiles of 256 x 256
+  int32_t out_bf16;
+  int* err;
+};
+
+__device__ __forceinline__ void pair_tile_origin(const PairArgs& a, int t, int& m0, int& n0) {
+  const int band = t / (kBandN * a.m_tiles);
+  const int r = t - band * kBandN * a.m_tiles;
+  const int width = min(kBandN, a.n_tiles - band * kBandN);
+  m0 = (r / width) * kQTile;
+  n0 = (band * kBandN + r % width) * kQTile;
+}
+
+__global__ void __launch_bounds__(kPThreads, 1)
+    gemm_mxf4_pair(const __grid_constant__ CUtensorMap amap,
+                   const __grid_constant__ CUtensorMap bmap,
+                   const __grid_constant__ CUtensorMap sfamap,
+                   const __grid_constant__ CUtensorMap sfbmap,
+                   const __grid_constant__ CUtensorMap cmap, const PairArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
+  uint8_t* staging = base + kQStages * kQStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kQStaging);
+  uint64_t* empty = full + kQStages;
+  uint64_t* acc_full = empty + kQStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  const int n_tiles_total = a.m_tiles * a.n_tiles;
+  const int nk = a.k_tiles;
+
+  if (tid == 0) {
+    for (int st = 0; st < kQStages; ++st) {
+      mbar_init(&full[st], 1);               // rank 0's producer, plus the pair's bytes
+      mbar_init(&empty[st], 1);              // rank 0's commit, multicast
+    }
+    mbar_init(acc_full, 1);                  // rank 0's commit, multicast
+    mbar_init(acc_empty, 8);                 // the four epilogue warps of each CTA
+    fence_mbar_init_cluster();
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, kTmemCols);
+  tmem_fence_before();
+  cluster_sync();                            // barriers of both CTAs initialised
+  tmem_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_map(&amap);
+      tma_prefetch_map(&bmap);
+      tma_prefetch_map(&sfamap);
+      tma_prefetch_map(&sfbmap);
+      int s = 0, g = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = pair; t < n_tiles_total && ok; t += n_pairs) {
+        int m0, n0;
+        pair_tile_origin(a, t, m0, n0);
+        const int am0 = m0 + (int)rank * kBM, bn0 = n0 + (int)rank * kQBN;
+        for (int kt = 0; kt < nk; ++kt, ++g) {
+          if (g >= kQStages && !mbar_wait(&empty[s], phase)) {
+            ok = false;
+            break;
+          }
+          uint8_t* stg = base + s * kQStage;
+          const uint32_t fb = cluster_addr(&full[s], 0);
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], kQTxBytes);
+          uint8_t* sfa = stg + kATile + kQBTile;
+          // Scales: chunks 2 kt, 2 kt + 1 of this CTA's A row tile and of
+          // the tile's two B row tiles (zero past the ends).
+          tma_load_4d_pair(sfa, &sfamap, 0, 0, 2 * kt, am0 / 128, fb);
+          tma_load_4d_pair(sfa + kSfaBytes, &sfbmap, 0, 0, 2 * kt, n0 / 128, fb);
+          tma_load_2d_pair(stg, &amap, kt * kBKBytes, am0, fb);
+          tma_load_2d_pair(stg + kATile, &bmap, kt * kBKBytes, bn0, fb);
+          if (++s == kQStages) {
+            s = 0;
+            if (g >= kQStages) phase ^= 1;
+          }
+        }
+      }
+      if (!ok) atomicOr(a.err, kErrProducerWait);
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------- scale copies + MMA
+    if (rank == 0 && lane == 0) {
+      int s = 0, i = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      auto ktile = [&](int kt, auto full_tile) -> bool {
+        if (!mbar_wait(&full[s], phase)) return false;
+        tmem_fence_after();
+        const uint8_t* stg = base + s * kQStage;
+        const uint8_t* sfa = stg + kATile + kQBTile;
+        const uint8_t* sfb = sfa + kSfaBytes;
+        const uint32_t tsfa = tmem_base + kSfCol0 + s * (kSfColsA + kSfColsB);
+        const uint32_t tsfb = tsfa + kSfColsA;
+#pragma unroll
+        for (int c = 0; c < kChunksPerStage; ++c) {
+          tmem_cp_pair_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
+#pragma unroll
+          for (int gb = 0; gb < kBN / 128; ++gb)
+            tmem_cp_pair_32x128b_x4(tsfb + 8 * c + 4 * gb,
+                                    smem_desc_rows16(smem_addr(sfb + (2 * gb + c) * kSfChunk)));
+        }
+        const uint64_t adesc = smem_desc_sw128(smem_addr(stg));
+        const uint64_t bdesc = smem_desc_sw128(smem_addr(stg + kATile));
+        const int n_mma = decltype(full_tile)::value
+                              ? kBK / kMmaK
+                              : min(kBK / kMmaK, (a.K - kt * kBK + kMmaK - 1) / kMmaK);
+#pragma unroll
+        for (int kk = 0; kk < kBK / kMmaK; ++kk) {
+          if (!decltype(full_tile)::value && kk >= n_mma) break;
+          const uint32_t sf_id = 2u * (kk & 1);
+          const uint32_t idesc = kIdescMxf4Pair | (sf_id << 29) | (sf_id << 4);
+          mma_mxf4_pair(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
+                        tsfb + 8 * (kk >> 1), (kt | kk) != 0);
+        }
+        mma_commit_pair(&empty[s]);
+        if (++s == kQStages) {
+          s = 0;
+          phase ^= 1;
+        }
+        return true;
+      };
+      for (int t = pair; t < n_tiles_total && ok; t += n_pairs, ++i) {
+        // The accumulators are free once both CTAs' epilogues read tile i - 1.
+        if (i >= 1 && !mbar_wait_cluster(acc_empty, (i - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tmem_fence_after();
+        const int nk_full = a.K % kBK == 0 ? nk : nk - 1;
+        int kt = 0;
+        for (; ok && kt < nk_full; ++kt) ok = ktile(kt, std::true_type{});
+        if (ok && kt < nk) ok = ktile(kt, std::false_type{});
+        mma_commit_pair(acc_full);           // also after a failed wait: epilogues go on
+      }
+      if (!ok) atomicOr(a.err, kErrConsumerWait);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // This CTA's 128 accumulator rows (TMEM lane quarter = warp mod 4),
+    // through the staging box as 128-byte-swizzled boxes of 128 rows x 128
+    // bytes, one box at a time.
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
+    const bool issuer = warp == 2 && lane == 0;
+    const uint32_t acc_empty0 = cluster_addr(acc_empty, 0);
+    constexpr int kParts = kBM / kQBoxRows;         // row boxes per column box
+    const int part = r / kQBoxRows;
+    uint8_t* srow = staging + (r - part * kQBoxRows) * 128;
+    auto epi_sync = [] { asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory"); };
+    auto store_box = [&](int row0, int col, const uint32_t (&wv)[32]) {
+#pragma unroll
+      for (int pp = 0; pp < kParts; ++pp) {
+        if (issuer) bulk_wait_read_0();
+        epi_sync();
+        if (part == pp) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(srow + 16 * (c ^ (r & 7))) =
+                make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        epi_sync();
+        if (issuer) {
+          tma_store_2d(&cmap, staging, col, row0 + pp * kQBoxRows);
+          bulk_commit();
+        }
+      }
+    };
+    bool ok = true;
+    int i = 0;
+    for (int t = pair; t < n_tiles_total; t += n_pairs, ++i) {
+      int m0, n0;
+      pair_tile_origin(a, t, m0, n0);
+      const int row0 = m0 + (int)rank * kBM;
+      // One AND-barrier makes a timeout the same for the four warps, which
+      // then stop (one bounded wait per failure, not one per tile).
+      ok = bar_and(3, 4 * 32, mbar_wait(acc_full, i & 1));
+      if (!ok) break;
+      tmem_fence_after();
+      if (a.out_bf16) {
+        uint32_t h[kBN / 2];
+#pragma unroll
+        for (int v = 0; v < kBN / 32; ++v) {
+          uint32_t x[32];
+          tmem_ld32(taddr + 32 * v, x);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const __nv_bfloat162 p =
+                __floats2bfloat162_rn(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1]));
+            h[16 * v + q] = *reinterpret_cast<const uint32_t*>(&p);
+          }
+        }
+        tmem_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty0);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          uint32_t wv[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) wv[k] = h[32 * b + k];
+          store_box(row0, n0 + 64 * b, wv);
+        }
+      } else {
+#pragma unroll 1
+        for (int b = 0; b < kBN / 32; ++b) {
+          uint32_t x[32];
+          tmem_ld32(taddr + 32 * b, x);
+          tmem_wait_ld();
+          if (b == kBN / 32 - 1) {
+            tmem_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty0);
+          }
+          store_box(row0, n0 + 32 * b, x);
+        }
+      }
+    }
+    if (!ok && lane == 0) atomicOr(a.err, kErrConsumerWait);
+    if (issuer) bulk_wait_all();
+    tmem_fence_before();
+  }
+  // Neither CTA leaves, nor frees its TMEM, before the other has made all its
+  // arrivals on its barriers and the MMAs on its memory have completed: every
+  // wait above is bounded, so both CTAs get here.
+  __syncwarp();
+  cluster_sync();
+  if (warp == 1) {
+    tmem_fence_after();
+    tmem_dealloc_pair(tmem_base, kTmemCols);
+  }
+}
+
 }  // namespace
 }  // namespace kq
 
@@ -819,6 +1104,68 @@ bool persistent_gemm() {
 bool persistent_gemm16() {
   const char* e = getenv("KQ_GEMM16_PERSISTENT");
   return e ? atoi(e) != 0 : true;
+}
+
+// The CTA-pair kernel for scales per 32 (KQ_GEMM_PAIR=1 selects it).
+bool pair_gemm() {
+  const char* e = getenv("KQ_GEMM_PAIR");
+  return e ? atoi(e) != 0 : false;
+}
+
+// Tiled scales [row tiles][4-scale columns][512 bytes] as a 4-D byte tensor
+// {256, 2, columns, row tiles}; a box {256, 2, 2, box_tiles} is the two
+// columns of one k-tile for box_tiles row tiles (zeros past either end).
+bool encode_scales_map(CUtensorMap* map, const uint8_t* sf, int64_t row_tiles, int64_t cols,
+                       int box_tiles) {
+  const cuuint64_t dims[4] = {256, 2, static_cast<cuuint64_t>(cols),
+                              static_cast<cuuint64_t>(row_tiles)};
+  const cuuint64_t strides[3] = {256, 512, static_cast<cuuint64_t>(cols) * 512};
+  const cuuint32_t box[4] = {256, 2, 2, static_cast<cuuint32_t>(box_tiles)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return tensor_map_encoder()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(sf),
+                              dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Launches the CTA-pair kernel: clusters of two, as many as can be resident.
+int launch_gemm_pair(const CUtensorMap& amap, const uint8_t* qb, const uint8_t* sa,
+                     const uint8_t* sb, const CUtensorMap& cmap, const GemmArgs& g,
+                     const DeviceInfo* di, int dev, cudaStream_t st) {
+  CUtensorMap bmap, sfamap, sfbmap;
+  if (!encode_codes_map(&bmap, qb, g.N, g.K, kQBN) ||
+      !encode_scales_map(&sfamap, sa, (g.M + 127) / 128, g.sf_tiles_k, 1) ||
+      !encode_scales_map(&sfbmap, sb, g.sf_tiles_n, g.sf_tiles_k, 2))
+    return record_cuda_error(cudaErrorInvalidValue);
+  PairArgs pa{};
+  pa.K = g.K;
+  pa.k_tiles = g.k_tiles;
+  pa.m_tiles = (g.M + kQTile - 1) / kQTile;
+  pa.n_tiles = (g.N + kQTile - 1) / kQTile;
+  pa.out_bf16 = g.out_bf16;
+  pa.err = g.err;
+  int rc = allow_smem<gemm_mxf4_pair>(kQSmem, dev);
+  if (rc != KQ_OK) return rc;
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kPThreads);
+  cfg.dynamicSmemBytes = kQSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * (di->sms / 2)));
+  int clusters = 0;
+  cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, gemm_mxf4_pair, &cfg);
+  if (e != cudaSuccess || clusters < 1) return record_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
+  const int64_t tiles = (int64_t)pa.m_tiles * pa.n_tiles;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * std::min<int64_t>(tiles, clusters)));
+  e = cudaLaunchKernelEx(&cfg, gemm_mxf4_pair, amap, bmap, sfamap, sfbmap, cmap, pa);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  return KQ_OK;
 }
 
 int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const uint8_t* sb,
@@ -860,11 +1207,13 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   // TMA-store epilogue when the output row pitch is a multiple of 16 bytes.
   const int esize = c_dtype == KQ_OUT_BF16 ? 2 : 4;
   a.tma_store = (N * esize) % 16 == 0;
+  const bool pair = tiled && a.tma_store && scale_block == 32 && pair_gemm();
   cmap = amap;
   if (a.tma_store) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * esize};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize), kBM};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize),
+                               static_cast<cuuint32_t>(pair ? kQBoxRows : kBM)};
     const cuuint32_t estr[2] = {1, 1};
     if (tensor_map_encoder()(&cmap,
                              esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -887,6 +1236,8 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled16>>(G::kSmem, dev);
     if (rc != KQ_OK) return rc;
     gemm_mxf4_kernel<kSfTiled16><<<grid, 32 * kSfWarp0, G::kSmem, st>>>(amap, bmap, cmap, a);
+  } else if (pair) {
+    return launch_gemm_pair(amap, qb, sa, sb, cmap, a, di, dev, st);
   } else if (tiled && a.tma_store && persistent_gemm()) {
     rc = allow_smem<gemm_mxf4_persistent<kSfTiled>>(PGeom<kSfTiled>::kSmem, dev);
     if (rc != KQ_OK) return rc;
