@@ -496,6 +496,9 @@ __global__ void __launch_bounds__(kAdaCons, 1)
   float4* modtab = slots + kAdaSlotBufs * kAdaHalves * kAdaSlots;  // [16][kAdaCons]
   const int tid = threadIdx.x;
   const int S = a.stages;
+  // Programmatic dependent launch: nothing global is read or written before
+  // the previous kernel of the stream has completed.
+  pdl_wait_then_trigger();
   if (tid == 0) {
     for (int s = 0; s < S; ++s) mbar_init(&full[s], 1);
     mbar_init(&statbar[0], kAdaWarps);
@@ -591,11 +594,13 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   if (y) {
     rc = allow_smem<adaln_kernel<1>>(smem, dev);
     if (rc != KQ_OK) return rc;
-    adaln_kernel<1><<<grid, kAdaCons, smem, st>>>(map, a);
+    cudaError_t e = launch_pdl(adaln_kernel<1>, dim3(grid), dim3(kAdaCons), smem, st, map, a);
+    if (e != cudaSuccess) return record_cuda_error(e);
   } else {
     rc = allow_smem<adaln_kernel<0>>(smem, dev);
     if (rc != KQ_OK) return rc;
-    adaln_kernel<0><<<grid, kAdaCons, smem, st>>>(map, a);
+    cudaError_t e = launch_pdl(adaln_kernel<0>, dim3(grid), dim3(kAdaCons), smem, st, map, a);
+    if (e != cudaSuccess) return record_cuda_error(e);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_error(e);

@@ -619,6 +619,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __syncthreads();
   tmem_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Set-up above overlaps the previous kernel of the stream (programmatic
+  // dependent launch); operands are read and C written only after this.
+  pdl_wait_then_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -1229,8 +1232,9 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
     rc = allow_smem<gemm_mxf4_persistent<kSfTiled16>>(PGeom<kSfTiled16>::kSmem, dev);
     if (rc != KQ_OK) return rc;
     const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
-    gemm_mxf4_persistent<kSfTiled16>
-        <<<pgrid, kPThreads, PGeom<kSfTiled16>::kSmem, st>>>(amap, bmap, cmap, a);
+    cudaError_t le = launch_pdl(gemm_mxf4_persistent<kSfTiled16>, dim3(pgrid), dim3(kPThreads),
+                                PGeom<kSfTiled16>::kSmem, st, amap, bmap, cmap, a);
+    if (le != cudaSuccess) return record_cuda_error(le);
   } else if (scale_block == 16) {
     using G = StageGeom<kSfTiled16>;
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled16>>(G::kSmem, dev);
@@ -1242,8 +1246,9 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
     rc = allow_smem<gemm_mxf4_persistent<kSfTiled>>(PGeom<kSfTiled>::kSmem, dev);
     if (rc != KQ_OK) return rc;
     const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
-    gemm_mxf4_persistent<kSfTiled>
-        <<<pgrid, kPThreads, PGeom<kSfTiled>::kSmem, st>>>(amap, bmap, cmap, a);
+    cudaError_t le = launch_pdl(gemm_mxf4_persistent<kSfTiled>, dim3(pgrid), dim3(kPThreads),
+                                PGeom<kSfTiled>::kSmem, st, amap, bmap, cmap, a);
+    if (le != cudaSuccess) return record_cuda_error(le);
   } else if (tiled) {
     // No scale warps: six warps.
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled>>(kSmemBytes, dev);

@@ -49,6 +49,32 @@ int allow_smem(int bytes, int dev) {
   return KQ_OK;
 }
 
+// Launches `kernel` with programmatic stream serialization, so that its
+// set-up overlaps the tail of the previous kernel of the stream (the kernel
+// executes griddepcontrol.wait before its first global read or write); a
+// plain launch where the runtime refuses the attribute.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    kernel<<<grid, block, smem, st>>>(args...);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
 // Launchers defined in other translation units.
 int launch_mma_kron(const uint16_t* x, int64_t M, int64_t d, const float* params, uint8_t* q,
                     uint8_t* scales, float* y, cudaStream_t st);

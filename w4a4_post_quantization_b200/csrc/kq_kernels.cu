@@ -401,13 +401,11 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     fence_mbar_init();
   }
   __syncthreads();
-  // Programmatic dependent launch: everything above overlaps the previous
+  // Programmatic dependent launch: the set-up above overlaps the previous
   // kernel of the stream; every global read and write of this grid comes
-  // after the wait, which returns once that kernel has completed and its
-  // memory is visible.  The next kernel may then start its own set-up as
-  // soon as SMs free up (it waits the same way before touching memory).
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // after the wait.  The next kernel may then start its own set-up as soon
+  // as SMs free up (it waits the same way before touching memory).
+  pdl_wait_then_trigger();
 
   const int panel = blockIdx.x % a.panels;
   const int cpp = gridDim.x / a.panels;           // CTAs per panel
@@ -800,24 +798,8 @@ int launch_panel_cfg(const uint16_t* x, int64_t M, int64_t d, const float* aux, 
   const int64_t resident = (int64_t)di.sms * Cfg::kMinBlocks;
   const int64_t per_panel = std::max<int64_t>(1, std::min<int64_t>(resident / a.panels, row_tiles));
   const int grid = static_cast<int>(per_panel * a.panels);
-  // Launched with programmatic stream serialization (the kernel waits for
-  // its predecessor itself); a plain launch where the runtime refuses it.
-  cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(Cfg::kThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-  cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, panel_kernel<kXf, kOut, Cfg>, map, a);
-  if (e != cudaSuccess) {
-    (void)cudaGetLastError();
-    panel_kernel<kXf, kOut, Cfg><<<grid, Cfg::kThreads, smem, st>>>(map, a);
-    e = cudaGetLastError();
-  }
+  cudaError_t e = launch_pdl(panel_kernel<kXf, kOut, Cfg>, dim3(static_cast<unsigned>(grid)),
+                             dim3(Cfg::kThreads), static_cast<size_t>(smem), st, map, a);
   if (e != cudaSuccess) return cuda_fail(e);
   return KQ_OK;
 }
