@@ -90,6 +90,7 @@ __global__ void __launch_bounds__(kGradThreads)
     params_grad_kernel(const GradArgs a) {
   __shared__ float red[kGradRowLanes][kGradBlocksPerCta][kGradAcc];
   __shared__ bool last;
+  pdl_wait_then_trigger();     // programmatic dependent launch: no global access before
   const int bl = threadIdx.x % kGradBlocksPerCta, rl = threadIdx.x / kGradBlocksPerCta;
   const int j = blockIdx.x * kGradBlocksPerCta + bl;
   float acc[kGradAcc];
@@ -192,6 +193,7 @@ __global__ void __launch_bounds__(kResThreads)
                     double* partial, unsigned int* counter, double* sumsq) {
   __shared__ double red[kResThreads];
   __shared__ bool last;
+  pdl_wait_then_trigger();     // programmatic dependent launch: no global access before
   double acc = 0.0;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -226,6 +228,7 @@ __global__ void __launch_bounds__(kResThreads)
 __global__ void adam_kernel(float* p, const float* g0, const float* g1, float* m, float* v,
                             int64_t n, float lr, float beta1, float cbeta1, float beta2,
                             float cbeta2, float eps, float corr1, float corr2) {
+  pdl_wait_then_trigger();     // programmatic dependent launch: no global access before
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
     const float g = g0[i] + (g1 ? g1[i] : 0.f);
@@ -299,11 +302,9 @@ extern "C" int kq_transform_params_grad(const float* z, const float* zq, const f
   a.reg = reg;
   const dim3 grid((nb + kGradBlocksPerCta - 1) / kGradBlocksPerCta, splits);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (inverse_transpose)
-    params_grad_kernel<true><<<grid, kGradThreads, 0, st>>>(a);
-  else
-    params_grad_kernel<false><<<grid, kGradThreads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = inverse_transpose
+                      ? launch_pdl(params_grad_kernel<true>, grid, dim3(kGradThreads), 0, st, a)
+                      : launch_pdl(params_grad_kernel<false>, grid, dim3(kGradThreads), 0, st, a);
   if (e != cudaSuccess) return record_cuda_error(e);
   return KQ_OK;
 }
@@ -321,11 +322,10 @@ extern "C" int kq_residual(const float* y, const float* y_ref, int64_t n, float 
   if (rc != KQ_OK) return rc;
   const int64_t want = (n + kResThreads - 1) / kResThreads;
   const int grid = static_cast<int>(std::min<int64_t>(want, std::min(4096, di->sms * 8)));
-  residual_kernel<<<grid, kResThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      y, y_ref, n, scale, out,
-      reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + 256),
-      static_cast<unsigned int*>(workspace), sumsq);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(residual_kernel, dim3(grid), dim3(kResThreads), 0,
+                             static_cast<cudaStream_t>(stream), y, y_ref, n, scale, out,
+                             reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + 256),
+                             static_cast<unsigned int*>(workspace), sumsq);
   if (e != cudaSuccess) return record_cuda_error(e);
   return KQ_OK;
 }
@@ -344,11 +344,11 @@ extern "C" int kq_adam_step(float* params, const float* grad0, const float* grad
   const float corr1 = static_cast<float>(1.0 - std::pow(beta1, step));
   const float corr2 = static_cast<float>(1.0 - std::pow(beta2, step));
   const int grid = static_cast<int>(std::min<int64_t>((n + 255) / 256, di->sms * 4));
-  adam_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      params, grad0, grad1, m, v, n, static_cast<float>(lr), static_cast<float>(beta1),
+  cudaError_t e = launch_pdl(
+      adam_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), params, grad0,
+      grad1, m, v, n, static_cast<float>(lr), static_cast<float>(beta1),
       static_cast<float>(1.0 - beta1), static_cast<float>(beta2),
       static_cast<float>(1.0 - beta2), static_cast<float>(eps), corr1, corr2);
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_error(e);
   return KQ_OK;
 }

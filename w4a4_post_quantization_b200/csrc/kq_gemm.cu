@@ -295,6 +295,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tmem_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Programmatic dependent launch: no global access before this.
+  pdl_wait_then_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA codes
@@ -1239,7 +1241,9 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
     using G = StageGeom<kSfTiled16>;
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled16>>(G::kSmem, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<kSfTiled16><<<grid, 32 * kSfWarp0, G::kSmem, st>>>(amap, bmap, cmap, a);
+    cudaError_t le = launch_pdl(gemm_mxf4_kernel<kSfTiled16>, grid, dim3(32 * kSfWarp0), G::kSmem,
+                                st, amap, bmap, cmap, a);
+    if (le != cudaSuccess) return record_cuda_error(le);
   } else if (pair) {
     return launch_gemm_pair(amap, qb, sa, sb, cmap, a, di, dev, st);
   } else if (tiled && a.tma_store && persistent_gemm()) {
@@ -1253,15 +1257,21 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
     // No scale warps: six warps.
     rc = allow_smem<gemm_mxf4_kernel<kSfTiled>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<kSfTiled><<<grid, 32 * kSfWarp0, kSmemBytes, st>>>(amap, bmap, cmap, a);
+    cudaError_t le = launch_pdl(gemm_mxf4_kernel<kSfTiled>, grid, dim3(32 * kSfWarp0), kSmemBytes,
+                                st, amap, bmap, cmap, a);
+    if (le != cudaSuccess) return record_cuda_error(le);
   } else if ((a.sf_stride % 4 == 0) && al(sa, 4) && al(sb, 4)) {
     rc = allow_smem<gemm_mxf4_kernel<kSfRowWords>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<kSfRowWords><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, cmap, a);
+    cudaError_t le = launch_pdl(gemm_mxf4_kernel<kSfRowWords>, grid, dim3(kGemmThreads),
+                                kSmemBytes, st, amap, bmap, cmap, a);
+    if (le != cudaSuccess) return record_cuda_error(le);
   } else {
     rc = allow_smem<gemm_mxf4_kernel<kSfRowBytes>>(kSmemBytes, dev);
     if (rc != KQ_OK) return rc;
-    gemm_mxf4_kernel<kSfRowBytes><<<grid, kGemmThreads, kSmemBytes, st>>>(amap, bmap, cmap, a);
+    cudaError_t le = launch_pdl(gemm_mxf4_kernel<kSfRowBytes>, grid, dim3(kGemmThreads),
+                                kSmemBytes, st, amap, bmap, cmap, a);
+    if (le != cudaSuccess) return record_cuda_error(le);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_error(e);
