@@ -127,6 +127,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
   float* tab = reinterpret_cast<float*>(base + a.stages * kTileBytes);
   uint64_t* full = reinterpret_cast<uint64_t*>(tab + table_floats(kXf, a.nb));
   uint64_t* empty = full + a.stages;
+  pdl_wait_then_trigger();     // programmatic dependent launch: no global access before
 
   const int tid = threadIdx.x;
   if (tid == 0) {
@@ -501,6 +502,7 @@ __global__ void __launch_bounds__(kDirectThreads)
     direct_kernel(const void* __restrict__ xin, int64_t M, const LaunchArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* tab = reinterpret_cast<float*>(smem_raw);
+  pdl_wait_then_trigger();     // programmatic dependent launch: no global access before
   const int j0 = blockIdx.y * kDirectThreads;
   const int jn = min(kDirectThreads, a.nb - j0);
   build_table<kXf>(tab, a, j0, jn, threadIdx.x, blockDim.x);
@@ -568,6 +570,7 @@ __global__ void __launch_bounds__(256)
     dequant_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ scales, int64_t G,
                    float* __restrict__ y) {
   __shared__ float lut[16];
+  pdl_wait_then_trigger();     // programmatic dependent launch: no global access before
   if (threadIdx.x < 16) {
     const int c = threadIdx.x, e = (c >> 1) & 3, m = c & 1;
     const float mag = e == 0 ? 0.5f * m : ldexpf(1.0f + 0.5f * m, e - 1);
@@ -692,7 +695,9 @@ int launch_tma(const uint16_t* x, int64_t M, int64_t d, LaunchArgs a, cudaStream
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
     const int grid = std::min(la.n_tiles, di.sms);
-    tma_kernel<kXf, kOut><<<grid, kTmaThreads, smem, st>>>(map, la);
+    cudaError_t le = launch_pdl(tma_kernel<kXf, kOut>, dim3(grid), dim3(kTmaThreads), smem, st,
+                                map, la);
+    if (le != cudaSuccess) return cuda_fail(le);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e);
   }
@@ -843,7 +848,11 @@ int launch_direct(const void* x, int64_t M, int64_t d, LaunchArgs a, cudaStream_
   const int64_t want = std::max<int64_t>(1, (int64_t)di.sms * 8 / panels);
   const int rows = static_cast<int>(std::min<int64_t>(M, std::min<int64_t>(want, 65535)));
   dim3 grid(rows, panels);
-  direct_kernel<kXf, kOut, kF32In><<<grid, kDirectThreads, smem, st>>>(x, M, a);
+  {
+    cudaError_t le = launch_pdl(direct_kernel<kXf, kOut, kF32In>, grid, dim3(kDirectThreads), smem,
+                                st, x, M, a);
+    if (le != cudaSuccess) return cuda_fail(le);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return KQ_OK;
@@ -1083,7 +1092,11 @@ extern "C" int kq_dequantize(const uint8_t* q_packed, const uint8_t* scales, int
   const int64_t G = M * (d / kBlock);
   const int64_t want = (G + 255) / 256;
   const int grid = static_cast<int>(std::min<int64_t>(want, (int64_t)di->sms * 8));
-  dequant_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(q_packed, scales, G, y);
+  {
+    cudaError_t le = launch_pdl(dequant_kernel, dim3(grid), dim3(256), 0,
+                                static_cast<cudaStream_t>(stream), q_packed, scales, G, y);
+    if (le != cudaSuccess) return cuda_fail(le);
+  }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return KQ_OK;
