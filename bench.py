@@ -659,6 +659,8 @@ def run_gpu(args):
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3,
                            **({"gemm_shape_mnk": gemm_mnk} if args.op == "gemm" else {})),
             "hbm_frac": value / world / peak if args.op != "gemm" else None,
+            # Absolute throughput beside the bytes: elements of x per second, all ranks.
+            "elements_per_s": (M * d * world / (ms_max * 1e-3)) if args.op != "gemm" else None,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": args.steps, "variants": variants,
         }
