@@ -449,8 +449,8 @@ def run_gpu(args):
         qw, sw = kq.quantize_weight_tiled(Wg, pg)
         xg = w.device_randn_bf16((gm, gk), case.seed + 11, dev)
         qt, st_ = kq.quantize_tiled(xg, pg)
-        del Wg, xg
         cg = torch.empty((gm, gn), dtype=torch.bfloat16, device=dev)
+        layer_in = (xg, Wg, pg)
         gemm_flops = 2.0 * gm * gn * gk
     elif args.op == "gemm":
         # The layer the codes feed, as the timed step: C = Q(x T) Q(W T^-T)^T
@@ -458,9 +458,9 @@ def run_gpu(args):
         # quantizers write their scales in the tensor cores' tiled layout.
         Wg = w.device_randn_bf16((d, d), case.seed + 7, dev)
         qw, sw = kq.quantize_weight_tiled(Wg, params)
-        del Wg
         qt, st_ = kq.quantize_tiled(x, params)
         cg = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
+        layer_in = (x, Wg, params)
 
     if args.op == "gemm":
         def step():
@@ -513,7 +513,28 @@ def run_gpu(args):
 
     # Comparators and the copy ceiling on the same input (context, same GPU).
     variants = {}
-    if not args.quick:
+    if args.op == "gemm" and not args.quick:
+        # The linear layer as a user runs it: activations quantized on the fly
+        # (the weight offline), then the W4A4 product; against the same
+        # product in bf16 through torch.matmul (cuBLAS).
+        xl, wl, pl = layer_in
+        cb = torch.empty_like(cg)
+        n_l = max(3, min(args.steps, 20))
+        ms_b, _ = time_steps(lambda: torch.matmul(xl, wl.t(), out=cb), n_l, 3, stream)
+        ms_qa, _ = time_steps(lambda: kq.quantize_tiled(xl, pl, qt, st_), n_l, 3, stream)
+
+        def layer_step():
+            kq.quantize_tiled(xl, pl, qt, st_)
+            kq.gemm_mxfp4_tiled(qt, st_, qw, sw, out=cg, out_dtype=torch.bfloat16)
+        ms_l, _ = time_steps(layer_step, n_l, 3, stream)
+        ms_b, ms_qa, ms_l = (max_over_ranks(v, dev) for v in (ms_b, ms_qa, ms_l))
+        variants["layer"] = {
+            "shape_mnk": gemm_mnk, "out": "bf16", "steps": n_l,
+            "bf16_matmul": {"ms": ms_b, "tflops": gemm_flops / (ms_b * 1e-3) / 1e12},
+            "w4a4": {"ms": ms_l, "quantize_activations_ms": ms_qa,
+                     "tflops": gemm_flops / (ms_l * 1e-3) / 1e12},
+            "speedup_over_bf16": ms_b / ms_l}
+    if not args.quick and args.op != "gemm":
         ms_h, _ = time_steps(lambda: kq.quantize_hadamard(x, q, s), args.steps, args.warmup, stream)
         ms_s, _ = time_steps(lambda: kq.quantize_smooth(x, inv_s, q, s), args.steps, args.warmup,
                              stream)
@@ -535,7 +556,7 @@ def run_gpu(args):
             ms_i, _ = time_steps(lambda: kq.quantize(x, params, q, s, impl=code), args.steps,
                                  args.warmup, stream)
             impls[name] = alg_bytes / (max_over_ranks(ms_i, dev) * 1e-3) / 1e9
-        variants = {
+        variants.update({
             "eager_gbs": aggregate_gbs(alg_bytes, world, 1, eager_max),
             "kq_quantize_impl_gbs": impls,
             "hadamard": {"gbs": alg_bytes / (ms_max_h * 1e-3) / 1e9, "ms": ms_max_h},
@@ -547,7 +568,7 @@ def run_gpu(args):
                             "op": "LayerNorm + AdaLN modulate + transform + MXFP4, one pass"},
             "kronecker_over_smooth_speed": ms_max_s / ms_max,
             "d2d_copy_gbs": 2 * x.numel() * 2 / (ms_max_c * 1e-3) / 1e9,
-        }
+        })
         del buf
         # The layer the codes feed: C = Q(x T) Q(W T^-T)^T with a square
         # synthetic weight (d x d), bf16 output, block-scaled tcgen05 GEMM.
