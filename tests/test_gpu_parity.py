@@ -167,6 +167,27 @@ def test_singular_shear_factor_takes_the_plain_form():
     check_mx4(q.cpu().numpy(), s.cpu().numpy(), y64, cond)
 
 
+def test_panel_kernel_one_and_many_thread_rows_per_block():
+    """The panel kernel at widths where many thread-rows of a CTA share each
+    column block (36 blocks: 32 rows; 144 blocks: 8) and where one does (229
+    blocks, a prime width: the whole row is one panel), and with the plain
+    form forced on one panel by a singular factor in block 7: each matches
+    the oracle."""
+    for nb, M, singular in ((36, 131, False), (144, 37, False), (229, 9, False), (36, 70, True)):
+        d = nb * 32
+        x = w.random_bf16((M, d), seed=nb + M)
+        p = w.draw_params(d, 4)
+        if singular:
+            p = p.copy()
+            p[7, 1] = [-1.0, 1.0, 1.0]
+        q, s = kq.quantize(_gpu(x), _params_dev(p), impl=kq.KQ_IMPL_PANEL)
+        torch.cuda.synchronize()
+        x64 = o.bf16_bits_to_float64(x.view(torch.int16).numpy().view(np.uint16))
+        y64 = o.transform(x64, p)
+        st = check_mx4(q.cpu().numpy(), s.cpu().numpy(), y64, o.abs_transform(x64, p))
+        assert st["scale_exempt"] <= 2 and st["code_exempt"] <= max(4, st["elements"] // 10000)
+
+
 # ------------------------------------------------------------- edge cases
 def _edge(x_t, params, inv_s=None, bound=True):
     if inv_s is None:
