@@ -305,23 +305,56 @@ def _config(d, M, impl, block=32):
 
 # Per-config table: the three quantizers at every config (C0..C4, first gain
 # input), per-launch CUDA events with L2 flushed before every launch.
-PER_CONFIG_REPS = 50
-PER_CONFIG_WARMUP = 10
+PER_CONFIG_REPS = 50          # single-launch samples per quantizer and config
+PER_CONFIG_BLOCKS = 5         # back-to-back blocks per quantizer and config
+PER_CONFIG_BLOCK = 100        # launches per block (at least one pass over the copies)
+PER_CONFIG_MAX_COPIES = 512
 LATENCY_BOUND_US = 10.0     # roofline time below this: launch latency dominates
+HOST_AHEAD_CYCLES = 40_000_000   # about 20 ms of device sleep, far longer than queueing 50 launches
 
 
 def per_config_table(dev, peak, stress=None):
-    """Median, p10 and p90 per launch of kq_quantize, kq_quantize_hadamard and
-    kq_quantize_smooth at every config.  Before each launch a buffer of twice
-    the L2 size is overwritten, so every launch reads x from HBM; configs whose
-    roofline time is under LATENCY_BOUND_US are labelled latency-bound.
-    ``stress`` = (x, params, inv_s) already on the device reuses C4's input."""
+    """kq_quantize, kq_quantize_hadamard and kq_quantize_smooth at every config,
+    two ways.  Back to back: blocks of launches cycle over enough copies of x
+    (and of the outputs) that every launch reads x from HBM (each copy was
+    last touched three L2 sizes of traffic earlier); one event pair around a
+    block, the median over blocks.  Single launch: a buffer of twice the L2
+    size is overwritten before each launch and an event pair brackets it;
+    this includes the event and launch overhead (about 6 us for an empty
+    kernel timed the same way).  Configs whose roofline time is under
+    LATENCY_BOUND_US are labelled latency-bound.  ``stress`` = (x, params,
+    inv_s) already on the device reuses C4's input."""
     import numpy as np
     import torch
     import workloads as w
     import w4a4_post_quantization_b200 as kq
     flush = torch.empty(int(2 * L2_BYTES) // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    def block_us(fns, n):
+        torch.cuda.synchronize()
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            fns[i % len(fns)]()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e3 / n
+
+    def single_us(fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(PER_CONFIG_REPS)]
+        torch.cuda.synchronize()
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return float(np.median([e0.elapsed_time(e1) * 1e3 for e0, e1 in ev]))
+
     rows = []
     for name, cfg in w.CONFIGS.items():
         for di in range(len(cfg["d"])):
@@ -333,38 +366,37 @@ def per_config_table(dev, peak, stress=None):
                 params = torch.from_numpy(c.params).to(dev)
                 inv_s = torch.from_numpy(c.inv_s).to(dev)
             M, d = x.shape
-            q = torch.empty((M, d // 2), dtype=torch.uint8, device=dev)
-            s = torch.empty((M, d // 32), dtype=torch.uint8, device=dev)
             alg = w.algorithmic_bytes(M, d)
-            fns = {"kron": lambda: kq.quantize(x, params, q, s),
-                   "hadamard": lambda: kq.quantize_hadamard(x, q, s),
-                   "smooth": lambda: kq.quantize_smooth(x, inv_s, q, s)}
+            ncopy = min(PER_CONFIG_MAX_COPIES, max(1, int(np.ceil(3 * L2_BYTES / alg))))
+            xs = [x] + [x.clone() for _ in range(ncopy - 1)]
+            qs = [torch.empty((M, d // 2), dtype=torch.uint8, device=dev) for _ in range(ncopy)]
+            ss = [torch.empty((M, d // 32), dtype=torch.uint8, device=dev) for _ in range(ncopy)]
+            fams = {"kron": [lambda i=i: kq.quantize(xs[i], params, qs[i], ss[i]) for i in range(ncopy)],
+                    "hadamard": [lambda i=i: kq.quantize_hadamard(xs[i], qs[i], ss[i])
+                                 for i in range(ncopy)],
+                    "smooth": [lambda i=i: kq.quantize_smooth(xs[i], inv_s, qs[i], ss[i])
+                               for i in range(ncopy)]}
+            n = max(PER_CONFIG_BLOCK, ncopy)
             row = {"config": f"{name} d={d}", "M": M, "d": d, "algorithmic_bytes": alg,
+                   "copies": ncopy, "launches_per_block": n,
                    "regime": ("latency-bound" if alg / (peak * 1e9) * 1e6 < LATENCY_BOUND_US
                               else "bandwidth")}
-            for vname, fn in fns.items():
-                for _ in range(PER_CONFIG_WARMUP):
-                    fn()
-                ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                      for _ in range(PER_CONFIG_REPS)]
-                torch.cuda.synchronize()
-                for e0, e1 in ev:
-                    flush.zero_()
-                    e0.record(stream)
-                    fn()
-                    e1.record(stream)
-                torch.cuda.synchronize()
-                us = np.array([e0.elapsed_time(e1) * 1e3 for e0, e1 in ev])
-                med = float(np.median(us))
-                row[vname] = {"median_us": med, "p10_us": float(np.percentile(us, 10)),
-                              "p90_us": float(np.percentile(us, 90)),
+            for vname, fns in fams.items():
+                for f in fns:
+                    f()
+                blocks = [block_us(fns, n) for _ in range(PER_CONFIG_BLOCKS)]
+                med = float(np.median(blocks))
+                row[vname] = {"us": med, "min_us": float(min(blocks)), "max_us": float(max(blocks)),
                               "gbs": alg / (med * 1e-6) / 1e9,
-                              "frac": alg / (med * 1e-6) / 1e9 / peak}
+                              "frac": alg / (med * 1e-6) / 1e9 / peak,
+                              "single_launch_us": single_us(fns[0])}
             rows.append(row)
-            del q, s
+            del xs, qs, ss
     del flush
-    return {"reps": PER_CONFIG_REPS, "warmup": PER_CONFIG_WARMUP,
-            "l2": "a 2x L2 buffer overwritten before every launch",
+    return {"blocks": PER_CONFIG_BLOCKS, "single_launch_reps": PER_CONFIG_REPS,
+            "l2": "back to back over rotating copies of x (3x L2 of traffic between two uses "
+                  "of a copy); single launch after overwriting a 2x L2 buffer",
+            "host": "launches queued behind a device sleep: events time the device only",
             "latency_bound_below_us": LATENCY_BOUND_US, "rows": rows}
 
 
