@@ -313,6 +313,26 @@ LATENCY_BOUND_US = 10.0     # roofline time below this: launch latency dominates
 HOST_AHEAD_CYCLES = 40_000_000   # about 20 ms of device sleep, far longer than queueing 50 launches
 
 
+def gemm_kernel_name() -> str:
+    """The 32-element tiled-scale product kernel the library selects: the
+    persistent kernel unless KQ_GEMM_PERSISTENT=0, the CTA pair with
+    KQ_GEMM_PAIR=1 (the same switches the library reads)."""
+    def flag(var, default):           # the library's reading: atoi(value) != 0
+        v = os.environ.get(var)
+        if v is None:
+            return default
+        m = re.match(r"\s*[+-]?\d+", v)
+        return bool(m) and int(m.group()) != 0
+
+    if flag("KQ_GEMM_PAIR", False):
+        name = "gemm_mxf4_pair"
+    elif not flag("KQ_GEMM_PERSISTENT", True):
+        name = "gemm_mxf4_kernel"
+    else:
+        name = "gemm_mxf4_persistent"
+    return f"{name}<tiled scales> (tcgen05.mma kind::mxf4)"
+
+
 def per_config_table(dev, peak, stress=None):
     """kq_quantize, kq_quantize_hadamard and kq_quantize_smooth at every config,
     two ways.  Back to back: blocks of launches cycle over enough copies of x
@@ -620,7 +640,7 @@ def run_gpu(args):
             "shape_mnk": [M, d, d], "out": "bf16", "steps": g_steps, "ms": ms_max_g,
             "tflops": tflops, "peak_tflops": fp4_peak, "peak_source": fp4_src,
             "frac": tflops / fp4_peak,
-            "kernel": "gemm_mxf4_kernel<tiled scales> (tcgen05.mma kind::mxf4)"}
+            "kernel": gemm_kernel_name()}
         del qw, sw, cg, qt, st_
         if world == 1 and args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"]:
             variants["per_config"] = per_config_table(dev, measured_peak()[0],
@@ -664,14 +684,14 @@ def run_gpu(args):
         roof_gemm = {"bound": "tensor", "achieved": tf, "peak": fp4_peak, "unit": "TFLOP/s",
                      "frac": tf / fp4_peak, "peak_source": fp4_src, "traffic": None,
                      "algorithmic_flops_per_launch": gemm_flops,
-                     "kernel": "gemm_mxf4_kernel<tiled scales> (tcgen05.mma kind::mxf4)"}
+                     "kernel": gemm_kernel_name()}
     roof = {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
             "frac": per_launch_gbs / peak, "peak_source": peak_src,
             "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.md")
                         if args.op == "kron" else None),
             "algorithmic_bytes_per_launch": alg_bytes,
             "kernel": {"kron": "panel_kernel<kron, mx4>", "kron16": "panel_kernel<kron16, mx4>",
-                       "gemm": "gemm_mxf4_kernel",
+                       "gemm": gemm_kernel_name(),
                        "kron_mma": "mma_kernel", "adaln": "adaln_kernel<mx4>",
                        "hadamard": "panel_kernel<hadamard, mx4>",
                        "smooth": "panel_kernel<smooth, mx4>"}[args.op],
