@@ -15,7 +15,7 @@ the axiom and free-parameter ledger, "What would settle it"):
   (Appendix D.1 as the ledger quotes it);
 * the initialization is the Hadamard transform.
 
-Readings where the pages print no formula (listed in the design doc):
+Readings where the pages print no formula:
 
 * loss ``L = L_out + lam_A L_A + lam_W L_W`` with
   ``L_out = |Q(A) Q(B)^T - X W^T|^2 / |X W^T|^2``, ``A = X T``,

@@ -22,7 +22,7 @@ blocking, fusion or reordering beyond the definitions:
    scale and E2M1 elements (the OCP Microscaling formats the paper cites for
    "MXFP4e2"; abstract and "Core claim").
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 
 * the scale exponent is ``floor(log2(amax)) - 2`` (2 = the largest E2M1
   exponent), clamped to ``[-127, 127]``; an all-zero block gets ``-127``;

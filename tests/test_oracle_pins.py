@@ -72,7 +72,7 @@ def test_transform_matches_factorwise_contraction():
 
 
 def test_unit_determinant_every_block_of_every_config():
-    """det K = prod_k det(G_k)^16 = 1 for the BASELINE-form factors."""
+    """det K = prod_k det(G_k)^16 = 1 for the factors G = [[1,0],[a,1]] [[b,c],[0,1/b]]."""
     for name, di, gi in w.all_case_keys():
         seed = w.case_seed(name, di, gi)
         d = w.CONFIGS[name]["d"][di]
@@ -119,7 +119,7 @@ def test_eq6_form_at_hadamard_init_gives_sylvester_hadamard():
     np.testing.assert_allclose(o.hadamard_block(), K, atol=1e-15)
 
 
-def test_baseline_form_signed_hadamard():
+def test_lu_form_signed_hadamard():
     """(a,b,c) = (-1, 1/sqrt2, 1/sqrt2) gives G = [[1,1],[-1,1]]/sqrt2, so
     K = diag((-1)^popcount(r)) H32 / sqrt32, orthonormal."""
     s = 1 / math.sqrt(2)
