@@ -7,8 +7,9 @@ checked against it and it is never on the product path.
 What it follows (KroQuant review, pith.science: "What carries the argument",
 the axiom and free-parameter ledger, "What would settle it"):
 
-* the transform is learned per layer by minimizing the quantized output MSE
-  with auxiliary per-operand regularization (Eq. 2, 7, 9), with a
+* each layer's transform is fitted by driving down the mean squared error
+  of the quantized layer output, plus one extra penalty term for each of the
+  two quantized operands (Eq. 2, 7, 9), with a
   straight-through estimator through the quantizer (Section 3.3);
 * the regularization weights are set from the loss ratios at the
   initialization (Eq. 10); the optimizer is Adam, 100 steps, lr 1e-2
