@@ -687,8 +687,10 @@ def run_gpu(args):
                      "kernel": gemm_kernel_name()}
     roof = {"bound": "hbm", "achieved": per_launch_gbs, "peak": peak, "unit": "GB/s",
             "frac": per_launch_gbs / peak, "peak_source": peak_src,
+            # The capture is of one full-size stress launch: other row counts
+            # get no traffic figure.
             "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.md")
-                        if args.op == "kron" else None),
+                        if args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"] else None),
             "algorithmic_bytes_per_launch": alg_bytes,
             "kernel": {"kron": "panel_kernel<kron, mx4>", "kron16": "panel_kernel<kron16, mx4>",
                        "gemm": gemm_kernel_name(),
