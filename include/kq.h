@@ -151,7 +151,10 @@ int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const float* params1
  *   aligned; tokens_per_sample >= 1; 0 <= eps (finite).
  * d must be a positive multiple of 32 and at most 12288 (384 blocks).  The
  * statistics are float32 (two-pass per block, combined pairwise across the
- * row in a fixed order); h, the transform and the decision are float32. */
+ * row in a fixed order); h, the transform and the decision are float32.
+ * With eps = 0 a row whose d values are all equal has no normalized value
+ * (0 / 0): its codes and scale bytes are unspecified, nothing else is
+ * affected and no error is raised; any eps > 0 maps such a row to shift. */
 int kq_quantize_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
                       const uint16_t* scale, int64_t tokens_per_sample, float eps,
                       const float* params, uint8_t* q_packed, uint8_t* scales, void* stream);
