@@ -1,9 +1,12 @@
 """Multi-process host logic of the benchmark at world size 2 over gloo (CPU):
-row shards of one batch, whole-job throughput from the slowest rank, and the
-max-over-ranks reduction.  The quantizer itself has no data-path collective:
-every rank works on its own rows."""
+row shards of one batch, whole-job throughput from the slowest rank, the
+max-over-ranks reduction, and that reduction ending with an error when a
+rank has left.  The quantizer itself has no data-path collective: every rank
+works on its own rows."""
+import datetime
 import os
 import socket
+import time
 
 import numpy as np
 import pytest
@@ -65,3 +68,41 @@ def test_aggregate_throughput_counts_every_rank():
 def test_single_process_needs_no_process_group():
     assert not dist.is_initialized()
     assert bench.max_over_ranks(3.5) == 3.5
+
+
+def _worker_one_leaves(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        # Leaves between steps, with no collective of its own in flight.
+        out[1] = "left"
+        os._exit(0)
+    t0 = time.monotonic()
+    try:
+        bench.max_over_ranks(1.0)
+        out[0] = ("returned", time.monotonic() - t0)
+    except Exception as e:                     # the expected outcome
+        out[0] = ("raised", time.monotonic() - t0, type(e).__name__)
+    finally:
+        try:
+            dist.destroy_process_group()
+        except Exception:
+            pass
+
+
+@pytest.mark.timeout(180)
+def test_a_rank_that_leaves_ends_the_others_reduction_with_an_error():
+    """The max-over-ranks reduction that closes every timed region must not
+    wait for good on a rank that has gone: with a short process-group
+    timeout the remaining rank gets an error, well inside a minute."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    mp.start_processes(_worker_one_leaves, args=(world, _free_port(), out), nprocs=world,
+                       join=True, start_method="spawn")
+    assert out[1] == "left"
+    assert out[0][0] == "raised", out[0]
+    assert out[0][1] < 60.0
