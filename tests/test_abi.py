@@ -98,6 +98,58 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.kq_gemm_mxfp4(FAKE, FAKE, FAKE, FAKE, 1 << 31, 4, 64, FAKE, 0, None) == 1
 
 
+def test_block16_tiled_and_weight_entries_check_on_the_host(lib):
+    """The block-16, tiled-scale and weight-side entry points reject bad
+    shapes, null and misaligned pointers before any CUDA call."""
+    for f in (lib.kq_quantize16_tiled, lib.kq_quantize_weight16, lib.kq_quantize_weight16_tiled,
+              lib.kq_quantize_tiled, lib.kq_quantize_weight_tiled):
+        assert f(FAKE, 4, 48, FAKE, FAKE, FAKE, None) == 1           # d not a multiple of 32
+        assert f(FAKE, -1, 64, FAKE, FAKE, FAKE, None) == 1
+        assert f(None, 4, 64, FAKE, FAKE, FAKE, None) == 1
+        assert f(FAKE, 4, 64, None, FAKE, FAKE, None) == 1
+        assert f(FAKE + 8, 4, 64, FAKE, FAKE, FAKE, None) == 1       # x not 16-B aligned
+        assert f(FAKE, 4, 64, FAKE, FAKE + 4, FAKE, None) == 1       # q not 16-B aligned
+        assert f(None, 0, 64, None, None, None, None) == 0            # empty: nothing to do
+    assert lib.kq_quantize16_tiled(FAKE, 4, 64, FAKE, FAKE, FAKE + 4, None) == 1       # tiled: 16-B
+    assert lib.kq_quantize_weight16_tiled(FAKE, 4, 64, FAKE, FAKE, FAKE + 4, None) == 1
+    assert lib.kq_quantize_weight16(FAKE, 4, 64, FAKE, FAKE, FAKE + 1, None) == 1      # 2-B scales
+    assert lib.kq_fold_weight16(FAKE, 4, 64, FAKE, FAKE + 4, None) == 1
+    assert lib.kq_fold_weight16(FAKE, 4, 64, None, FAKE, None) == 1
+    assert lib.kq_scales16_tiled_bytes(0, 64) == 0 and lib.kq_scales16_tiled_bytes(4, 48) == 0
+    assert lib.kq_scales16_tiled_bytes(130, 544) == 2 * 9 * 512     # 34 scales: nine 4-columns
+    g16 = lib.kq_gemm_mxfp4_16_tiled
+    assert g16(FAKE, FAKE, FAKE, FAKE, 4, 4, 48, FAKE, 0, None) == 1             # K % 32
+    assert g16(FAKE, FAKE, FAKE, FAKE, 4, 4, 64, FAKE, 2, None) == 1             # dtype
+    assert g16(FAKE, FAKE + 4, FAKE, FAKE, 4, 4, 64, FAKE, 0, None) == 1         # tiled: 16-B
+    assert g16(FAKE, FAKE, None, FAKE, 4, 4, 64, FAKE, 0, None) == 1
+    assert g16(None, None, None, None, 0, 4, 64, None, 0, None) == 0
+
+
+def test_calibration_entries_check_on_the_host(lib):
+    grad = lib.kq_transform_params_grad
+    ws = lib.kq_transform_params_grad_workspace_bytes(16, 64)
+    assert ws > 256 and lib.kq_transform_params_grad_workspace_bytes(16, 48) == 0
+    assert grad(FAKE, FAKE, FAKE, 0, 64, FAKE, 0, 0.1, FAKE, FAKE, FAKE, ws, None) == 1   # M < 1
+    assert grad(FAKE, FAKE, FAKE, 16, 48, FAKE, 0, 0.1, FAKE, FAKE, FAKE, ws, None) == 1
+    assert grad(FAKE, FAKE, None, 16, 64, FAKE, 0, 0.1, FAKE, FAKE, FAKE, ws, None) == 1
+    assert grad(FAKE + 4, FAKE, FAKE, 16, 64, FAKE, 0, 0.1, FAKE, FAKE, FAKE, ws, None) == 1
+    assert grad(FAKE, FAKE, FAKE, 16, 64, FAKE, 0, float("nan"), FAKE, FAKE, FAKE, ws, None) == 1
+    assert grad(FAKE, FAKE, FAKE, 16, 64, FAKE, 0, 0.1, FAKE, FAKE, FAKE + 16, ws, None) == 1
+    res = lib.kq_residual
+    rws = lib.kq_residual_workspace_bytes()
+    assert res(FAKE, FAKE, 0, 1.0, FAKE, FAKE, FAKE, rws, None) == 1               # n < 1
+    assert res(FAKE, FAKE, 8, 1.0, FAKE, FAKE, FAKE, rws - 1, None) == 1           # workspace
+    assert res(FAKE, FAKE, 8, float("inf"), FAKE, FAKE, FAKE, rws, None) == 1
+    assert res(FAKE, FAKE, 8, 1.0, FAKE, FAKE + 4, FAKE, rws, None) == 1           # sumsq 8-B
+    adam = lib.kq_adam_step
+    assert adam(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1, 1e-2, 0.9, 0.999, 1e-8, None) == 1
+    assert adam(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 0, 1e-2, 0.9, 0.999, 1e-8, None) == 1   # step 0
+    assert adam(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 1, 1e-2, 1.0, 0.999, 1e-8, None) == 1   # beta1
+    assert adam(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 1, 1e-2, 0.9, 0.999, 0.0, None) == 1    # eps
+    assert adam(FAKE, FAKE, FAKE, FAKE, FAKE, 8, 1, float("nan"), 0.9, 0.999, 1e-8, None) == 1
+    assert adam(None, FAKE, FAKE, FAKE, FAKE, 8, 1, 1e-2, 0.9, 0.999, 1e-8, None) == 1
+
+
 def test_empty_input_needs_no_device(lib):
     assert lib.kq_quantize(None, 0, 64, None, None, None, None) == 0
     assert lib.kq_dequantize(None, None, 0, 64, None, None) == 0
