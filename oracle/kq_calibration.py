@@ -203,15 +203,3 @@ def calibrate(x64, w64, steps: int = 100, lr: float = 1e-2, params0=None):
         p, m, v = adam_step(p, g, m, v, t, lr)
     return p.astype(np.float32), history, (lam_a, lam_w)
 
-
-def smooth_output_loss(x64, w64, alpha: float = 0.5):
-    """Output loss of the per-channel-scaling baseline (SmoothQuant:
-    ``s_c = max|x_c|^alpha / max|w_c|^(1-alpha)``, ``X diag(s)^-1`` and
-    ``diag(s) W^T``), the comparator of the review's falsifier."""
-    ax = np.abs(x64).max(axis=0)
-    aw = np.abs(w64).max(axis=0)
-    s = np.where((ax > 0) & (aw > 0), ax ** alpha / np.maximum(aw, 1e-300) ** (1 - alpha), 1.0)
-    Aq = fake_quant(x64 / s[None, :])
-    Bq = fake_quant(w64 * s[None, :])
-    y_ref = x64 @ w64.T
-    return np.sum((Aq @ Bq.T - y_ref) ** 2) / np.sum(y_ref ** 2)
