@@ -35,6 +35,9 @@ UNIT = "GB/s"
 GEMM_METRIC = "W4A4 MXFP4 GEMM TFLOP/s on the transformed layer (M x d x d)"
 WORKLOAD = "stress"
 FALLBACK_HBM_GBS = 6650.0
+# Nominal B200 HBM3e bandwidth (8 TB/s): the spec figure, reported beside the
+# fraction of the measured copy bandwidth.
+SPEC_HBM_GBS = 8000.0
 CPU_SAMPLE_ROWS = 4096
 REFERENCE_BUDGET_S = 60.0
 E2E_WORKSPACE_BYTES = 64 << 20
@@ -113,23 +116,20 @@ def kernel_source_hash() -> str:
 
 
 def profiled_traffic(kernel_hash: str, name: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    """DRAM bytes per launch from a committed ncu record (JSON under
+    ``profiles/``), if it was taken on the current kernel sources (else
+    None)."""
     path = os.path.join(ROOT, "profiles", name)
     try:
-        text = open(path).read()
-    except OSError:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    kv = {}
-    for line in text.splitlines():
-        if ":" in line and line.startswith("- "):
-            k, v = line[2:].split(":", 1)
-            kv[k.strip()] = v.strip().strip("`")
-    if kv.get("kernel_source_hash") != kernel_hash:
+    if not isinstance(rec, dict) or rec.get("kernel_source_hash") != kernel_hash:
         return None
     try:
-        return float(kv["dram_bytes_per_full_launch"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_per_full_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
@@ -143,7 +143,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, local_rank: int, period_s: float = 0.002):
+    def __init__(self, local_rank: int, period_s: float = 0.0005):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
@@ -391,33 +391,122 @@ def per_config_table(dev, peak, stress=None):
             xs = [x] + [x.clone() for _ in range(ncopy - 1)]
             qs = [torch.empty((M, d // 2), dtype=torch.uint8, device=dev) for _ in range(ncopy)]
             ss = [torch.empty((M, d // 32), dtype=torch.uint8, device=dev) for _ in range(ncopy)]
+            seed = w.case_seed(name, di, 0)
+            p16 = torch.from_numpy(w.draw_params16(d, seed)).to(dev)
+            s16s = [torch.empty((M, d // 16), dtype=torch.uint8, device=dev) for _ in range(ncopy)]
+            tokens = w.TOKENS_PER_SAMPLE[name]
+            a_sh, a_sc = (t.to(dev) for t in w.draw_adaln(-(-M // tokens), d, seed))
             fams = {"kron": [lambda i=i: kq.quantize(xs[i], params, qs[i], ss[i]) for i in range(ncopy)],
                     "hadamard": [lambda i=i: kq.quantize_hadamard(xs[i], qs[i], ss[i])
                                  for i in range(ncopy)],
                     "smooth": [lambda i=i: kq.quantize_smooth(xs[i], inv_s, qs[i], ss[i])
-                               for i in range(ncopy)]}
+                               for i in range(ncopy)],
+                    "kron_tcgen05": [lambda i=i: kq.quantize(xs[i], params, qs[i], ss[i],
+                                                             impl=kq.KQ_IMPL_MMA)
+                                     for i in range(ncopy)],
+                    "kron16": [lambda i=i: kq.quantize16(xs[i], p16, qs[i], s16s[i])
+                               for i in range(ncopy)],
+                    "adaln": [lambda i=i: kq.quantize_adaln(xs[i], a_sh, a_sc, tokens, params, 1e-6,
+                                                            qs[i], ss[i])
+                              for i in range(ncopy)]}
             n = max(PER_CONFIG_BLOCK, ncopy)
             row = {"config": f"{name} d={d}", "M": M, "d": d, "algorithmic_bytes": alg,
                    "copies": ncopy, "launches_per_block": n,
                    "regime": ("latency-bound" if alg / (peak * 1e9) * 1e6 < LATENCY_BOUND_US
                               else "bandwidth")}
             for vname, fns in fams.items():
+                # The block-16 variant writes twice the scale bytes.
+                b = M * d * (2.0 + 0.5 + 1.0 / 16) if vname == "kron16" else alg
                 for f in fns:
                     f()
                 blocks = [block_us(fns, n) for _ in range(PER_CONFIG_BLOCKS)]
                 med = float(np.median(blocks))
                 row[vname] = {"us": med, "min_us": float(min(blocks)), "max_us": float(max(blocks)),
-                              "gbs": alg / (med * 1e-6) / 1e9,
-                              "frac": alg / (med * 1e-6) / 1e9 / peak,
+                              "gbs": b / (med * 1e-6) / 1e9,
+                              "frac": b / (med * 1e-6) / 1e9 / peak,
+                              "frac_spec": b / (med * 1e-6) / 1e9 / SPEC_HBM_GBS,
                               "single_launch_us": single_us(fns[0])}
             rows.append(row)
-            del xs, qs, ss
+            del xs, qs, ss, s16s
     del flush
     return {"blocks": PER_CONFIG_BLOCKS, "single_launch_reps": PER_CONFIG_REPS,
             "l2": "back to back over rotating copies of x (3x L2 of traffic between two uses "
                   "of a copy); single launch after overwriting a 2x L2 buffer",
             "host": "launches queued behind a device sleep: events time the device only",
             "latency_bound_below_us": LATENCY_BOUND_US, "rows": rows}
+
+
+# The W4A4 layer at DiT shapes (M tokens x N out x K in): the square layer
+# of the stress input, PixArt-Sigma's MLP up-projection and FLUX.1's.
+LAYER_SHAPES = (("stress square", 16384, 12288, 12288), ("pixart_sigma mlp", 8192, 4608, 1152),
+                ("flux_schnell mlp", 4608, 12288, 3072))
+
+
+def layer_table(dev, stream, steps: int):
+    """Per shape: the block-scaled product alone (TFLOP/s and its fraction of
+    the FP4 peak) and the layer as a user runs it (activations quantized on
+    the fly into the tiled scale layout, then the product), beside the same
+    product in bf16 through torch.matmul."""
+    import torch
+    import workloads as w
+    import w4a4_post_quantization_b200 as kq
+    fp4_peak, fp4_src = measured_fp4_peak()
+    out = {"peak_tflops": fp4_peak, "peak_source": fp4_src, "kernel": gemm_kernel_name(),
+           "out": "bf16", "steps": steps, "rows": []}
+    for label, M, N, K in LAYER_SHAPES:
+        seed = 4242 + K
+        p = torch.from_numpy(w.draw_params(K, seed)).to(dev)
+        wt = w.device_randn_bf16((N, K), seed + 7, dev)
+        xa = w.device_randn_bf16((M, K), seed + 11, dev)
+        qw, sw = kq.quantize_weight_tiled(wt, p)
+        qa, sa = kq.quantize_tiled(xa, p)
+        c = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        flops = 2.0 * M * N * K
+        ms_g, _ = time_steps(lambda: kq.gemm_mxfp4_tiled(qa, sa, qw, sw, out=c,
+                                                         out_dtype=torch.bfloat16),
+                             steps, 3, stream)
+
+        def layer():
+            kq.quantize_tiled(xa, p, qa, sa)
+            kq.gemm_mxfp4_tiled(qa, sa, qw, sw, out=c, out_dtype=torch.bfloat16)
+        ms_l, _ = time_steps(layer, steps, 3, stream)
+        ms_b, _ = time_steps(lambda: torch.matmul(xa, wt.t(), out=c), steps, 3, stream)
+        tf = flops / (ms_g * 1e-3) / 1e12
+        out["rows"].append({"layer": label, "shape_mnk": [M, N, K], "gemm_ms": ms_g,
+                            "gemm_tflops": tf, "gemm_frac": tf / fp4_peak,
+                            "layer_ms": ms_l, "layer_tflops": flops / (ms_l * 1e-3) / 1e12,
+                            "bf16_matmul_ms": ms_b, "layer_speedup_over_bf16": ms_b / ms_l})
+        del qw, sw, qa, sa, c, wt, xa
+    return out
+
+
+CONFIG_LABELS = {"tiny d=1152": "C0", "pixart_sigma d=1152": "C1a", "pixart_sigma d=4608": "C1b",
+                 "sana d=2240": "C2a", "sana d=5600": "C2b", "flux_schnell d=3072": "C3a",
+                 "flux_schnell d=12288": "C3b", "stress d=12288": "C4"}
+SUMMARY_COLS = ("kron", "hadamard", "smooth", "kron_tcgen05", "kron16", "adaln")
+
+
+def compact_summary(variants):
+    """The headline figures of the variants, rounded, in a few hundred
+    characters (the end of the line): fraction of the measured HBM peak per
+    config and quantizer (back to back), the per-config microseconds of
+    kq_quantize, and the layer's fraction of the FP4 peak per shape."""
+    summ = {}
+    pc = variants.get("per_config")
+    if pc:
+        summ["per_config_cols"] = list(SUMMARY_COLS)
+        summ["frac_of_measured_hbm"] = {
+            CONFIG_LABELS.get(r["config"], r["config"]):
+                [round(r[c]["frac"], 3) if c in r else None for c in SUMMARY_COLS]
+            for r in pc["rows"]}
+        summ["kron_us"] = {CONFIG_LABELS.get(r["config"], r["config"]): round(r["kron"]["us"], 1)
+                           for r in pc["rows"]}
+    lt = variants.get("layers")
+    if lt:
+        summ["gemm_frac_of_fp4"] = {r["layer"]: round(r["gemm_frac"], 3) for r in lt["rows"]}
+        summ["layer_speedup_over_bf16"] = {r["layer"]: round(r["layer_speedup_over_bf16"], 2)
+                                           for r in lt["rows"]}
+    return summ
 
 
 # --------------------------------------------------------------- GPU leg
@@ -622,29 +711,12 @@ def run_gpu(args):
             "d2d_copy_gbs": 2 * x.numel() * 2 / (ms_max_c * 1e-3) / 1e9,
         })
         del buf
-        # The layer the codes feed: C = Q(x T) Q(W T^-T)^T with a square
-        # synthetic weight (d x d), bf16 output, block-scaled tcgen05 GEMM.
-        W = w.device_randn_bf16((d, d), case.seed + 7, dev)
-        qw, sw = kq.quantize_weight_tiled(W, params)
-        del W
-        qt, st_ = kq.quantize_tiled(x, params)
-        cg = torch.empty((M, d), dtype=torch.bfloat16, device=dev)
-        g_steps = max(3, min(args.steps, 40))
-        ms_g, _ = time_steps(
-            lambda: kq.gemm_mxfp4_tiled(qt, st_, qw, sw, out=cg, out_dtype=torch.bfloat16),
-            g_steps, 3, stream)
-        ms_max_g = max_over_ranks(ms_g, dev)
-        fp4_peak, fp4_src = measured_fp4_peak()
-        tflops = 2.0 * M * d * d / (ms_max_g * 1e-3) / 1e12
-        variants["w4a4_gemm"] = {
-            "shape_mnk": [M, d, d], "out": "bf16", "steps": g_steps, "ms": ms_max_g,
-            "tflops": tflops, "peak_tflops": fp4_peak, "peak_source": fp4_src,
-            "frac": tflops / fp4_peak,
-            "kernel": gemm_kernel_name()}
-        del qw, sw, cg, qt, st_
         if world == 1 and args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"]:
             variants["per_config"] = per_config_table(dev, measured_peak()[0],
                                                       (x, params, inv_s))
+            # The layer the codes feed, C = Q(x T) Q(W T^-T)^T, on the block-
+            # scaled tensor cores at three DiT shapes.
+            variants["layers"] = layer_table(dev, stream, max(3, min(args.steps, 40)))
 
     # End to end through the public API: pinned host x in, pinned host codes
     # and scales out, streamed through a device workspace (kq_quantize_host).
@@ -689,7 +761,7 @@ def run_gpu(args):
             "frac": per_launch_gbs / peak, "peak_source": peak_src,
             # The capture is of one full-size stress launch: other row counts
             # get no traffic figure.
-            "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.md")
+            "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.json")
                         if args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"] else None),
             "algorithmic_bytes_per_launch": alg_bytes,
             "kernel": {"kron": "panel_kernel<kron, mx4>", "kron16": "panel_kernel<kron16, mx4>",
@@ -734,10 +806,15 @@ def run_gpu(args):
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3,
                            **({"gemm_shape_mnk": gemm_mnk} if args.op == "gemm" else {})),
             "hbm_frac": value / world / peak if args.op != "gemm" else None,
+            "hbm_frac_spec": value / world / SPEC_HBM_GBS if args.op != "gemm" else None,
+            "spec_hbm_gbs": SPEC_HBM_GBS,
             # Absolute throughput beside the bytes: elements of x per second, all ranks.
             "elements_per_s": (M * d * world / (ms_max * 1e-3)) if args.op != "gemm" else None,
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
             "gpu_launches": args.steps, "variants": variants,
+            # Last, so that the end of the line carries the headline figures.
+            "summary": dict(compact_summary(variants), hbm_frac=round(value / world / peak, 4),
+                            hbm_frac_spec=round(value / world / SPEC_HBM_GBS, 4)),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

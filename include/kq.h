@@ -93,8 +93,12 @@ int kq_quantize_hadamard(const uint16_t* x, int64_t M, int64_t d,
 int kq_quantize_smooth(const uint16_t* x, int64_t M, int64_t d, const float* inv_s,
                        uint8_t* q_packed, uint8_t* scales, void* stream);
 
-/* y = x T in float32 (the kq_quantize transform without quantization), for
- * parity checks. */
+/* y = x T in float32: the Kronecker block transform of kq_quantize (KroQuant
+ * review, "What carries the argument": K^(j) = G1 (x) ... (x) G5 per 32-channel
+ * block; "Circularity Check", Eq. 1: the activations are multiplied on the
+ * right, A T), stopped before the quantizer, for parity checks.  Same
+ * arguments and layout as kq_quantize; y: [M][d] float32, 16-byte aligned,
+ * written by the call.  KQ_ERR_INVALID for the same argument errors. */
 int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float* params,
                  float* y, void* stream);
 
@@ -279,8 +283,13 @@ int kq_scales_to_tiled(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* 
 int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,
                          float* x, void* stream);
 
-/* y = E2M1(code) * 2^(scale - 127) in float32 (exact; scale byte 0xFF gives
- * NaN, results beyond the float32 range give +-Inf). */
+/* y = E2M1(code) * 2^(scale - 127) in float32: the value MXFP4 codes and
+ * their shared E8M0 scale stand for (the OCP Microscaling definition the
+ * review cites for MXFP4: E2M1 elements with magnitudes {0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6}, an E8M0 power-of-two scale per 32 elements).  Exact; scale byte
+ * 0xFF gives NaN, results beyond the float32 range give +-Inf.  q_packed
+ * [M][d/2] and scales [M][d/32] as kq_quantize writes them; y [M][d] float32,
+ * 16-byte aligned. */
 int kq_dequantize(const uint8_t* q_packed, const uint8_t* scales, int64_t M, int64_t d,
                   float* y, void* stream);
 
@@ -319,7 +328,14 @@ size_t kq_quantize_host_workspace_bytes(int64_t d, int64_t rows_per_chunk);
  * through a KQ_STATIC_STAGING_BYTES staging area that is part of the library
  * itself.  Each GPU on which that area is loaded keeps it until the process
  * exits.  The first call on a device looks up the area's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * (cudaGetSymbolAddress) and keeps it for later calls; make that first call
+ * before any stream capture.  The kept address belongs to the device's
+ * primary context: it is valid only while that context lives, so a process
+ * that resets the device (cudaDeviceReset) must not call this entry point
+ * again.  The call uses the current device; `stream` must belong to it.
+ * The call is asynchronous, like kq_quantize_host: it returns once the work
+ * is queued, and `stream` completes when the last outputs have reached host
+ * memory; the host buffers must stay valid until then.
  * All calls share the one area and the last call's data stays in it: calls
  * that overlap on the GPU (on different streams, or from several host
  * threads) race and must be serialised by the caller.  KQ_ERR_INVALID for

@@ -24,6 +24,8 @@ import numpy as np
 from oracle import kq_oracle as o
 
 TOL = 1e-5
+# E2M1 rounding boundaries: midpoints of neighbouring grid magnitudes.
+MIDPOINTS = (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0)
 
 
 def unpack(q: np.ndarray) -> np.ndarray:
@@ -107,10 +109,67 @@ def check_mx4(q_gpu, s_gpu, y64, cond, tol: float = TOL, strict_zero_sign: bool 
                   float(vb[tuple(i)])) for i in idx]))
     differ = c_gpu != codes_ref
     zero_sign = differ & ((c_gpu & 7) == 0) & ((codes_ref & 7) == 0)
+    # The literal reading of the rule, counted beside the componentwise one:
+    # a differing scale byte whose block maximum is not within tol relative
+    # of a power of two, and a differing code (against the oracle's code
+    # under the scale the GPU chose) whose scaled value is not within tol
+    # relative of an E2M1 midpoint.
+    amax_ref = blk.max(axis=2)
+    with np.errstate(divide="ignore"):
+        p2 = np.ldexp(1.0, np.round(np.log2(np.where(amax_ref > 0, amax_ref, 1.0))).astype(np.int64))
+    scale_lit = np.abs(amax_ref - p2) <= tol * p2
+    s_diff = s_int != s_ref
+    code_diff = (c_gpu != ref_same_scale) & ~(((c_gpu & 7) == 0) & ((ref_same_scale & 7) == 0))
+    av = np.abs(v)
+    near_mid = np.zeros(av.shape, dtype=bool)
+    for mid in MIDPOINTS:
+        near_mid |= np.abs(av - mid) <= tol * mid
     return {
-        "scale_exempt": int((s_int != s_ref).sum()),
+        "scale_exempt": int(s_diff.sum()),
         "code_exempt": int((differ & ~zero_sign).sum()),
         "zero_sign_exempt": int(zero_sign.sum()),
+        "scale_outside_literal": int((s_diff & ~scale_lit).sum()),
+        "code_differs_under_gpu_scale": int(code_diff.sum()),
+        "code_outside_literal": int((code_diff & ~near_mid).sum()),
         "blocks": int(M * nb),
         "elements": int(M * d),
     }
+
+
+def relative_outside(y_gpu: np.ndarray, y64: np.ndarray, tol: float = TOL) -> int:
+    """Entries with |y_gpu - y64| > tol |y64|: those that pass the
+    componentwise bound only because their terms cancel."""
+    err = np.abs(np.asarray(y_gpu, dtype=np.float64) - y64)
+    return int((err > tol * np.abs(y64)).sum())
+
+
+def merge_stats(total: dict, part: dict) -> dict:
+    """Adds one chunk's counts to a running total (worst ratios take the max)."""
+    for k, v in part.items():
+        if k.startswith("worst"):
+            total[k] = max(total.get(k, 0.0), v)
+        else:
+            total[k] = total.get(k, 0) + v
+    return total
+
+
+def check_chunk(job):
+    """Compares one row chunk of the GPU's outputs with the oracle; runs in a
+    spawned worker (numpy only).  ``job`` = (kind, x_bits, aux, outputs):
+    kind "kron" (aux = params; outputs q, s, y), "hadamard" (q, s) or
+    "smooth" (aux = inv_s; q, s).  Returns the chunk's counts."""
+    kind, bits, aux, out = job
+    x64 = o.bf16_bits_to_float64(bits)
+    if kind == "kron":
+        y64 = o.transform(x64, aux)
+        cond = o.abs_transform(x64, aux)
+        st = {"worst_transform_ratio": check_transform(out["y"], y64, cond),
+              "transform_outside_relative": relative_outside(out["y"], y64)}
+        st.update(check_mx4(out["q"], out["s"], y64, cond))
+    elif kind == "hadamard":
+        y64 = o.transform_hadamard(x64)
+        st = check_mx4(out["q"], out["s"], y64, o.abs_transform_hadamard(x64))
+    else:
+        y64 = o.transform_smooth(x64, aux)
+        st = check_mx4(out["q"], out["s"], y64, np.zeros_like(y64), strict_zero_sign=True)
+    return st

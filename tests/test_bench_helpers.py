@@ -1,43 +1,55 @@
 """Host-side helpers of bench.py (CPU): the DRAM-traffic lookup in a committed
-ncu summary, which must answer only for the kernel source it was taken on,
-and the name of the product kernel the library's switches select."""
+ncu record, which must answer only for the kernel source it was taken on,
+the name of the product kernel the library's switches select, and the
+compact summary at the end of the line."""
+import json
 import os
 
 import bench
 
 
-def _summary(tmp_path, text):
+def _record(tmp_path, rec):
     d = tmp_path / "profiles"
     d.mkdir()
-    (d / "t.md").write_text(text)
+    (d / "t.json").write_text(json.dumps(rec))
     return str(tmp_path)
 
 
 def test_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
-    root = _summary(tmp_path, "# x\n\n- kernel_source_hash: `abc123`\n"
-                              "- dram_bytes_per_full_launch: `1000`\n")
+    root = _record(tmp_path, {"kernel_source_hash": "abc123", "dram_bytes_per_full_launch": 1000})
     monkeypatch.setattr(bench, "ROOT", root)
-    assert bench.profiled_traffic("abc123", "t.md") == 1000.0
-    assert bench.profiled_traffic("def456", "t.md") is None      # kernel changed since
-    assert bench.profiled_traffic("abc123", "missing.md") is None
+    assert bench.profiled_traffic("abc123", "t.json") == 1000.0
+    assert bench.profiled_traffic("def456", "t.json") is None      # kernel changed since
+    assert bench.profiled_traffic("abc123", "missing.json") is None
 
 
 def test_traffic_needs_both_keys(tmp_path, monkeypatch):
-    root = _summary(tmp_path, "- kernel_source_hash: `abc123`\n")
+    root = _record(tmp_path, {"kernel_source_hash": "abc123"})
     monkeypatch.setattr(bench, "ROOT", root)
-    assert bench.profiled_traffic("abc123", "t.md") is None
+    assert bench.profiled_traffic("abc123", "t.json") is None
 
 
-def test_committed_traffic_profile_parses():
-    """The committed summary names a hash and a byte count; whether the hash
+def test_committed_traffic_record_parses():
+    """The committed record names a hash and a byte count; whether the hash
     is the current one decides only whether the bench reports it."""
-    path = os.path.join(bench.ROOT, "profiles", "kq_quantize_stress_traffic.md")
-    text = open(path).read()
-    assert "- kernel_source_hash: `" in text
-    assert "- dram_bytes_per_full_launch: `" in text
-    h = [l for l in text.splitlines() if l.startswith("- kernel_source_hash:")][0]
-    hval = h.split(":", 1)[1].strip().strip("`")
-    assert bench.profiled_traffic(hval, "kq_quantize_stress_traffic.md") > 4e8
+    path = os.path.join(bench.ROOT, "profiles", "kq_quantize_stress_traffic.json")
+    rec = json.load(open(path))
+    assert bench.profiled_traffic(rec["kernel_source_hash"], "kq_quantize_stress_traffic.json") > 4e8
+    assert "ncu" in rec["command"]
+
+
+def test_compact_summary_is_short_and_complete():
+    cfgs = list(bench.CONFIG_LABELS)
+    row = lambda c: dict({"config": c}, **{k: {"frac": 0.123456, "us": 12.3456}
+                                           for k in bench.SUMMARY_COLS})
+    variants = {"per_config": {"rows": [row(c) for c in cfgs]},
+                "layers": {"rows": [{"layer": l[0], "gemm_frac": 0.7654321,
+                                     "layer_speedup_over_bf16": 2.3456}
+                                    for l in bench.LAYER_SHAPES]}}
+    summ = bench.compact_summary(variants)
+    assert set(summ["frac_of_measured_hbm"]) == set(bench.CONFIG_LABELS.values())
+    assert summ["frac_of_measured_hbm"]["C4"] == [0.123] * len(bench.SUMMARY_COLS)
+    assert len(json.dumps(summ)) < 1200
 
 
 def test_gemm_kernel_name_follows_the_library_switches(monkeypatch):

@@ -5,7 +5,7 @@ import pytest
 
 import workloads as w
 from oracle import kq_oracle as o
-from tests.parity import check_mx4, check_transform
+from tests.parity import check_mx4, check_transform, relative_outside
 
 
 @pytest.fixture(scope="module")
@@ -67,3 +67,38 @@ def test_transform_error_beyond_tolerance_fails(case):
     bad[2, 5] += 2e-5 * cond[2, 5]
     with pytest.raises(AssertionError):
         check_transform(bad, y64, cond)
+
+
+def test_literal_band_counts():
+    """A code that differs where its scaled value sits on an E2M1 midpoint is
+    inside the literal band; one that differs only because the componentwise
+    band is wide (cancelling terms) is counted outside it; so is a scale byte
+    that differs away from a power of two."""
+    y = np.zeros((1, 64))
+    y[0, 0] = 4.0            # block 0: scale 2^0, unit steps
+    y[0, 1] = 1.25           # an exact midpoint between 1 and 1.5
+    y[0, 2] = 2.2            # far from every midpoint
+    y[0, 32] = 3.0           # block 1: amax 3, away from a power of two
+    codes, s = o.mxfp4_quantize(y)
+    cond = np.zeros_like(y)
+    cond[0, 1] = 1.0
+    cond[0, 2] = 1e5         # a cancelling sum: wide componentwise band
+    cond[0, 32] = 1e5
+    got = codes.copy()
+    got[0, 1] = 3            # 1.5 instead of the even 1.0: on the midpoint
+    got[0, 2] = 5            # 3.0 instead of 2.0: allowed by the wide band only
+    st = check_mx4(o.pack_codes(got), s, y, cond)
+    assert st["code_differs_under_gpu_scale"] == 2
+    assert st["code_outside_literal"] == 1
+    s2 = s.copy()
+    s2[0, 1] += 1            # block 1 at twice the scale: 3.0 is coded as 3 (code 5), not 6
+    got = codes.copy()
+    got[0, 32] = 5
+    st = check_mx4(o.pack_codes(got), s2, y, cond)
+    assert st["scale_exempt"] == 1 and st["scale_outside_literal"] == 1
+
+
+def test_relative_outside_counts_cancelling_entries():
+    y64 = np.array([[1.0, 1e-9, -2.0]])
+    y_gpu = y64 + np.array([[1e-7, 1e-7, 0.0]])
+    assert relative_outside(y_gpu, y64) == 1

@@ -642,7 +642,10 @@ def quantize_host_static(x: torch.Tensor, params: torch.Tensor, q: torch.Tensor,
     """quantize_host without a workspace, for callers that cannot allocate
     device memory: the rows pass through a 16 MiB staging area built into the
     library.  Calls that overlap on the GPU share that area and must be
-    serialised.  Runs on ``stream`` (default: the current CUDA stream)."""
+    serialised.  Runs on ``stream`` (default: the current CUDA stream of
+    ``params``' device), with that device made current for the call.  The
+    call is asynchronous: the host outputs are complete once the stream has
+    reached this point, and every host buffer must stay alive until then."""
     _host_tensor(x, torch.bfloat16, "x")
     M, d = _shape(x)
     _host_tensor(q, torch.uint8, "q")
@@ -650,9 +653,12 @@ def quantize_host_static(x: torch.Tensor, params: torch.Tensor, q: torch.Tensor,
     if tuple(q.shape) != (M, d // 2) or tuple(scales.shape) != (M, d // 32):
         raise ValueError("output shapes must be [M, d/2] and [M, d/32]")
     _params(params, d)
-    st = stream if stream is not None else _stream(params.device)
-    rc = lib().kq_quantize_host_static(x.data_ptr(), M, d, params.data_ptr(), q.data_ptr(),
-                                       scales.data_ptr(), st)
+    # The staging area is looked up on the current device: make it the one
+    # that holds the parameters and the stream.
+    with torch.cuda.device(params.device):
+        st = stream if stream is not None else _stream(params.device)
+        rc = lib().kq_quantize_host_static(x.data_ptr(), M, d, params.data_ptr(),
+                                           q.data_ptr(), scales.data_ptr(), st)
     _check("kq_quantize_host_static", rc)
     return q, scales
 
