@@ -693,7 +693,8 @@ def run_gpu(args):
         ms_max_c = max_over_ranks(ms_c, dev)
         impls = {}
         for name, code in (("panel", kq.KQ_IMPL_PANEL), ("tma_flat", kq.KQ_IMPL_TMA),
-                           ("direct", kq.KQ_IMPL_DIRECT), ("tcgen05_dense_k", kq.KQ_IMPL_MMA)):
+                           ("direct", kq.KQ_IMPL_DIRECT), ("tcgen05_dense_k", kq.KQ_IMPL_MMA),
+                           ("warp_shuffle", kq.KQ_IMPL_WARP)):
             ms_i, _ = time_steps(lambda: kq.quantize(x, params, q, s, impl=code), args.steps,
                                  args.warmup, stream)
             impls[name] = alg_bytes / (max_over_ranks(ms_i, dev) * 1e-3) / 1e9

@@ -65,7 +65,7 @@ enum {
     KQ_IMPL_AUTO = 0,       /* what kq_quantize uses */
     KQ_IMPL_TMA = 1,        /* TMA-staged, persistent, thread per 32-block */
     KQ_IMPL_DIRECT = 2,     /* direct 32-byte global loads, thread per 32-block */
-    KQ_IMPL_WARP = 3,       /* one 32-block per warp, shuffle butterfly */
+    KQ_IMPL_WARP = 3,       /* one 32-block per warp, lane = element, shuffle butterfly */
     KQ_IMPL_PANEL = 4,      /* TMA-staged column panels, factors in registers */
     KQ_IMPL_MMA = 5         /* tensor cores: dense K^(j) as three bf16 terms, tcgen05.mma */
 };

@@ -128,6 +128,8 @@ def check_mx4(q_gpu, s_gpu, y64, cond, tol: float = TOL, strict_zero_sign: bool 
         "scale_exempt": int(s_diff.sum()),
         "code_exempt": int((differ & ~zero_sign).sum()),
         "zero_sign_exempt": int(zero_sign.sum()),
+        # a zero code of the other sign where the exact value is not zero
+        "zero_sign_outside_literal": int((zero_sign & (y64 != 0)).sum()),
         "scale_outside_literal": int((s_diff & ~scale_lit).sum()),
         "code_differs_under_gpu_scale": int(code_diff.sum()),
         "code_outside_literal": int((code_diff & ~near_mid).sum()),

@@ -110,7 +110,7 @@ def test_full_size_sampled_rows(key):
 
 
 IMPLS = {"panel": kq.KQ_IMPL_PANEL, "tma": kq.KQ_IMPL_TMA, "direct": kq.KQ_IMPL_DIRECT,
-         "mma": kq.KQ_IMPL_MMA}
+         "mma": kq.KQ_IMPL_MMA, "warp": kq.KQ_IMPL_WARP}
 
 
 @pytest.mark.parametrize("impl", sorted(IMPLS))

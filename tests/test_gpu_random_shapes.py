@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 
 kq = pytest.importorskip("w4a4_post_quantization_b200")
 
-IMPLS = [kq.KQ_IMPL_AUTO, kq.KQ_IMPL_PANEL, kq.KQ_IMPL_TMA, kq.KQ_IMPL_DIRECT, kq.KQ_IMPL_MMA]
+IMPLS = [kq.KQ_IMPL_AUTO, kq.KQ_IMPL_PANEL, kq.KQ_IMPL_TMA, kq.KQ_IMPL_DIRECT, kq.KQ_IMPL_MMA,
+         kq.KQ_IMPL_WARP]
 
 
 def _shapes():

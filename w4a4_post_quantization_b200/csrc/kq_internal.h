@@ -78,5 +78,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Launchers defined in other translation units.
 int launch_mma_kron(const uint16_t* x, int64_t M, int64_t d, const float* params, uint8_t* q,
                     uint8_t* scales, float* y, cudaStream_t st);
+int launch_warp_kron(const uint16_t* x, int64_t M, int64_t d, const float* params, uint8_t* q,
+                     uint8_t* scales, cudaStream_t st);
 
 }  // namespace kq

@@ -884,6 +884,10 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
       else
         impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
     }
+    if (impl == KQ_IMPL_WARP) {
+      if (kXf != kXfKron || kOut != kOutMx4) return KQ_ERR_INVALID;
+      return launch_warp_kron(x, M, d, aux, q, scales, st);
+    }
     if (impl == KQ_IMPL_MMA) {
       if (kXf != kXfKron) return KQ_ERR_INVALID;
       return launch_mma_kron(x, M, d, aux, kOut == kOutMx4 ? q : nullptr,
