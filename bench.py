@@ -143,7 +143,7 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, local_rank: int, period_s: float = 0.0005):
+    def __init__(self, local_rank: int, period_s: float = 0.0):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()

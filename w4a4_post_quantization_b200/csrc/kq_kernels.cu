@@ -412,6 +412,41 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   const int cpp = gridDim.x / a.panels;           // CTAs per panel
   const int k0 = blockIdx.x / a.panels;           // first row tile of this CTA
   const int n_local = k0 < a.row_tiles ? (a.row_tiles - k0 + cpp - 1) / cpp : 0;
+  const bool active = tid < a.W * a.R;
+  const int j = panel * a.W + (tid % a.W);
+
+  // Parameters first.  Each consumer thread reads its unit's parameters (or
+  // reciprocal scales) into registers, and the whole CTA waits until they
+  // have arrived before the producer issues the first tile loads: issued
+  // behind the tiles' DRAM traffic, these few L2 reads were measured to
+  // return several microseconds late, and every thread's coefficients wait
+  // for them.
+  constexpr int kUnitParams = kron5(kXf) ? 15 : kron4(kXf) ? 24 : kXf == kXfSmooth ? 32 : 0;
+  float prm[kUnitParams > 0 ? kUnitParams : 1];
+  float arrived = 0.0f;
+  if constexpr (kUnitParams > 0) {
+    if (tid < kCons && active) {
+      const float* src = a.aux + (int64_t)j * kUnitParams;
+      if constexpr (kXf == kXfSmooth) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const float4 v = reinterpret_cast<const float4*>(src)[t];
+          prm[4 * t] = v.x;
+          prm[4 * t + 1] = v.y;
+          prm[4 * t + 2] = v.z;
+          prm[4 * t + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int t = 0; t < kUnitParams; ++t) prm[t] = src[t];
+      }
+      // A value that depends on every load: the barrier below then waits
+      // for them.
+#pragma unroll
+      for (int t = 0; t < kUnitParams; ++t) arrived += prm[t];
+    }
+  }
+  asm volatile("bar.sync 2, %0;" ::"r"(Cfg::kThreads), "f"(arrived) : "memory");
 
   if (tid >= kCons) {
     if (tid == kCons) {
@@ -445,9 +480,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     return;
   }
 
-  const bool active = tid < a.W * a.R;
   const int rho = tid / a.W;
-  const int j = panel * a.W + (tid % a.W);
   using SD = std::conditional_t<kron4(kXf), ShearDiag16, ShearDiag>;
   using PF = std::conditional_t<kron4(kXf), PlainFactors16, PlainFactors>;
   SD sd;
@@ -456,8 +489,7 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
   if constexpr (kron5(kXf) || kron4(kXf)) {
     // Parameters per thread unit: 5 x 3 for a 32-block, 2 x 4 x 3 for a pair
     // of 16-blocks.
-    constexpr int kUnitParams = kron5(kXf) ? 15 : 24;
-    const float* p = a.aux + (int64_t)j * kUnitParams;
+    const float* p = prm;
     if constexpr (kron5(kXf)) {
       if (active) plain = load_shear_diag<kXf == kXfKronInvT>(sd, p) ? 0 : 1;
     } else {
@@ -476,13 +508,8 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
     }
   } else if constexpr (kXf == kXfSmooth) {
     if (active) {
-      const float4* v = reinterpret_cast<const float4*>(a.aux + (int64_t)j * kBlock);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const float4 x = v[t];
-        sd.delta[2 * t] = pack2(x.x, x.y);
-        sd.delta[2 * t + 1] = pack2(x.z, x.w);
-      }
+      for (int t = 0; t < 16; ++t) sd.delta[t] = pack2(prm[2 * t], prm[2 * t + 1]);
     }
   }
   if (plain)
