@@ -133,7 +133,7 @@ __device__ __forceinline__ bool load_shear_in(ShearIn& f, const float* p) {
   for (int k = 0; k < kFactors; ++k) {
     double g00, g01, g10, g11;
     factor_entries<false>(p, k, g00, g01, g10, g11);
-    const double ra = g10 / g11, rb = g01 / g00;
+    const double ra = g10 * recip_d(g11), rb = g01 * recip_d(g00);
     ok = ok && (g00 != 0.0) && (g11 != 0.0) && isfinite(ra) && isfinite(rb);
     growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
     r10[k] = (float)ra;

@@ -169,6 +169,20 @@ __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v
   return r;
 }
 
+// 1/v in double to about 2^-46 relative: the float32 reciprocal refined by
+// one Newton step in double (the seed's relative error e becomes e^2), in
+// place of a full double division; the exact division where v lies outside
+// the range in which the float seed is a normal number.  The coefficients
+// built from it are rounded to float32, so the result matches the exact
+// quotient's except within 2^-46 of a float32 rounding boundary.
+__device__ __forceinline__ double recip_d(double v) {
+  const double av = fabs(v);
+  if (!(av > 0x1p-120 && av < 0x1p120)) return 1.0 / v;
+  const double r0 = static_cast<double>(__frcp_rn(static_cast<float>(v)));
+  const double e = __fma_rn(-v, r0, 1.0);
+  return __fma_rn(r0, e, r0);
+}
+
 // ------------------------------------------------------ block transforms
 // A 32-element block lives in u[16]; u[m] holds elements 2m (low) and 2m+1.
 //
@@ -224,7 +238,7 @@ __device__ __forceinline__ void kron_entry(float* entry, const float* p, bool in
 #pragma unroll
   for (int k = 0; k < kFactors; ++k) {
     const double a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
-    double g00 = b, g01 = c, g10 = a * b, g11 = __fma_rn(a, c, 1.0 / b);
+    double g00 = b, g01 = c, g10 = a * b, g11 = __fma_rn(a, c, recip_d(b));
     if (inverse) {
       const double t00 = g11, t01 = -g01, t10 = -g10, t11 = g00;
       g00 = t00; g01 = t01; g10 = t10; g11 = t11;
@@ -272,7 +286,7 @@ template <bool kInvT = false>
 __device__ __forceinline__ void factor_entries(const float* p, int k, double& g00, double& g01,
                                                double& g10, double& g11) {
   const double a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
-  const double e00 = b, e01 = c, e10 = a * b, e11 = __fma_rn(a, c, 1.0 / b);
+  const double e00 = b, e01 = c, e10 = a * b, e11 = __fma_rn(a, c, recip_d(b));
   if (kInvT) {
     g00 = e11;
     g01 = -e10;
@@ -302,8 +316,8 @@ __device__ __forceinline__ bool load_shear_diag(ShearDiag& f, const float* p) {
     factor_entries<kInvT>(p, k, a00, a01, a10, a11);
     g00[k] = a00;
     g11[k] = a11;
-    const double ra = kInvT ? a10 / a00 : static_cast<double>(p[3 * k + 0]);
-    const double rb = a01 / a11;
+    const double ra = kInvT ? a10 * recip_d(a00) : static_cast<double>(p[3 * k + 0]);
+    const double rb = a01 * recip_d(a11);
     ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
     growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
     r10[k] = (float)ra;
@@ -437,8 +451,8 @@ __device__ __forceinline__ bool load_shear_diag16(ShearDiag16& f, const float* p
       factor_entries<kInvT>(ph, k, a00, a01, a10, a11);
       g00[k] = a00;
       g11[k] = a11;
-      const double ra = kInvT ? a10 / a00 : static_cast<double>(ph[3 * k + 0]);
-      const double rb = a01 / a11;
+      const double ra = kInvT ? a10 * recip_d(a00) : static_cast<double>(ph[3 * k + 0]);
+      const double rb = a01 * recip_d(a11);
       ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
       growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
       r10[k] = (float)ra;

@@ -102,7 +102,7 @@ __device__ __forceinline__ void build_factor_table(float* gtab, const float* par
     g[0] = static_cast<float>(b);
     g[1] = static_cast<float>(c);
     g[2] = static_cast<float>(a * b);
-    g[3] = static_cast<float>(__fma_rn(a, c, 1.0 / b));
+    g[3] = static_cast<float>(__fma_rn(a, c, recip_d(b)));
   }
 }
 

@@ -50,7 +50,7 @@ __global__ void __launch_bounds__(kWarpThreads)
 #pragma unroll
       for (int k = 0; k < kFactors; ++k) {
         const double a = p[3 * k], b = p[3 * k + 1], c = p[3 * k + 2];
-        const double g00 = b, g01 = c, g10 = a * b, g11 = __fma_rn(a, c, 1.0 / b);
+        const double g00 = b, g01 = c, g10 = a * b, g11 = __fma_rn(a, c, recip_d(b));
         const int bit = (lane >> (4 - k)) & 1;
         c_own[k] = static_cast<float>(bit ? g11 : g00);
         c_other[k] = static_cast<float>(bit ? g01 : g10);
