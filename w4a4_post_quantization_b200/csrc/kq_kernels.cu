@@ -763,19 +763,38 @@ double panel_shape(int nb, int cons, int rpt, int sms, int* W_out, int* R_out) {
 using PanelV0 = PanelCfg<12, 2, 1>;
 using PanelV1 = PanelCfg<8, 2, 1>;
 using PanelV2 = PanelCfg<15, 1, 1>;
-constexpr int kDefaultPanel = 0;
+using PanelV4 = PanelCfg<16, 1, 1>;
 constexpr int kPanelMaxStages = 6;
-
-// KQ_PANEL_VARIANT selects another compiled shape (read at every call; for
-// tuning measurements only).
-int panel_variant() {
-  const char* e = getenv("KQ_PANEL_VARIANT");
-  return e ? atoi(e) : kDefaultPanel;
-}
 
 template <class Cfg>
 double panel_use(int nb, int sms, int* W, int* R) {
   return panel_shape(nb, Cfg::kCons, Cfg::kRpt, sms * Cfg::kMinBlocks, W, R);
+}
+
+// Launch shape by the work per SM.  Measured on B200, back to back over cold
+// copies of x, microseconds per launch with 12 x 2 / 15 x 1 / 16 x 1
+// consumer warps x rows: 8192 x 1152 9.24 / 8.69 / 8.61; 8192 x 4608
+// 22.6 / 22.0 / 22.1; 4096 x 2240 9.23 / 8.60 / 8.27; 4096 x 5600
+// 16.2 / 15.6 / 15.5; 4608 x 3072 11.3 / 11.3 / 10.9; 4608 x 12288
+// 30.5 / 30.1 / 50.9; 16384 x 12288 87.1 / 88.6 / 152.  Up to about 24K
+// blocks per SM the one-row shapes win (a shorter chain per tile, more
+// warps); above that two rows per thread do.  16 x 1 is taken for rows of up
+// to 256 blocks (it runs the 384-block rows on 128-block panels, measured
+// slow) where its panel keeps 90 % of the 512 threads busy, 15 x 1 where its
+// panel keeps three quarters of 480 busy; else the two-row shape, whose 384
+// threads divide more widths.
+int auto_panel_variant(int64_t M, int nb, int sms) {
+  int W = 0, R = 0;
+  if (M * nb > static_cast<int64_t>(sms) * 24576) return 0;
+  if (nb <= 256 && panel_use<PanelV4>(nb, sms, &W, &R) >= 0.9) return 4;
+  return panel_use<PanelV2>(nb, sms, &W, &R) >= 0.75 ? 2 : 0;
+}
+
+// KQ_PANEL_VARIANT (0, 1, 2 or 4) forces one compiled shape (read at every
+// call; for tuning measurements only).
+int panel_variant(int64_t M, int nb, int sms) {
+  const char* e = getenv("KQ_PANEL_VARIANT");
+  return e ? atoi(e) : auto_panel_variant(M, nb, sms);
 }
 
 template <int kXf, int kOut, class Cfg>
@@ -840,12 +859,15 @@ template <int kXf, int kOut>
 int launch_panel(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q,
                  uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev,
                  int32_t scale_tiles_k = 0) {
-  switch (panel_variant()) {
+  switch (panel_variant(M, static_cast<int>(d / kBlock), di.sms)) {
     case 1:
       return launch_panel_cfg<kXf, kOut, PanelV1>(x, M, d, aux, q, scales, y, st, di, dev,
                                                   scale_tiles_k);
     case 2:
       return launch_panel_cfg<kXf, kOut, PanelV2>(x, M, d, aux, q, scales, y, st, di, dev,
+                                                  scale_tiles_k);
+    case 4:
+      return launch_panel_cfg<kXf, kOut, PanelV4>(x, M, d, aux, q, scales, y, st, di, dev,
                                                   scale_tiles_k);
     default:
       return launch_panel_cfg<kXf, kOut, PanelV0>(x, M, d, aux, q, scales, y, st, di, dev,
@@ -853,11 +875,12 @@ int launch_panel(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint
   }
 }
 
-bool panel_fits(int nb, int sms) {
+bool panel_fits(int64_t M, int nb, int sms) {
   int W = 0, R = 0;
-  switch (panel_variant()) {
+  switch (panel_variant(M, nb, sms)) {
     case 1: return panel_use<PanelV1>(nb, sms, &W, &R) >= 0.75;
     case 2: return panel_use<PanelV2>(nb, sms, &W, &R) >= 0.75;
+    case 4: return panel_use<PanelV4>(nb, sms, &W, &R) >= 0.75;
     default: return panel_use<PanelV0>(nb, sms, &W, &R) >= 0.75;
   }
 }
@@ -906,7 +929,7 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
     return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
   } else {
     if (impl == KQ_IMPL_AUTO) {
-      if (nb <= 65535 && panel_fits(static_cast<int>(nb), di->sms) && M < (int64_t(1) << 30))
+      if (nb <= 65535 && panel_fits(M, static_cast<int>(nb), di->sms) && M < (int64_t(1) << 30))
         impl = KQ_IMPL_PANEL;
       else
         impl = nb <= kTmaMaxNb ? KQ_IMPL_TMA : KQ_IMPL_DIRECT;
