@@ -129,8 +129,12 @@ def inverse_transform(y64: np.ndarray, params: np.ndarray) -> np.ndarray:
 
 
 def transform_hadamard(x64: np.ndarray) -> np.ndarray:
-    H = hadamard_block()
-    return _apply_blocks(x64, lambda j: H)
+    """``y = x H_32 / sqrt(32)`` per block: the +-1 Sylvester sums first, then
+    one division by ``sqrt(32)``.  For bf16 input the sums are exact in
+    float64 (when a block's exponents span less than 40 binades), so a sum
+    that cancels is exactly zero, and each output carries one rounding."""
+    H = scipy.linalg.hadamard(BLOCK).astype(np.float64)
+    return _apply_blocks(x64, lambda j: H) / math.sqrt(BLOCK)
 
 
 def transform_smooth(x64: np.ndarray, inv_s: np.ndarray) -> np.ndarray:

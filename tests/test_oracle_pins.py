@@ -623,3 +623,14 @@ def test_block16_product_brute_force():
         for n in range(N):
             assert C[m, n] == sum(val(ca[m, k], sa[m, k // 16]) * val(cb[n, k], sb[n, k // 16])
                                   for k in range(K))
+
+
+def test_hadamard_cancelling_sum_is_exactly_zero():
+    """x H_32 / sqrt(32) with x = e_0 + e_1: H[0][c] + H[1][c] is 2 for even c
+    and 0 for odd c (Sylvester order: row 1 alternates signs), so the odd
+    outputs are exact zeros and the even ones 2 / sqrt(32)."""
+    x = np.zeros((1, 32))
+    x[0, 0] = x[0, 1] = 1.0
+    y = o.transform_hadamard(x)[0]
+    assert (y[1::2] == 0.0).all()
+    np.testing.assert_allclose(y[0::2], 2.0 / math.sqrt(32.0), rtol=1e-15)
