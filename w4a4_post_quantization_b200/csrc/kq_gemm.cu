@@ -558,7 +558,8 @@ bool encode_codes_map(CUtensorMap* map, const uint8_t* q, int64_t rows, int64_t 
 // epilogue thread holds its row's 256 outputs as 128 registers of bf16
 // pairs, so the accumulator is released as soon as it has been read and the
 // MMAs of tile i + 1 start while tile i's four boxes still leave by TMA.
-constexpr int kStagingBytes = kOutBoxBytes;              // 16 KiB: one box
+constexpr int kStagingBytes = kOutBoxBytes;              // 16 KiB: four 4 KiB boxes
+constexpr int kPBoxRows = 32;                            // rows of one output box
 constexpr int kPThreads = 32 * 6;
 
 // Stages of the persistent kernel per scale mode: four of 51 KiB with scales
@@ -729,28 +730,28 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    // Rows of TMEM lane quarter (warp mod 4); the tile leaves through the
-    // staging box as 128-byte-swizzled boxes of 128 rows x 128 bytes (row
-    // r's 16-byte chunk c at c ^ (r mod 8)), one box at a time.
+    // Rows of TMEM lane quarter (warp mod 4).  Each warp sends its 32 rows
+    // on its own: a 4 KiB slice of the staging area holds one box of 32 rows
+    // x 128 bytes (128-byte swizzle: row r's 16-byte chunk c at c ^ (r mod
+    // 8)), stored by the warp's first lane, so the four warps' stores
+    // proceed side by side with no barrier between them.
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
     const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
-    const bool issuer = warp == 2 && lane == 0;
-    uint8_t* srow = staging + r * 128;
-    auto epi_sync = [] { asm volatile("bar.sync 3, %0;" ::"r"(4 * 32) : "memory"); };
-    // Box `col` of the tile from the staging box: wait until the previous
-    // store has read it, fill it, store it.
+    uint8_t* wstage = staging + quarter * (kPBoxRows * 128);
+    uint8_t* srow = wstage + lane * 128;
+    // Box `col` of this warp's rows: wait until its previous store has read
+    // the slice, fill it, store it.
     auto store_box = [&](int m0, int col, const uint32_t (&wv)[32]) {
-      if (issuer) bulk_wait_read_0();
-      epi_sync();
+      if (lane == 0) bulk_wait_read_0();
+      __syncwarp();
 #pragma unroll
       for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(srow + 16 * (c ^ (r & 7))) =
+        *reinterpret_cast<uint4*>(srow + 16 * (c ^ (lane & 7))) =
             make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
       fence_proxy_async_smem();
-      epi_sync();
-      if (issuer) {
-        tma_store_2d(&cmap, staging, col, m0);
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(&cmap, wstage, col, m0 + quarter * kPBoxRows);
         bulk_commit();
       }
     };
@@ -766,18 +767,25 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       tmem_fence_after();
       if (a.out_bf16) {
+        // The row's 256 columns in two rounds of four loads with one wait
+        // each, so that the loads' latencies overlap and the accumulator is
+        // released sooner.
+        constexpr int kLdPerWait = 4;
         uint32_t h[kBN / 2];                      // the row as bf16 pairs
 #pragma unroll
-        for (int v = 0; v < kBN / 32; ++v) {
-          uint32_t x[32];
-          tmem_ld32(taddr + 32 * v, x);
+        for (int v0 = 0; v0 < kBN / 32; v0 += kLdPerWait) {
+          uint32_t x[kLdPerWait][32];
+#pragma unroll
+          for (int u = 0; u < kLdPerWait; ++u) tmem_ld32(taddr + 32 * (v0 + u), x[u]);
           tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const __nv_bfloat162 p =
-                __floats2bfloat162_rn(__uint_as_float(x[2 * q]), __uint_as_float(x[2 * q + 1]));
-            h[16 * v + q] = *reinterpret_cast<const uint32_t*>(&p);
-          }
+          for (int u = 0; u < kLdPerWait; ++u)
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+              const __nv_bfloat162 p = __floats2bfloat162_rn(__uint_as_float(x[u][2 * q]),
+                                                             __uint_as_float(x[u][2 * q + 1]));
+              h[16 * (v0 + u) + q] = *reinterpret_cast<const uint32_t*>(&p);
+            }
         }
         // Every column has been read: the MMAs of the next tile may start.
         tmem_fence_before();
@@ -807,7 +815,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
       }
     }
-    if (issuer) bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
     tmem_fence_before();
   }
   asm volatile("bar.sync 2, %0;" ::"r"(5 * 32) : "memory");
@@ -1217,8 +1226,13 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   if (a.tma_store) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(N) * esize};
+    // Output boxes of 128 bytes x 128 rows (per-tile kernel), the pair
+    // kernel's rows, or 32 rows (persistent kernels: one box per warp).
+    const bool pers = scale_block == 16 ? persistent_gemm16()
+                                        : (!pair && tiled && persistent_gemm());
     const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esize),
-                               static_cast<cuuint32_t>(pair ? kQBoxRows : kBM)};
+                               static_cast<cuuint32_t>(pair ? kQBoxRows
+                                                            : pers ? kPBoxRows : kBM)};
     const cuuint32_t estr[2] = {1, 1};
     if (tensor_map_encoder()(&cmap,
                              esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
