@@ -78,8 +78,11 @@ static_assert(kSfCol0 + kStages * (kSfColsA + kSfColsB) <= kTmemCols, "TMEM colu
 // kind::mxf4), K-major, N = 256, E8M0 scales, M = 128, dense K = 64.  The
 // scale-factor ids (byte of the 32-bit TMEM word holding the first scale of
 // the MMA's K range) go in bits 29-30 (A) and 4-5 (B).
-constexpr uint32_t kIdescMxf4 = (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (1u << 23) |
-                                (uint32_t(kBM >> 4) << 24);
+__host__ __device__ constexpr uint32_t idesc_mxf4(int bn) {
+  return (1u << 7) | (1u << 10) | (uint32_t(bn >> 3) << 17) | (1u << 23) |
+         (uint32_t(kBM >> 4) << 24);
+}
+constexpr uint32_t kIdescMxf4 = idesc_mxf4(kBN);
 
 struct GemmArgs {
   int32_t M, N, K;
@@ -207,37 +210,41 @@ __device__ __forceinline__ void mma_mxf4_b16(uint32_t tmem_d, uint64_t adesc, ui
 // the descriptors' start address steps by 2 (x16 B).  Scales per 32: two per
 // row and MMA, bytes 0-1 or 2-3 of the chunk's 32-bit word (scale-factor
 // id); scales per 16: four per row and MMA, chunk kk, the whole word.
-template <int kSfMode, int kN>
+// kBNt: the tile's N (B rows), 256 or 128; B's scales take 4 TMEM columns
+// per 128-row group and chunk.
+template <int kSfMode, int kN, int kBNt = kBN>
 __device__ __forceinline__ void ktile_mmas(uint32_t tmem, uint64_t adesc, uint64_t bdesc,
                                            uint32_t tsfa, uint32_t tsfb, int kt) {
+  constexpr uint32_t kId = idesc_mxf4(kBNt);
+  constexpr int kBCols = 4 * (kBNt / 128);
 #pragma unroll
   for (int kk = 0; kk < kN; ++kk) {
     if constexpr (kSfMode == kSfTiled16) {
-      mma_mxf4_b16(tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdescMxf4, tsfa + 4 * kk,
-                   tsfb + 8 * kk, (kt | kk) != 0);
+      mma_mxf4_b16(tmem, adesc + 2 * kk, bdesc + 2 * kk, kId, tsfa + 4 * kk,
+                   tsfb + kBCols * kk, (kt | kk) != 0);
     } else {
       const uint32_t sf_id = 2u * (kk & 1);
-      const uint32_t idesc = kIdescMxf4 | (sf_id << 29) | (sf_id << 4);
+      const uint32_t idesc = kId | (sf_id << 29) | (sf_id << 4);
       mma_mxf4(tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, tsfa + 4 * (kk >> 1),
-               tsfb + 8 * (kk >> 1), (kt | kk) != 0);
+               tsfb + kBCols * (kk >> 1), (kt | kk) != 0);
     }
   }
 }
 
 // A k-tile's MMAs; a last k-tile that ends inside the stage issues none
 // over its zero fill (K elements left: rem).
-template <int kSfMode>
+template <int kSfMode, int kBNt = kBN>
 __device__ __forceinline__ void issue_ktile(uint32_t tmem, uint64_t adesc, uint64_t bdesc,
                                             uint32_t tsfa, uint32_t tsfb, int kt, int rem) {
   static_assert(kBK / kMmaK == 4, "four MMAs per k-tile");
   if (rem > 3 * kMmaK)
-    ktile_mmas<kSfMode, 4>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+    ktile_mmas<kSfMode, 4, kBNt>(tmem, adesc, bdesc, tsfa, tsfb, kt);
   else if (rem > 2 * kMmaK)
-    ktile_mmas<kSfMode, 3>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+    ktile_mmas<kSfMode, 3, kBNt>(tmem, adesc, bdesc, tsfa, tsfb, kt);
   else if (rem > kMmaK)
-    ktile_mmas<kSfMode, 2>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+    ktile_mmas<kSfMode, 2, kBNt>(tmem, adesc, bdesc, tsfa, tsfb, kt);
   else
-    ktile_mmas<kSfMode, 1>(tmem, adesc, bdesc, tsfa, tsfb, kt);
+    ktile_mmas<kSfMode, 1, kBNt>(tmem, adesc, bdesc, tsfa, tsfb, kt);
 }
 
 template <int kSfMode>
@@ -562,41 +569,58 @@ constexpr int kStagingBytes = kOutBoxBytes;              // 16 KiB: four 4 KiB b
 constexpr int kPBoxRows = 32;                            // rows of one output box
 constexpr int kPThreads = 32 * 6;
 
-// Stages of the persistent kernel per scale mode: four of 51 KiB with scales
-// per 32, three of 54 KiB with scales per 16 (four do not fit beside the
-// staging box).
-template <int kSfMode>
-struct PGeom : StageGeom<kSfMode> {
-  static constexpr int kStages = kSfMode == kSfTiled16 ? 3 : 4;
-  static constexpr int kSmem = 1024 + kStages * StageGeom<kSfMode>::kStage + kStagingBytes +
-                               (2 * kStages + 4) * 8 + 16;
+// Geometry of the persistent kernel per scale mode and tile width N:
+//   N = 256, one accumulator of 256 TMEM columns: four stages of 51 KiB with
+//   scales per 32, three of 54 KiB with scales per 16 (four do not fit
+//   beside the staging box);
+//   N = 128 (scales per 32), two accumulators of 128 columns, so that the
+//   MMAs of tile i + 1 run while the epilogue drains tile i: six stages of
+//   34 KiB.
+template <int kSfMode, int kBNt = kBN>
+struct PGeom {
+  static constexpr int kChunks = kSfMode == kSfTiled16 ? 4 : kChunksPerStage;
+  static constexpr int kGroups = kBNt / 128;               // 128-row groups of B
+  static constexpr int kBTile = kBNt * kBKBytes;
+  static constexpr int kSfa = kChunks * kSfChunk;
+  static constexpr int kSfb = kChunks * kGroups * kSfChunk;
+  static constexpr int kStage = kATile + kBTile + kSfa + kSfb;
+  static constexpr int kColsA = 4 * kChunks;
+  static constexpr int kColsB = 4 * kGroups * kChunks;
+  static constexpr int kAcc = kBNt == 128 ? 2 : 1;         // accumulators
+  static constexpr int kSfCol0 = kAcc * kBNt;
+  static constexpr int kStages = kBNt == 128 ? 6 : (kSfMode == kSfTiled16 ? 3 : 4);
+  static constexpr int kSmem = 1024 + kStages * kStage + kStagingBytes +
+                               (2 * kStages + 2 * kAcc + 2) * 8 + 16;
+  static_assert(kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
   static_assert(kSmem <= 232448, "shared memory");
-  static_assert(kSfCol0 + kStages * (StageGeom<kSfMode>::kColsA + StageGeom<kSfMode>::kColsB) <=
-                    kTmemCols, "TMEM columns");
+  static_assert(kSfCol0 + kStages * (kColsA + kColsB) <= kTmemCols, "TMEM columns");
 };
 
-__device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, int& n0) {
+// Tile t of the banded order (bands of kBandN column tiles, the row tile
+// changing fastest), for tiles of bn columns.
+__device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, int& n0,
+                                            int bn = kBN) {
   const int band = t / (kBandN * a.m_tiles);
   const int r = t - band * kBandN * a.m_tiles;
   const int width = min(kBandN, a.n_tiles - band * kBandN);
   m0 = (r / width) * kBM;
-  n0 = (band * kBandN + r % width) * kBN;
+  n0 = (band * kBandN + r % width) * bn;
 }
 
-template <int kSfMode>
+template <int kSfMode, int kBNt>
 __global__ void __launch_bounds__(kPThreads, 1)
     gemm_mxf4_persistent(const __grid_constant__ CUtensorMap amap,
                          const __grid_constant__ CUtensorMap bmap,
                          const __grid_constant__ CUtensorMap cmap, const GemmArgs a) {
-  using P = PGeom<kSfMode>;
+  using P = PGeom<kSfMode, kBNt>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = smem_raw + ((1024u - (smem_addr(smem_raw) & 1023u)) & 1023u);
   uint8_t* staging = base + P::kStages * P::kStage;
   uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
   uint64_t* empty = full + P::kStages;
   uint64_t* acc_full = empty + P::kStages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* mma_done = acc_empty + 1;
+  uint64_t* acc_empty = acc_full + P::kAcc;
+  uint64_t* mma_done = acc_empty + P::kAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n_tiles_total = a.m_tiles * a.n_tiles;
@@ -604,7 +628,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   for (int st = 0; st < P::kStages; ++st)
     for (int i = tid; i < (P::kSfa + P::kSfb) / 16; i += blockDim.x)
-      reinterpret_cast<uint4*>(base + st * P::kStage + kATile + kBTile)[i] =
+      reinterpret_cast<uint4*>(base + st * P::kStage + kATile + P::kBTile)[i] =
           make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (tid == 0) {
@@ -612,8 +636,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(&full[st], 1);
       mbar_init(&empty[st], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);                 // one arrival per epilogue warp
+    for (int b = 0; b < P::kAcc; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);           // one arrival per epilogue warp
+    }
     mbar_init(mma_done, 1);
     fence_mbar_init();
   }
@@ -636,8 +662,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x) {
         int m0, n0;
-        tile_origin(a, t, m0, n0);
-        const int b_tiles = min(kBN / 128, a.sf_tiles_n - n0 / 128);
+        tile_origin(a, t, m0, n0, kBNt);
+        const int b_tiles = min(P::kGroups, a.sf_tiles_n - n0 / 128);
         for (int kt = 0; kt < nk; ++kt, ++g) {
           if (g >= P::kStages && !mbar_wait(&empty[s], phase)) {
             ok = false;
@@ -645,9 +671,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
           }
           uint8_t* stg = base + s * P::kStage;
           const int avail = min(P::kChunks, a.sf_tiles_k - P::kChunks * kt);
-          mbar_arrive_expect_tx(&full[s], kATile + kBTile +
+          mbar_arrive_expect_tx(&full[s], kATile + P::kBTile +
                                               (uint32_t)(avail * (1 + b_tiles)) * kSfChunk);
-          uint8_t* sfa = stg + kATile + kBTile;
+          uint8_t* sfa = stg + kATile + P::kBTile;
           bulk_load(sfa, a.sa + ((int64_t)(m0 / 128) * a.sf_tiles_k + P::kChunks * kt) *
                                   kSfChunk, avail * kSfChunk, &full[s]);
           for (int gb = 0; gb < b_tiles; ++gb)
@@ -677,6 +703,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (lane == 0) {
       int s = 0, i = 0;
       uint32_t phase = 0;
+      uint32_t tacc = tmem_base;             // the accumulator of the current tile
       bool ok = true;
       // One k-tile: its stage's scales into TMEM, its MMAs (all four in a
       // full k-tile, so that path has no branch; a last k-tile that ends
@@ -685,24 +712,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (!mbar_wait(&full[s], phase)) return false;
         tmem_fence_after();
         const uint8_t* stg = base + s * P::kStage;
-        const uint8_t* sfa = stg + kATile + kBTile;
+        const uint8_t* sfa = stg + kATile + P::kBTile;
         const uint8_t* sfb = sfa + P::kSfa;
-        const uint32_t tsfa = tmem_base + kSfCol0 + s * (P::kColsA + P::kColsB);
+        const uint32_t tsfa = tmem_base + P::kSfCol0 + s * (P::kColsA + P::kColsB);
         const uint32_t tsfb = tsfa + P::kColsA;
 #pragma unroll
         for (int c = 0; c < P::kChunks; ++c) {
           tmem_cp_32x128b_x4(tsfa + 4 * c, smem_desc_rows16(smem_addr(sfa + c * kSfChunk)));
 #pragma unroll
-          for (int gb = 0; gb < kBN / 128; ++gb)
-            tmem_cp_32x128b_x4(tsfb + 8 * c + 4 * gb,
+          for (int gb = 0; gb < P::kGroups; ++gb)
+            tmem_cp_32x128b_x4(tsfb + 4 * P::kGroups * c + 4 * gb,
                                smem_desc_rows16(smem_addr(sfb + (P::kChunks * gb + c) * kSfChunk)));
         }
         const uint64_t adesc = smem_desc_sw128(smem_addr(stg));
         const uint64_t bdesc = smem_desc_sw128(smem_addr(stg + kATile));
         if constexpr (decltype(full_tile)::value)
-          ktile_mmas<kSfMode, kBK / kMmaK>(tmem_base, adesc, bdesc, tsfa, tsfb, kt);
+          ktile_mmas<kSfMode, kBK / kMmaK, kBNt>(tacc, adesc, bdesc, tsfa, tsfb, kt);
         else
-          issue_ktile<kSfMode>(tmem_base, adesc, bdesc, tsfa, tsfb, kt, a.K - kt * kBK);
+          issue_ktile<kSfMode, kBNt>(tacc, adesc, bdesc, tsfa, tsfb, kt, a.K - kt * kBK);
         mma_commit(&empty[s]);
         if (++s == P::kStages) {
           s = 0;
@@ -711,17 +738,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
         return true;
       };
       for (int t = blockIdx.x; t < n_tiles_total && ok; t += gridDim.x, ++i) {
-        // The accumulator is free once the epilogue has read tile i - 1.
-        if (i >= 1 && !mbar_wait(acc_empty, (i - 1) & 1)) {
+        // Accumulator i mod kAcc is free once the epilogue has read tile
+        // i - kAcc.
+        const int b = i % P::kAcc;
+        if (i >= P::kAcc && !mbar_wait(&acc_empty[b], ((i / P::kAcc) - 1) & 1)) {
           ok = false;
           break;
         }
+        tacc = tmem_base + b * kBNt;
         tmem_fence_after();
         const int nk_full = a.K % kBK == 0 ? nk : nk - 1;
         int kt = 0;
         for (; ok && kt < nk_full; ++kt) ok = ktile(kt, std::true_type{});
         if (ok && kt < nk) ok = ktile(kt, std::false_type{});
-        if (ok) mma_commit(acc_full);
+        if (ok) mma_commit(&acc_full[b]);
       }
       if (!ok) atomicOr(a.err, kErrConsumerWait);
       mma_commit(mma_done);
@@ -758,9 +788,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
     int i = 0;
     for (int t = blockIdx.x; t < n_tiles_total; t += gridDim.x, ++i) {
       int m0, n0;
-      tile_origin(a, t, m0, n0);
+      tile_origin(a, t, m0, n0, kBNt);
+      const int b = i % P::kAcc;
+      const uint32_t tb = taddr + b * kBNt;
       // One AND-barrier makes a timeout the same for the four warps.
-      const bool got = mbar_wait(acc_full, i & 1);
+      const bool got = mbar_wait(&acc_full[b], (i / P::kAcc) & 1);
       if (!bar_and(3, 4 * 32, got)) {
         if (lane == 0) atomicOr(a.err, kErrConsumerWait);
         break;
@@ -771,12 +803,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // each, so that the loads' latencies overlap and the accumulator is
         // released sooner.
         constexpr int kLdPerWait = 4;
-        uint32_t h[kBN / 2];                      // the row as bf16 pairs
+        uint32_t h[kBNt / 2];                     // the row as bf16 pairs
 #pragma unroll
-        for (int v0 = 0; v0 < kBN / 32; v0 += kLdPerWait) {
+        for (int v0 = 0; v0 < kBNt / 32; v0 += kLdPerWait) {
           uint32_t x[kLdPerWait][32];
 #pragma unroll
-          for (int u = 0; u < kLdPerWait; ++u) tmem_ld32(taddr + 32 * (v0 + u), x[u]);
+          for (int u = 0; u < kLdPerWait; ++u) tmem_ld32(tb + 32 * (v0 + u), x[u]);
           tmem_wait_ld();
 #pragma unroll
           for (int u = 0; u < kLdPerWait; ++u)
@@ -790,28 +822,28 @@ __global__ void __launch_bounds__(kPThreads, 1)
         // Every column has been read: the MMAs of the next tile may start.
         tmem_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(acc_empty);
+        if (lane == 0) mbar_arrive(&acc_empty[b]);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
+        for (int ob = 0; ob < kBNt / 64; ++ob) {
           uint32_t wv[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) wv[k] = h[32 * b + k];
-          store_box(m0, n0 + 64 * b, wv);
+          for (int k = 0; k < 32; ++k) wv[k] = h[32 * ob + k];
+          store_box(m0, n0 + 64 * ob, wv);
         }
       } else {
         // float32: eight boxes of 32 columns, each read out of TMEM as it
         // goes; the accumulator is released after the last read.
 #pragma unroll 1
-        for (int b = 0; b < kBN / 32; ++b) {
+        for (int ob = 0; ob < kBNt / 32; ++ob) {
           uint32_t x[32];
-          tmem_ld32(taddr + 32 * b, x);
+          tmem_ld32(tb + 32 * ob, x);
           tmem_wait_ld();
-          if (b == kBN / 32 - 1) {
+          if (ob == kBNt / 32 - 1) {
             tmem_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
           }
-          store_box(m0, n0 + 32 * b, x);
+          store_box(m0, n0 + 32 * ob, x);
         }
       }
     }
@@ -1120,6 +1152,17 @@ bool persistent_gemm16() {
   return e ? atoi(e) != 0 : true;
 }
 
+// Tile width of the persistent kernel with scales per 32: 256 columns with
+// one accumulator, or 128 with two (the next tile's MMAs overlap the
+// epilogue's drain, at twice the A traffic per flop).  KQ_GEMM_BN=128/256
+// forces either (measurements, tests).
+int gemm_tile_n(int64_t K) {
+  const char* e = getenv("KQ_GEMM_BN");
+  if (e) return atoi(e) == 128 ? 128 : 256;
+  (void)K;
+  return 256;
+}
+
 // The CTA-pair kernel for scales per 32 (KQ_GEMM_PAIR=1 selects it).
 bool pair_gemm() {
   const char* e = getenv("KQ_GEMM_PAIR");
@@ -1245,11 +1288,12 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   const dim3 grid(static_cast<unsigned>(a.m_tiles * a.n_tiles));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (scale_block == 16 && a.tma_store && persistent_gemm16()) {
-    rc = allow_smem<gemm_mxf4_persistent<kSfTiled16>>(PGeom<kSfTiled16>::kSmem, dev);
+    rc = allow_smem<gemm_mxf4_persistent<kSfTiled16, kBN>>(PGeom<kSfTiled16>::kSmem, dev);
     if (rc != KQ_OK) return rc;
     const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
-    cudaError_t le = launch_pdl(gemm_mxf4_persistent<kSfTiled16>, dim3(pgrid), dim3(kPThreads),
-                                PGeom<kSfTiled16>::kSmem, st, amap, bmap, cmap, a);
+    cudaError_t le = launch_pdl(gemm_mxf4_persistent<kSfTiled16, kBN>, dim3(pgrid),
+                                dim3(kPThreads), PGeom<kSfTiled16>::kSmem, st, amap, bmap, cmap,
+                                a);
     if (le != cudaSuccess) return record_cuda_error(le);
   } else if (scale_block == 16) {
     using G = StageGeom<kSfTiled16>;
@@ -1261,11 +1305,25 @@ int launch_gemm(const uint8_t* qa, const uint8_t* sa, const uint8_t* qb, const u
   } else if (pair) {
     return launch_gemm_pair(amap, qb, sa, sb, cmap, a, di, dev, st);
   } else if (tiled && a.tma_store && persistent_gemm()) {
-    rc = allow_smem<gemm_mxf4_persistent<kSfTiled>>(PGeom<kSfTiled>::kSmem, dev);
-    if (rc != KQ_OK) return rc;
-    const int pgrid = static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
-    cudaError_t le = launch_pdl(gemm_mxf4_persistent<kSfTiled>, dim3(pgrid), dim3(kPThreads),
-                                PGeom<kSfTiled>::kSmem, st, amap, bmap, cmap, a);
+    cudaError_t le;
+    if (gemm_tile_n(K) == 128) {
+      // Tiles of 128 columns with two accumulators.
+      a.n_tiles = static_cast<int32_t>((N + 127) / 128);
+      if (!encode_codes_map(&bmap, qb, N, K, 128)) return record_cuda_error(cudaErrorInvalidValue);
+      rc = allow_smem<gemm_mxf4_persistent<kSfTiled, 128>>(PGeom<kSfTiled, 128>::kSmem, dev);
+      if (rc != KQ_OK) return rc;
+      const int pgrid =
+          static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
+      le = launch_pdl(gemm_mxf4_persistent<kSfTiled, 128>, dim3(pgrid), dim3(kPThreads),
+                      PGeom<kSfTiled, 128>::kSmem, st, amap, bmap, cmap, a);
+    } else {
+      rc = allow_smem<gemm_mxf4_persistent<kSfTiled, kBN>>(PGeom<kSfTiled>::kSmem, dev);
+      if (rc != KQ_OK) return rc;
+      const int pgrid =
+          static_cast<int>(std::min<int64_t>((int64_t)a.m_tiles * a.n_tiles, di->sms));
+      le = launch_pdl(gemm_mxf4_persistent<kSfTiled, kBN>, dim3(pgrid), dim3(kPThreads),
+                      PGeom<kSfTiled>::kSmem, st, amap, bmap, cmap, a);
+    }
     if (le != cudaSuccess) return record_cuda_error(le);
   } else if (tiled) {
     // No scale warps: six warps.
