@@ -289,11 +289,13 @@ def run_reference(args):
 L2_BYTES = 126e6
 
 
-def _config(d, M, impl, block=32):
+def _config(d, M, impl, block=32, case=None):
     x_mb = M * d * 2 / 1e6
     return {
-        "workload": f"bandwidth stress: M={M} tokens x d={d} bf16, Student-t(3), "
-                    "0.5% outlier channels x100, learned Kronecker-LU block params",
+        "workload": (f"bandwidth stress: M={M} tokens x d={d} bf16, Student-t(3), "
+                     "0.5% outlier channels x100, learned Kronecker-LU block params"
+                     if case is None else
+                     f"{case} (seeded DiT-shaped stand-in): M={M} tokens x d={d} bf16"),
         "M": M, "d": d, "block": block,
         "format": f"MXFP4 (E2M1 codes + E8M0 scale per {block})",
         "impl": impl,
@@ -577,8 +579,15 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
 
-    M = args.rows or w.CONFIGS[WORKLOAD]["M"]
-    case = w.make_case(WORKLOAD, M=M, row0=shard_row0(rank, -(-M // w.ROW_CHUNK) * w.ROW_CHUNK))
+    if args.case:
+        # Another config's input (profiling): name:d_index, full size.
+        cname, cdi = args.case.split(":")
+        case = w.make_case(cname, int(cdi))
+        M = case.M
+    else:
+        M = args.rows or w.CONFIGS[WORKLOAD]["M"]
+        case = w.make_case(WORKLOAD, M=M,
+                           row0=shard_row0(rank, -(-M // w.ROW_CHUNK) * w.ROW_CHUNK))
     d = case.d
     x = case.x.to(dev)
     params = torch.from_numpy(case.params).to(dev)
@@ -595,7 +604,7 @@ def run_gpu(args):
         alg_bytes = bytes16
     # AdaLN modulation of the batch's samples (bf16 [B, d], read once per
     # CTA and sample: not counted in the algorithmic bytes).
-    tokens = w.TOKENS_PER_SAMPLE[WORKLOAD]
+    tokens = w.TOKENS_PER_SAMPLE[args.case.split(":")[0] if args.case else WORKLOAD]
     ada_shift, ada_scale = (t.to(dev) for t in w.draw_adaln(-(-M // tokens), d, case.seed))
 
     gemm_flops = 2.0 * M * d * d
@@ -731,7 +740,7 @@ def run_gpu(args):
             "d2d_copy_gbs": 2 * x.numel() * 2 / (ms_max_c * 1e-3) / 1e9,
         })
         del buf
-        if world == 1 and args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"]:
+        if world == 1 and args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"] and not args.case:
             variants["per_config"] = per_config_table(dev, measured_peak()[0],
                                                       (x, params, inv_s))
             # The layer the codes feed, C = Q(x T) Q(W T^-T)^T, on the block-
@@ -782,7 +791,8 @@ def run_gpu(args):
             # The capture is of one full-size stress launch: other row counts
             # get no traffic figure.
             "traffic": (profiled_traffic(khash, "kq_quantize_stress_traffic.json")
-                        if args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"] else None),
+                        if args.op == "kron" and M == w.CONFIGS[WORKLOAD]["M"] and not args.case
+                        else None),
             "algorithmic_bytes_per_launch": alg_bytes,
             "kernel": {"kron": "panel_kernel<kron, mx4>", "kron16": "panel_kernel<kron16, mx4>",
                        "gemm": gemm_kernel_name(),
@@ -820,7 +830,8 @@ def run_gpu(args):
             "config": dict(_config(d, M, {"kron": "panel", "gemm": "tcgen05 kind::mxf4", "kron16": "panel", "hadamard": "panel",
                                           "smooth": "panel", "kron_mma": "tcgen05 dense K",
                                           "adaln": "fused rows"}[args.op],
-                                   16 if args.op == "kron16" else 32), op=args.op,
+                                   16 if args.op == "kron16" else 32,
+                                   args.case or None), op=args.op,
                            launch=("cuda_graph: the K steps captured once, replayed once"
                                    if args.launch == "graph" else "eager: one call per step"), global_batch_rows=M * world,
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3,
@@ -978,6 +989,9 @@ def main(argv=None):
                     metavar="M,N,K",
                     help="with --op gemm: time this layer shape instead of the stress "
                          "input's square layer (profiling)")
+    ap.add_argument("--case", default="", metavar="NAME:D_INDEX",
+                    help="time the quantizer on another config's full-size input, e.g. "
+                         "flux_schnell:0 (profiling only)")
     ap.add_argument("--rows", type=int, default=0,
                     help="rows of the stress input per GPU (default: its 16384); "
                          "smaller values are for profiling captures only")
