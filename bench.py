@@ -445,14 +445,23 @@ LAYER_SHAPES = (("stress square", 16384, 12288, 12288), ("pixart_sigma mlp", 819
 
 
 def queued_ms(fn, n: int, stream, warmup: int = 3) -> float:
-    """Average device time of ``n`` back-to-back calls, queued behind a device
+    """Average device time of back-to-back calls, queued behind a device
     sleep so that the host's per-call cost (argument checks, the launch) does
-    not leave the GPU idle between short kernels; CUDA events on ``stream``."""
+    not leave the GPU idle between short kernels; CUDA events on ``stream``.
+    At least ``n`` calls and about 2 ms of work are timed, after a few
+    untimed calls queued behind the sleep that bring the clocks back up."""
     import torch
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    fn()
+    torch.cuda.synchronize()
+    est = max(time.perf_counter() - t0, 1e-6)
+    n = max(n, min(2000, int(2e-3 / est) + 1))
     torch.cuda._sleep(HOST_AHEAD_CYCLES)
+    for _ in range(max(warmup, n // 4)):
+        fn()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(n):

@@ -782,19 +782,22 @@ double panel_use(int nb, int sms, int* W, int* R) {
 // to 256 blocks (it runs the 384-block rows on 128-block panels, measured
 // slow) where its panel keeps 90 % of the 512 threads busy, 15 x 1 where its
 // panel keeps three quarters of 480 busy; else the two-row shape, whose 384
-// threads divide more widths.
-int auto_panel_variant(int64_t M, int nb, int sms) {
+// threads divide more widths.  The 16-element variant (two blocks of four
+// factors a thread, a heavier set-up) keeps the two-row shape at every size
+// (measured: the one-row shapes lose at 8192 x 4608, 4096 x 5600 and
+// 4608 x 3072).
+int auto_panel_variant(int64_t M, int nb, int sms, bool one_row_ok) {
   int W = 0, R = 0;
-  if (M * nb > static_cast<int64_t>(sms) * 24576) return 0;
+  if (!one_row_ok || M * nb > static_cast<int64_t>(sms) * 24576) return 0;
   if (nb <= 256 && panel_use<PanelV4>(nb, sms, &W, &R) >= 0.9) return 4;
   return panel_use<PanelV2>(nb, sms, &W, &R) >= 0.75 ? 2 : 0;
 }
 
 // KQ_PANEL_VARIANT (0, 1, 2 or 4) forces one compiled shape (read at every
 // call; for tuning measurements only).
-int panel_variant(int64_t M, int nb, int sms) {
+int panel_variant(int64_t M, int nb, int sms, bool one_row_ok = true) {
   const char* e = getenv("KQ_PANEL_VARIANT");
-  return e ? atoi(e) : auto_panel_variant(M, nb, sms);
+  return e ? atoi(e) : auto_panel_variant(M, nb, sms, one_row_ok);
 }
 
 template <int kXf, int kOut, class Cfg>
@@ -859,7 +862,7 @@ template <int kXf, int kOut>
 int launch_panel(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q,
                  uint8_t* scales, float* y, cudaStream_t st, const DeviceInfo& di, int dev,
                  int32_t scale_tiles_k = 0) {
-  switch (panel_variant(M, static_cast<int>(d / kBlock), di.sms)) {
+  switch (panel_variant(M, static_cast<int>(d / kBlock), di.sms, !kron4(kXf))) {
     case 1:
       return launch_panel_cfg<kXf, kOut, PanelV1>(x, M, d, aux, q, scales, y, st, di, dev,
                                                   scale_tiles_k);
