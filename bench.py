@@ -163,30 +163,49 @@ class ClockSampler:
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
         except Exception as e:            # no NVML on this host
             self.nvml, self.error = None, repr(e)
+        self._arm()
 
     def _run(self):
+        # Polls from construction on, so that the thread and NVML are warm
+        # when the timed region starts; keeps what it reads while recording.
         n = self.nvml
         while not self._stop.is_set():
             try:
-                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                mhz = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
                 mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for k, bit in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(k)
             except Exception as e:
                 self.error = repr(e)
                 return
+            if self._recording:
+                self.samples.append(mhz)
+                for k, bit in self.REASONS.items():
+                    if mask & bit:
+                        self.reasons.add(k)
             time.sleep(self.period)
 
-    def start(self):
+    def _arm(self):
+        self._recording = False
         if self.nvml is not None:
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
 
+    def start(self):
+        """Records from now on (call right before the timed region)."""
+        if self._thread is not None:
+            # A short interpreter switch interval lets the sampling thread
+            # run between the launching thread's calls during a timed
+            # region of a few milliseconds.
+            self._switch = sys.getswitchinterval()
+            sys.setswitchinterval(5e-5)
+            self._recording = True
+
     def stop(self):
         if self._thread is not None:
+            self._recording = False
             self._stop.set()
             self._thread.join()
+            if hasattr(self, "_switch"):
+                sys.setswitchinterval(self._switch)
         return {
             "sm_mhz": statistics.median(self.samples) if self.samples else None,
             "sm_max_mhz": self.max_mhz,
