@@ -182,10 +182,57 @@ __device__ __forceinline__ void diag_pairs(const float* p, f2 (&dl)[16]) {
 }
 
 // Writes alpha = (1 + scale) delta and beta = shift delta of this thread's
-// block for sample b into its slice of the modulation table: chunk c (four
-// channels) of alpha at tab[c * kAdaCons + tid], of beta at
+// block for one sample into its slice of the modulation table: chunk c
+// (four channels) of alpha at tab[c * kAdaCons + tid], of beta at
 // tab[(8 + c) * kAdaCons + tid], so that a warp's 16-byte reads of one chunk
-// are consecutive.  delta = 1 for the plain form.
+// are consecutive.  delta = 1 for the plain form.  p: the block's 15
+// parameters; vs / vc: the sample's shift / scale of the block, 32 bf16 each.
+template <int kForm>
+__device__ __forceinline__ void write_modulation(const float* p, const uint4 (&vs)[4],
+                                                 const uint4 (&vc)[4], int tid, float4* tab) {
+  f2 dl[16];
+  if (kForm == 0) {
+    diag_pairs(p, dl);
+  } else {
+#pragma unroll
+    for (int m = 0; m < 16; ++m) dl[m] = pack2(1.0f, 1.0f);
+  }
+  const f2 one2 = pack2(1.0f, 1.0f);
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t ws[4] = {vs[t].x, vs[t].y, vs[t].z, vs[t].w};
+    const uint32_t wc[4] = {vc[t].x, vc[t].y, vc[t].z, vc[t].w};
+    float al[8], be[8];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const f2 dd = dl[4 * t + w];
+      const f2 av = mul2(add2(bf16x2_to_f2(wc[w]), one2), dd);
+      const f2 bv = mul2(bf16x2_to_f2(ws[w]), dd);
+      unpack2(av, al[2 * w], al[2 * w + 1]);
+      unpack2(bv, be[2 * w], be[2 * w + 1]);
+    }
+    tab[(2 * t) * kAdaCons + tid] = make_float4(al[0], al[1], al[2], al[3]);
+    tab[(2 * t + 1) * kAdaCons + tid] = make_float4(al[4], al[5], al[6], al[7]);
+    tab[(8 + 2 * t) * kAdaCons + tid] = make_float4(be[0], be[1], be[2], be[3]);
+    tab[(8 + 2 * t + 1) * kAdaCons + tid] = make_float4(be[4], be[5], be[6], be[7]);
+  }
+}
+
+// The sample's shift and scale words of block j.
+__device__ __forceinline__ void read_modulation(const AdaArgs& a, int64_t b, int j, uint4 (&vs)[4],
+                                                uint4 (&vc)[4]) {
+  const uint4* ps = reinterpret_cast<const uint4*>(a.shift + (b * a.nb + j) * 16);
+  const uint4* pc = reinterpret_cast<const uint4*>(a.scale + (b * a.nb + j) * 16);
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    vs[t] = __ldg(ps + t);
+    vc[t] = __ldg(pc + t);
+  }
+}
+
+// The modulation of sample b, read from global memory at a sample change
+// (16 bytes of shift and of scale at a time: the main loop's registers are
+// tight).
 template <int kForm>
 __device__ __forceinline__ void load_modulation(const AdaArgs& a, int64_t b, int j, int tid,
                                                 float4* tab) {
@@ -241,7 +288,8 @@ template <int kOut, int kForm>
 __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMap* xmap,
                                               uint8_t* stages, uint64_t* full, uint64_t* statbar,
                                               float4* slots, float4* modtab, int tid,
-                                              const ShearIn& si, const PlainFactors& pf) {
+                                              const ShearIn& si, const PlainFactors& pf,
+                                              int64_t b_end_first) {
   const int lane = tid & 31, warp = tid >> 5;
   const int nb = a.nb, R = a.R;
   const bool active = tid < R * nb;
@@ -336,7 +384,7 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
     if (lane == 0) mbar_arrive(&statbar[k & 1]);
   };
 
-  int64_t b_end = 0;                              // first row past this thread's sample
+  int64_t b_end = b_end_first;                    // first row past this thread's sample
   uint4 cn[kAdaHalves][4];
   bool ok = n_local > 0;
   int read = 0;                                   // groups whose data arrived
@@ -505,30 +553,77 @@ __global__ void __launch_bounds__(kAdaCons, 1)
     mbar_init(&statbar[1], kAdaWarps);
     fence_mbar_init();
     tma_prefetch_map(&xmap);
+  }
+
+  const bool active = tid < a.R * a.nb;
+  const int j = active ? tid % a.nb : 0;
+  // Parameters and the first sample's modulation first: issued behind the
+  // tiles' DRAM traffic, these few L2 reads return microseconds late, and
+  // the first group's apply waits for them.  The CTA waits until they have
+  // arrived, then the first groups' loads go out.
+  float prm[15];
+  uint4 vs[4], vc[4];
+  int64_t b_first = -1;
+  float arrived = 0.0f;
+  if (active) {
+#pragma unroll
+    for (int t = 0; t < 15; ++t) prm[t] = a.params[(int64_t)j * 15 + t];
+    const int64_t row0 = (int64_t)blockIdx.x * (kAdaHalves * a.R) + tid / a.nb;
+    if ((int)blockIdx.x < a.groups && row0 < a.M) {
+      b_first = row0 / a.tokens;
+      read_modulation(a, b_first, j, vs, vc);
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        arrived += __uint_as_float((vs[t].x ^ vs[t].w) & 0x007FFFFFu) +
+                   __uint_as_float((vc[t].x ^ vc[t].w) & 0x007FFFFFu);
+    }
+#pragma unroll
+    for (int t = 0; t < 15; ++t) arrived += prm[t];
+  }
+  asm volatile("bar.sync 2, %0;" ::"r"(kAdaCons), "f"(arrived) : "memory");
+  // The raw words wait in this thread's slice of the table until the form
+  // is known (their registers are needed for the set-up).
+  if (b_first >= 0)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      reinterpret_cast<uint4*>(modtab)[t * kAdaCons + tid] = vs[t];
+      reinterpret_cast<uint4*>(modtab)[(4 + t) * kAdaCons + tid] = vc[t];
+    }
+  if (tid == 0) {
     // The first S groups of this CTA.
     for (int s = 0; s < S; ++s) {
       const int64_t g = (int64_t)blockIdx.x + (int64_t)s * gridDim.x;
       if (g < a.groups) adaln_issue(a, &xmap, stages + s * a.stage_bytes, &full[s], (int)g);
     }
   }
-
-  const bool active = tid < a.R * a.nb;
-  const int j = active ? tid % a.nb : 0;
   ShearIn si;
   PlainFactors pf;
   int plain = 0;
-  if (active) plain = load_shear_in(si, a.params + (int64_t)j * 15) ? 0 : 1;
+  if (active) plain = load_shear_in(si, prm) ? 0 : 1;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
       "bar.red.or.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}"
       : "=r"(plain)
       : "r"(plain), "r"(kAdaCons)
       : "memory");
+  // The first sample's table, from the words read above; the consumer
+  // loop reloads it only when its rows enter another sample.
+  const int64_t b_end_first = b_first >= 0 ? (b_first + 1) * a.tokens : 0;
+  if (b_first >= 0)
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      vs[t] = reinterpret_cast<const uint4*>(modtab)[t * kAdaCons + tid];
+      vc[t] = reinterpret_cast<const uint4*>(modtab)[(4 + t) * kAdaCons + tid];
+    }
   if (plain) {
-    if (active) load_plain(pf, a.params + (int64_t)j * 15);
-    adaln_consume<kOut, 1>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf);
+    if (active) load_plain(pf, prm);
+    if (b_first >= 0) write_modulation<1>(prm, vs, vc, tid, modtab);
+    adaln_consume<kOut, 1>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf,
+                           b_end_first);
   } else {
-    adaln_consume<kOut, 0>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf);
+    if (b_first >= 0) write_modulation<0>(prm, vs, vc, tid, modtab);
+    adaln_consume<kOut, 0>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf,
+                           b_end_first);
   }
 }
 

@@ -596,6 +596,36 @@ struct PGeom {
   static_assert(kSfCol0 + kStages * (kColsA + kColsB) <= kTmemCols, "TMEM columns");
 };
 
+// L2 policies: the operand tiles are read again by other tiles of the band
+// (kept), the output is written once (evicted first), so that the output
+// stream does not push the operands out of L2.
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int c0, int c1,
+                                                 uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, const void* src, int c0,
+                                                  int c1, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1],"
+      " %4;" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_addr(src)), "r"(c0), "r"(c1), "l"(pol)
+      : "memory");
+}
+
 // Tile t of the banded order (bands of kBandN column tiles, the row tile
 // changing fastest), for tiles of bn columns.
 __device__ __forceinline__ void tile_origin(const GemmArgs& a, int t, int& m0, int& n0,
@@ -657,6 +687,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (lane == 0) {
       tma_prefetch_map(&amap);
       tma_prefetch_map(&bmap);
+      const uint64_t pol_keep = policy_evict_last();
       int s = 0, issued = 0, g = 0;          // g: k-tiles issued over all tiles
       uint32_t phase = 0;
       bool ok = true;
@@ -680,8 +711,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
             bulk_load(sfa + P::kSfa + gb * P::kChunks * kSfChunk,
                       a.sb + ((int64_t)(n0 / 128 + gb) * a.sf_tiles_k + P::kChunks * kt) *
                                  kSfChunk, avail * kSfChunk, &full[s]);
-          tma_load_2d(stg, &amap, kt * kBKBytes, m0, &full[s]);
-          tma_load_2d(stg + kATile, &bmap, kt * kBKBytes, n0, &full[s]);
+          tma_load_2d_hint(stg, &amap, kt * kBKBytes, m0, &full[s], pol_keep);
+          tma_load_2d_hint(stg + kATile, &bmap, kt * kBKBytes, n0, &full[s], pol_keep);
           issued = g + 1;
           if (++s == P::kStages) {
             s = 0;
@@ -768,6 +799,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int quarter = warp & 3;
     const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16);
     uint8_t* wstage = staging + quarter * (kPBoxRows * 128);
+    const uint64_t pol_stream = policy_evict_first();
     uint8_t* srow = wstage + lane * 128;
     // Box `col` of this warp's rows: wait until its previous store has read
     // the slice, fill it, store it.
@@ -781,7 +813,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_store_2d(&cmap, wstage, col, m0 + quarter * kPBoxRows);
+        tma_store_2d_hint(&cmap, wstage, col, m0 + quarter * kPBoxRows, pol_stream);
         bulk_commit();
       }
     };
