@@ -553,6 +553,9 @@ __global__ void __launch_bounds__(kAdaCons, 1)
     mbar_init(&statbar[1], kAdaWarps);
     fence_mbar_init();
     tma_prefetch_map(&xmap);
+    // The first group alone goes out beside the parameter reads (one group
+    // per SM adds little to their wait), the rest after them.
+    if ((int)blockIdx.x < a.groups) adaln_issue(a, &xmap, stages, &full[0], (int)blockIdx.x);
   }
 
   const bool active = tid < a.R * a.nb;
@@ -590,8 +593,8 @@ __global__ void __launch_bounds__(kAdaCons, 1)
       reinterpret_cast<uint4*>(modtab)[(4 + t) * kAdaCons + tid] = vc[t];
     }
   if (tid == 0) {
-    // The first S groups of this CTA.
-    for (int s = 0; s < S; ++s) {
+    // The next S - 1 groups of this CTA.
+    for (int s = 1; s < S; ++s) {
       const int64_t g = (int64_t)blockIdx.x + (int64_t)s * gridDim.x;
       if (g < a.groups) adaln_issue(a, &xmap, stages + s * a.stage_bytes, &full[s], (int)g);
     }

@@ -446,18 +446,24 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
       for (int t = 0; t < kUnitParams; ++t) arrived += prm[t];
     }
   }
+  // The first tile alone goes out beside the parameter reads (one tile per
+  // SM adds little to their wait), the rest after them.
+  if (tid == kCons && n_local > 0) {
+    tma_prefetch_map(&xmap);
+    mbar_arrive_expect_tx(&full[0], a.tile_bytes);
+    tma_load_3d(stages, &xmap, 0, panel * a.W, k0 * (kRpt * a.R), &full[0]);
+  }
   asm volatile("bar.sync 2, %0;" ::"r"(Cfg::kThreads), "f"(arrived) : "memory");
 
   if (tid >= kCons) {
     if (tid == kCons) {
-      tma_prefetch_map(&xmap);
-      int issued = 0;
+      int issued = n_local > 0 ? 1 : 0;
       bool ok = true;
-      int s = 0;
+      int s = issued % S;
       uint32_t phase = 0;                 // parity of the empty-barrier phase to wait for
-      int row0 = k0 * (kRpt * a.R);
       const int row_step = cpp * (kRpt * a.R);
-      for (int i = 0; i < n_local; ++i) {
+      int row0 = k0 * (kRpt * a.R) + issued * row_step;
+      for (int i = issued; i < n_local; ++i) {
         if (i >= S && !mbar_wait(&empty[s], phase)) {
           ok = false;
           break;
