@@ -123,21 +123,26 @@ struct ShearIn {
 };
 
 // Fills the form for the block with parameters p[15]; false if the block
-// must take the plain four-term stages instead (a vanishing diagonal entry,
-// or intermediate growth above the bound of the output-side shear form).
+// must take the plain four-term stages instead (an entry outside the float32
+// set-up range, a vanishing diagonal entry, or intermediate growth above the
+// bound of the output-side shear form).  In float32, as for the output-side
+// form: r01 = c / b and r10 = a b / g11 by one corrected division each, the
+// latter from the exact split of a b and the pair form of g11.
 __device__ __forceinline__ bool load_shear_in(ShearIn& f, const float* p) {
-  double growth = 1.0;
   bool ok = true;
+  float growth = 1.0f;
   float r10[kFactors], r01[kFactors];
 #pragma unroll
   for (int k = 0; k < kFactors; ++k) {
-    double g00, g01, g10, g11;
-    factor_entries<false>(p, k, g00, g01, g10, g11);
-    const double ra = g10 * recip_d(g11), rb = g01 * recip_d(g00);
-    ok = ok && (g00 != 0.0) && (g11 != 0.0) && isfinite(ra) && isfinite(rb);
-    growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
-    r10[k] = (float)ra;
-    r01[k] = (float)rb;
+    const float a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
+    float hi, lo;
+    g11_pair(a, b, c, hi, lo);
+    ok = ok && in_setup_range(b) && in_setup_range(hi) && fabsf(a) <= 0x1p100f &&
+         fabsf(c) <= 0x1p100f;
+    const float ab = __fmul_rn(a, b);
+    r10[k] = div_pair(ab, hi, lo, __fmaf_rn(a, b, -ab));
+    r01[k] = div_pair(c, b, 0.0f);
+    growth = __fmul_rn(growth, fmaxf(1.0f + fabsf(r10[k]), 1.0f + fabsf(r01[k])));
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -146,7 +151,7 @@ __device__ __forceinline__ bool load_shear_in(ShearIn& f, const float* p) {
   }
   f.r10b = r10[4];
   f.r01b = r01[4];
-  return ok && growth <= kShearGrowthMax;
+  return ok && growth <= static_cast<float>(kShearGrowthMax);
 }
 
 __device__ __forceinline__ void shear_in_apply(f2 (&u)[16], const ShearIn& f) {
@@ -163,22 +168,16 @@ __device__ __forceinline__ void shear_in_apply(f2 (&u)[16], const ShearIn& f) {
 }
 
 // Entries 2m and 2m + 1 of the diagonal (x) diag(g00_k, g11_k) of the block
-// with parameters p[15], factor k on index bit 4 - k, formed in double and
-// rounded once.
+// with parameters p[15], factor k on index bit 4 - k (float32 set-up).
 __device__ __forceinline__ void diag_pairs(const float* p, f2 (&dl)[16]) {
-  double g00[kFactors], g11[kFactors];
+  float d0[kFactors], d1[kFactors];
 #pragma unroll
   for (int k = 0; k < kFactors; ++k) {
-    double e01, e10;
-    factor_entries<false>(p, k, g00[k], e01, e10, g11[k]);
+    float lo;
+    d0[k] = p[3 * k + 1];
+    g11_pair(p[3 * k + 0], p[3 * k + 1], p[3 * k + 2], d1[k], lo);
   }
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    double t = 1.0;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) t *= ((2 * m) >> (4 - k)) & 1 ? g11[k] : g00[k];
-    dl[m] = pack2((float)(t * g00[4]), (float)(t * g11[4]));
-  }
+  delta_tree<kFactors>(d0, d1, dl);
 }
 
 // Writes alpha = (1 + scale) delta and beta = shift delta of this thread's

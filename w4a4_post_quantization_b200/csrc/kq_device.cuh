@@ -300,30 +300,129 @@ __device__ __forceinline__ void factor_entries(const float* p, int k, double& g0
   }
 }
 
+// ------------------------------------------- float32 factor set-up
+// The shear form's coefficients are formed in float32 arithmetic, a few
+// operations per factor on the full-rate pipes: double-precision set-up
+// (conversions to and from double, double products) was measured to take
+// about 2 us at the start of every CTA, on the critical path of the small
+// DiT shapes.  The entries that are not exact products come out within about
+// one float32 ulp of the exact values:
+//   g11 = a c + 1/b   as an unevaluated pair hi + lo (error ~2^-44 |1/b|),
+//   c / g11           from the pair by one corrected division,
+//   delta_i           a product of five float entries, four roundings.
+// Any block whose entries leave [2^-100, 2^100] takes the plain form, whose
+// coefficients are still formed in double (factor_entries).
+
+// The hardware's approximate reciprocal (within about an ulp; inputs are
+// kept inside [2^-100, 2^100] by the callers, so flushing of subnormals
+// never applies).
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// g11 = a c + 1/b as hi + lo: an approximate reciprocal r of b and its
+// residual e = 1 - b r, exact in float32 since r is within about an ulp of
+// 1/b, so that 1/b = r (1 + e + e^2 + ...) = r + r e to about 2^-46
+// relative; the product a c split exactly by an fma (Dekker's product); the
+// two large terms added by a two-sum (Knuth), the small ones after.
+__device__ __forceinline__ void g11_pair(float a, float b, float c, float& hi, float& lo) {
+  const float r = rcp_approx(b);
+  const float e = __fmaf_rn(-b, r, 1.0f);
+  const float pc = __fmul_rn(a, c);
+  const float pe = __fmaf_rn(a, c, -pc);
+  const float s = __fadd_rn(pc, r);
+  const float v = __fsub_rn(s, pc);
+  const float t = __fadd_rn(__fsub_rn(pc, __fsub_rn(s, v)), __fsub_rn(r, v));
+  const float rest = __fadd_rn(t, __fmaf_rn(r, e, pe));
+  hi = __fadd_rn(s, rest);
+  lo = __fsub_rn(rest, __fsub_rn(hi, s));
+}
+
+// (n + nl) / (hi + lo): the quotient q = n r by an approximate reciprocal r
+// of hi, then one correction by its residual n + nl - q (hi + lo) (Newton's
+// step for a quotient, as in Markstein's division), which leaves it within
+// about an ulp.
+__device__ __forceinline__ float div_pair(float n, float hi, float lo, float nl = 0.0f) {
+  const float rh = rcp_approx(hi);
+  const float q = __fmul_rn(n, rh);
+  const float rem = __fmaf_rn(-q, lo, __fmaf_rn(-q, hi, n) + nl);
+  return __fmaf_rn(rem, rh, q);
+}
+
+__device__ __forceinline__ bool in_setup_range(float v) {
+  const float av = fabsf(v);
+  return av >= 0x1p-100f && av <= 0x1p100f;
+}
+
+// Diagonal entries (g00_k, g11_k) and shear ratios (r10_k, r01_k) of the
+// factors of one block, in float32; false if the block must take the plain
+// form (an entry outside the set-up range, a vanishing diagonal entry, or
+// intermediate growth above kShearGrowthMax).  nf factors, p[3 nf].  For
+// G_k itself r10 = g10 / g00 = a exactly; for (G_k^-1)^T (kInvT) the
+// entries are [[g11, -a b], [-c, b]], so r01 = -a exactly and
+// r10 = -c / g11.
+template <bool kInvT, int nf>
+__device__ __forceinline__ bool shear_factors(const float* p, float (&d0)[nf], float (&d1)[nf],
+                                              float (&r10)[nf], float (&r01)[nf]) {
+  bool ok = true;
+  float growth = 1.0f;
+#pragma unroll
+  for (int k = 0; k < nf; ++k) {
+    const float a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
+    float hi, lo;
+    g11_pair(a, b, c, hi, lo);
+    ok = ok && in_setup_range(b) && in_setup_range(hi) && fabsf(a) <= 0x1p100f &&
+         fabsf(c) <= 0x1p100f;
+    const float q = div_pair(c, hi, lo);
+    if (kInvT) {
+      d0[k] = hi;
+      d1[k] = b;
+      r10[k] = -q;
+      r01[k] = -a;
+    } else {
+      d0[k] = b;
+      d1[k] = hi;
+      r10[k] = a;
+      r01[k] = q;
+    }
+    growth = __fmul_rn(growth, fmaxf(1.0f + fabsf(r10[k]), 1.0f + fabsf(r01[k])));
+  }
+  // NaN fails the comparison as well.
+  return ok && growth <= static_cast<float>(kShearGrowthMax);
+}
+
+// delta pairs (delta_2m, delta_2m+1) of a block of 2^nf elements from its
+// factors' diagonal entries, factor k on index bit nf - 1 - k: a product
+// tree from the last factor up, two entries per packed multiply.
+template <int nf>
+__device__ __forceinline__ void delta_tree(const float (&d0)[nf], const float (&d1)[nf],
+                                           f2* out) {
+  constexpr int kPairs = 1 << (nf - 1);
+  f2 t[kPairs];
+  t[0] = pack2(d0[nf - 1], d1[nf - 1]);
+#pragma unroll
+  for (int k = nf - 2; k >= 0; --k) {
+    // Entries with bit (nf - 2 - k) of m clear take d0[k], set d1[k]; bit
+    // nf - 2 - k of m is the most significant of the bits built so far.
+    const f2 lo = pack2(d0[k], d0[k]), hi = pack2(d1[k], d1[k]);
+#pragma unroll
+    for (int m = 0; m < (1 << (nf - 2 - k)); ++m) {
+      t[m + (1 << (nf - 2 - k))] = mul2(t[m], hi);
+      t[m] = mul2(t[m], lo);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < kPairs; ++m) out[m] = t[m];
+}
+
 // Fills the shear form for the block with parameters p[15]; returns false if
-// the block must use the plain form instead.  The shear below a factor is
-// r10 = g10 / g00 (which is exactly a for G_k itself) and above it
-// r01 = g01 / g11.
+// the block must use the plain form instead.
 template <bool kInvT = false>
 __device__ __forceinline__ bool load_shear_diag(ShearDiag& f, const float* p) {
-  double g00[kFactors], g11[kFactors];
-  double growth = 1.0;
-  bool ok = true;
-  float r10[kFactors], r01[kFactors];
-#pragma unroll
-  for (int k = 0; k < kFactors; ++k) {
-    double a00, a01, a10, a11;
-    factor_entries<kInvT>(p, k, a00, a01, a10, a11);
-    g00[k] = a00;
-    g11[k] = a11;
-    const double ra = kInvT ? a10 * recip_d(a00) : static_cast<double>(p[3 * k + 0]);
-    const double rb = a01 * recip_d(a11);
-    ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
-    growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
-    r10[k] = (float)ra;
-    r01[k] = (float)rb;
-  }
-  ok = ok && (growth <= kShearGrowthMax);
+  float d0[kFactors], d1[kFactors], r10[kFactors], r01[kFactors];
+  const bool ok = shear_factors<kInvT, kFactors>(p, d0, d1, r10, r01);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     f.r10[k] = pack2(r10[k], r10[k]);
@@ -331,15 +430,7 @@ __device__ __forceinline__ bool load_shear_diag(ShearDiag& f, const float* p) {
   }
   f.r10b = r10[4];
   f.r01b = r01[4];
-#pragma unroll
-  for (int m = 0; m < 16; ++m) {
-    double d0 = 1.0, d1;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) d0 *= ((2 * m) >> (4 - k)) & 1 ? g11[k] : g00[k];
-    d1 = d0 * g11[4];
-    d0 = d0 * g00[4];
-    f.delta[m] = pack2((float)d0, (float)d1);
-  }
+  delta_tree<kFactors>(d0, d1, f.delta);
   return ok;
 }
 
@@ -441,24 +532,8 @@ __device__ __forceinline__ bool load_shear_diag16(ShearDiag16& f, const float* p
   bool ok = true;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const float* ph = p + 12 * h;
-    double g00[kFactors16], g11[kFactors16];
-    double growth = 1.0;
-    float r10[kFactors16], r01[kFactors16];
-#pragma unroll
-    for (int k = 0; k < kFactors16; ++k) {
-      double a00, a01, a10, a11;
-      factor_entries<kInvT>(ph, k, a00, a01, a10, a11);
-      g00[k] = a00;
-      g11[k] = a11;
-      const double ra = kInvT ? a10 * recip_d(a00) : static_cast<double>(ph[3 * k + 0]);
-      const double rb = a01 * recip_d(a11);
-      ok = ok && (a11 != 0.0) && (a00 != 0.0) && isfinite(rb) && isfinite(ra);
-      growth *= fmax(1.0 + fabs(ra), 1.0 + fabs(rb));
-      r10[k] = (float)ra;
-      r01[k] = (float)rb;
-    }
-    ok = ok && (growth <= kShearGrowthMax);
+    float d0[kFactors16], d1[kFactors16], r10[kFactors16], r01[kFactors16];
+    ok = shear_factors<kInvT, kFactors16>(p + 12 * h, d0, d1, r10, r01) && ok;
 #pragma unroll
     for (int k = 0; k < 3; ++k) {
       f.r10[h][k] = pack2(r10[k], r10[k]);
@@ -466,13 +541,7 @@ __device__ __forceinline__ bool load_shear_diag16(ShearDiag16& f, const float* p
     }
     f.r10b[h] = r10[3];
     f.r01b[h] = r01[3];
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      double d0 = 1.0;
-#pragma unroll
-      for (int k = 0; k < 3; ++k) d0 *= ((2 * m) >> (3 - k)) & 1 ? g11[k] : g00[k];
-      f.delta[8 * h + m] = pack2((float)(d0 * g00[3]), (float)(d0 * g11[3]));
-    }
+    delta_tree<kFactors16>(d0, d1, f.delta + 8 * h);
   }
   return ok;
 }
