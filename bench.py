@@ -17,6 +17,7 @@ collective on the data path); the time is the maximum over ranks.
 from __future__ import annotations
 
 import argparse
+import collections
 import hashlib
 import json
 import multiprocessing as mp
@@ -167,50 +168,61 @@ class ClockSampler:
 
     def _run(self):
         # Polls from construction on, so that the thread and NVML are warm
-        # when the timed region starts; keeps what it reads while recording.
+        # when the timed region starts; every poll is kept with the times
+        # its queries started and ended.
         n = self.nvml
         while not self._stop.is_set():
+            t0 = time.perf_counter()
             try:
                 mhz = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
                 mask = n.nvmlDeviceGetCurrentClocksEventReasons(self.h)
             except Exception as e:
                 self.error = repr(e)
                 return
-            if self._recording:
-                self.samples.append(mhz)
-                for k, bit in self.REASONS.items():
-                    if mask & bit:
-                        self.reasons.add(k)
+            self._polls.append((t0, time.perf_counter(), mhz, mask))
             time.sleep(self.period)
 
     def _arm(self):
-        self._recording = False
+        self._polls = collections.deque(maxlen=100000)
+        self._t_start = self._t_end = None
         if self.nvml is not None:
             self._thread = threading.Thread(target=self._run, daemon=True)
             self._thread.start()
 
     def start(self):
-        """Records from now on (call right before the timed region)."""
+        """Marks the start of the timed region (call right before it)."""
         if self._thread is not None:
             # A short interpreter switch interval lets the sampling thread
-            # run between the launching thread's calls during a timed
-            # region of a few milliseconds.
+            # run between the launching thread's calls.
             self._switch = sys.getswitchinterval()
             sys.setswitchinterval(5e-5)
-            self._recording = True
+        self._t_start = time.perf_counter()
 
     def stop(self):
+        """Ends the region.  A poll counts when its queries overlap the region
+        (an NVML query can take longer than a short region lasts)."""
+        self._t_end = time.perf_counter()
         if self._thread is not None:
-            self._recording = False
             self._stop.set()
             self._thread.join()
             if hasattr(self, "_switch"):
                 sys.setswitchinterval(self._switch)
+        ts, te = self._t_start, self._t_end
+        polls = [p for p in self._polls
+                 if ts is not None and p[1] >= ts and p[0] <= te]
+        self.samples = [p[2] for p in polls]
+        for _, _, _, mask in polls:
+            for k, bit in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(k)
+        durs = [p[1] - p[0] for p in self._polls]
         return {
             "sm_mhz": statistics.median(self.samples) if self.samples else None,
             "sm_max_mhz": self.max_mhz,
             "reasons": sorted(self.reasons),
             "samples": len(self.samples),
+            "region_ms": round((te - ts) * 1e3, 3) if ts is not None else None,
+            "poll_ms": round(statistics.median(durs) * 1e3, 3) if durs else None,
             "source": "nvml" if self.nvml is not None else f"unavailable: {self.error}",
         }
 

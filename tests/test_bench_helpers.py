@@ -64,3 +64,42 @@ def test_gemm_kernel_name_follows_the_library_switches(monkeypatch):
     assert bench.gemm_kernel_name().startswith("gemm_mxf4_kernel<")
     monkeypatch.setenv("KQ_GEMM_PERSISTENT", "x")              # atoi("x") == 0
     assert bench.gemm_kernel_name().startswith("gemm_mxf4_kernel<")
+
+
+class _FakeNvml:
+    """Stands in for pynvml: each query takes 2 ms (longer than a short timed
+    region) and reports a fixed clock with the power-cap reason set."""
+    NVML_CLOCK_SM = 0
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return i
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        import time
+        time.sleep(0.002)
+        return 1890
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4
+
+
+def test_clock_sampler_counts_polls_overlapping_a_short_region(monkeypatch):
+    import sys
+    import time
+    monkeypatch.setitem(sys.modules, "pynvml", _FakeNvml())
+    monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    s = bench.ClockSampler(0)
+    time.sleep(0.01)
+    s.start()
+    time.sleep(0.001)                  # a region shorter than one poll
+    rec = s.stop()
+    assert rec["source"] == "nvml"
+    assert rec["samples"] >= 1 and rec["sm_mhz"] == 1890 and rec["sm_max_mhz"] == 1965
+    assert rec["reasons"] == ["sw_power_cap"]
+    assert rec["poll_ms"] >= 1.0 and 0.5 <= rec["region_ms"] < 50
