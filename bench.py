@@ -573,7 +573,10 @@ def compact_summary(variants):
 # --------------------------------------------------------------- GPU leg
 def time_steps(fn, steps: int, warmup: int, stream, sampler=None):
     """Average ms per step over exactly ``steps`` calls, CUDA events on
-    ``stream``, barrier + synchronize on both sides."""
+    ``stream``, barrier + synchronize on both sides.  The calls are queued
+    behind a short device sleep and three untimed calls, so that the host's
+    per-call cost (argument checks, the launch) does not leave the GPU idle
+    between steps of under 100 us; the timed region holds the steps alone."""
     import torch
     import torch.distributed as dist
     for _ in range(warmup):
@@ -583,6 +586,9 @@ def time_steps(fn, steps: int, warmup: int, stream, sampler=None):
     sync()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(min(HOST_AHEAD_CYCLES, 150_000 * (steps + 3)))
+    for _ in range(3):
+        fn()
     if sampler is not None:
         sampler.start()
     start.record(stream)
@@ -873,7 +879,7 @@ def run_gpu(args):
                                    16 if args.op == "kron16" else 32,
                                    args.case or None), op=args.op,
                            launch=("cuda_graph: the K steps captured once, replayed once"
-                                   if args.launch == "graph" else "eager: one call per step"), global_batch_rows=M * world,
+                                   if args.launch == "graph" else "eager: one call per step, queued behind a device sleep"), global_batch_rows=M * world,
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3,
                            **({"gemm_shape_mnk": gemm_mnk} if args.op == "gemm" else {})),
             "hbm_frac": value / world / peak if args.op != "gemm" else None,
