@@ -75,14 +75,13 @@ constexpr int kTmemCols = 512;
 static_assert(kSfCol0 + kStages * (kSfColsA + kSfColsB) <= kTmemCols, "TMEM columns");
 
 // Instruction descriptor, block-scaled kinds: A and B E2M1 (format 1 of
-// kind::mxf4), K-major, N = 256, E8M0 scales, M = 128, dense K = 64.  The
+// kind::mxf4), K-major, N = bn, E8M0 scales, M = 128, dense K = 64.  The
 // scale-factor ids (byte of the 32-bit TMEM word holding the first scale of
 // the MMA's K range) go in bits 29-30 (A) and 4-5 (B).
 __host__ __device__ constexpr uint32_t idesc_mxf4(int bn) {
   return (1u << 7) | (1u << 10) | (uint32_t(bn >> 3) << 17) | (1u << 23) |
          (uint32_t(kBM >> 4) << 24);
 }
-constexpr uint32_t kIdescMxf4 = idesc_mxf4(kBN);
 
 struct GemmArgs {
   int32_t M, N, K;
