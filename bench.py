@@ -516,6 +516,11 @@ def layer_table(dev, stream, steps: int):
            "timing": "back to back, queued behind a device sleep (host cost hidden)",
            "rows": []}
     for label, M, N, K in LAYER_SHAPES:
+        # Each shape starts from an idle GPU: right after the square shape's
+        # bf16 products (tens of ms at the power cap) the short-K product
+        # measured a third slower than on its own.
+        torch.cuda.synchronize()
+        time.sleep(0.5)
         seed = 4242 + K
         p = torch.from_numpy(w.draw_params(K, seed)).to(dev)
         wt = w.device_randn_bf16((N, K), seed + 7, dev)
@@ -573,10 +578,9 @@ def compact_summary(variants):
 # --------------------------------------------------------------- GPU leg
 def time_steps(fn, steps: int, warmup: int, stream, sampler=None):
     """Average ms per step over exactly ``steps`` calls, CUDA events on
-    ``stream``, barrier + synchronize on both sides.  The calls are queued
-    behind a short device sleep and three untimed calls, so that the host's
-    per-call cost (argument checks, the launch) does not leave the GPU idle
-    between steps of under 100 us; the timed region holds the steps alone."""
+    ``stream``, barrier + synchronize on both sides.  (Queuing the calls
+    behind a device sleep measured 1-1.5 % slower at 20 steps on two boxes,
+    so the host enqueues them as they run.)"""
     import torch
     import torch.distributed as dist
     for _ in range(warmup):
@@ -586,9 +590,6 @@ def time_steps(fn, steps: int, warmup: int, stream, sampler=None):
     sync()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
-    torch.cuda._sleep(min(HOST_AHEAD_CYCLES, 150_000 * (steps + 3)))
-    for _ in range(3):
-        fn()
     if sampler is not None:
         sampler.start()
     start.record(stream)
@@ -879,7 +880,7 @@ def run_gpu(args):
                                    16 if args.op == "kron16" else 32,
                                    args.case or None), op=args.op,
                            launch=("cuda_graph: the K steps captured once, replayed once"
-                                   if args.launch == "graph" else "eager: one call per step, queued behind a device sleep"), global_batch_rows=M * world,
+                                   if args.launch == "graph" else "eager: one call per step"), global_batch_rows=M * world,
                            parallelism=f"row shards x{world}", clock_ramp_s=0.3,
                            **({"gemm_shape_mnk": gemm_mnk} if args.op == "gemm" else {})),
             "hbm_frac": value / world / peak if args.op != "gemm" else None,
