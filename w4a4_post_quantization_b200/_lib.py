@@ -112,7 +112,15 @@ def _check(name: str, status: int) -> None:
         raise KQError(name, status, lib())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device) -> int:
+    """The handle of the current stream of `device` (without building a
+    torch.cuda.Stream object per call where torch offers the raw query)."""
+    if _raw_stream is not None:
+        return _raw_stream(device.index if device.index is not None
+                           else torch.cuda.current_device())
     return torch.cuda.current_stream(device).cuda_stream
 
 
