@@ -96,9 +96,13 @@ int kq_quantize_smooth(const uint16_t* x, int64_t M, int64_t d, const float* inv
 /* y = x T in float32: the Kronecker block transform of kq_quantize (KroQuant
  * review, "What carries the argument": K^(j) = G1 (x) ... (x) G5 per 32-channel
  * block; "Circularity Check", Eq. 1: the activations are multiplied on the
- * right, A T), stopped before the quantizer, for parity checks.  Same
+ * right, A T), stopped before the quantizer, for parity checks, round trips
+ * and the calibration.  Computed in double (every factor entry and every
+ * stage) and rounded once to float32, so each value is within 2^-24 of
+ * itself but where its terms cancel by about ten decimal orders.  Same
  * arguments and layout as kq_quantize; y: [M][d] float32, 16-byte aligned,
- * written by the call.  KQ_ERR_INVALID for the same argument errors. */
+ * written by the call.  KQ_ERR_INVALID for the same argument errors.  The
+ * transform, inverse and fold calls below are computed the same way. */
 int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float* params,
                  float* y, void* stream);
 

@@ -138,11 +138,44 @@ def check_mx4(q_gpu, s_gpu, y64, cond, tol: float = TOL, strict_zero_sign: bool 
     }
 
 
-def relative_outside(y_gpu: np.ndarray, y64: np.ndarray, tol: float = TOL) -> int:
-    """Entries with |y_gpu - y64| > tol |y64|: those that pass the
-    componentwise bound only because their terms cancel."""
+# Absolute floors of the literal check: relative to the terms' magnitudes,
+# because a sum the oracle cancels to exactly zero may come out as a residue
+# of the double-precision rounding of its terms (about 1e-16 of them); and
+# one float32 subnormal step, below which no float32 output can be relatively
+# accurate.
+LITERAL_FLOOR = 1e-12
+F32_SUBNORMAL_STEP = 2.0 ** -149
+
+
+def relative_outside(y_gpu: np.ndarray, y64: np.ndarray, tol: float = TOL,
+                     cond: np.ndarray = None) -> int:
+    """Entries with |y_gpu - y64| > tol |y64| (+ LITERAL_FLOOR cond when the
+    terms' magnitudes are given): those that pass the componentwise bound
+    only because their terms cancel."""
     err = np.abs(np.asarray(y_gpu, dtype=np.float64) - y64)
-    return int((err > tol * np.abs(y64)).sum())
+    bound = tol * np.abs(y64) + F32_SUBNORMAL_STEP
+    if cond is not None:
+        bound = bound + LITERAL_FLOOR * cond
+    return int((err > bound).sum())
+
+
+def check_transform_literal(y_gpu: np.ndarray, y64: np.ndarray, cond: np.ndarray,
+                            tol: float = TOL) -> float:
+    """The literal reading of the transform tolerance: every float32 value
+    within tol of the oracle's value relative to that value itself (up to
+    LITERAL_FLOOR of the terms' magnitudes and one float32 subnormal step),
+    on top of the componentwise band.  Returns the worst
+    |y_gpu - y64| / |y64| over entries that are normal float32 values."""
+    check_transform(y_gpu, y64, cond, tol)
+    n = relative_outside(y_gpu, y64, tol, cond)
+    if n:
+        err = np.abs(np.asarray(y_gpu, dtype=np.float64) - y64)
+        bad = np.argwhere(err > tol * np.abs(y64) + LITERAL_FLOOR * cond + F32_SUBNORMAL_STEP)[:5]
+        detail = [(tuple(i), float(y_gpu[tuple(i)]), float(y64[tuple(i)])) for i in bad]
+        raise AssertionError(f"{n} transformed values outside {tol} relative: {detail}")
+    err = np.abs(np.asarray(y_gpu, dtype=np.float64) - y64)
+    nz = np.abs(y64) >= 2.0 ** -126
+    return float((err[nz] / np.abs(y64[nz])).max()) if nz.any() else 0.0
 
 
 def merge_stats(total: dict, part: dict) -> dict:
@@ -166,7 +199,7 @@ def check_chunk(job):
         y64 = o.transform(x64, aux)
         cond = o.abs_transform(x64, aux)
         st = {"worst_transform_ratio": check_transform(out["y"], y64, cond),
-              "transform_outside_relative": relative_outside(out["y"], y64)}
+              "transform_outside_relative": relative_outside(out["y"], y64, cond=cond)}
         st.update(check_mx4(out["q"], out["s"], y64, cond))
     elif kind == "hadamard":
         y64 = o.transform_hadamard(x64)

@@ -13,7 +13,7 @@ import torch
 
 import workloads as w
 from oracle import kq_oracle as o
-from tests.parity import TOL, check_mx4, check_transform
+from tests.parity import TOL, check_mx4, check_transform, check_transform_literal
 
 pytestmark = pytest.mark.gpu
 
@@ -39,6 +39,7 @@ def _check(x_bits, params16, q, s, y, bound=True):
     x64 = o.bf16_bits_to_float64(x_bits)
     y64 = o.transform16(x64, params16)
     cond = o.abs_transform16(x64, params16)
+    check_transform_literal(y, y64, cond)
     worst = check_transform(y, y64, cond)
     st = check_mx4(q, s, y64, cond, block=16)
     if bound:
@@ -160,7 +161,7 @@ def test_block16_weight_fold_and_quantizer():
     w64 = o.bf16_bits_to_float64(_bits(W))
     f64 = o.fold_weight16(w64, p16)
     cond = o.abs_fold_weight16(w64, p16)
-    check_transform(f.cpu().numpy(), f64, cond)
+    check_transform_literal(f.cpu().numpy(), f64, cond)
     st = check_mx4(q.cpu().numpy(), s.cpu().numpy(), f64, cond, block=16)
     assert st["scale_exempt"] <= 2 and st["code_exempt"] <= 8
 

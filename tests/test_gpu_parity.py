@@ -12,7 +12,7 @@ import torch
 
 import workloads as w
 from oracle import kq_oracle as o
-from tests.parity import TOL, check_mx4, check_transform
+from tests.parity import TOL, check_mx4, check_transform, check_transform_literal
 
 pytestmark = pytest.mark.gpu
 
@@ -50,6 +50,8 @@ def _check_rows(out, x_bits, params, inv_s, rows=None, bound_exemptions=True):
     x64 = o.bf16_bits_to_float64(x_bits)
     y64 = o.transform(x64, params)
     cond = o.abs_transform(x64, params)
+    # kq_transform runs in double: the literal 1e-5 relative bound holds.
+    check_transform_literal(out["y"], y64, cond)
     worst = check_transform(out["y"], y64, cond)
     st = check_mx4(out["q"], out["s"], y64, cond)
     yh = o.transform_hadamard(x64)
@@ -168,7 +170,7 @@ def test_singular_shear_factor_takes_the_plain_form():
     x64 = o.bf16_bits_to_float64(c.x_bits())
     y64 = o.transform(x64, p)
     cond = o.abs_transform(x64, p)
-    check_transform(y.cpu().numpy(), y64, cond)
+    check_transform_literal(y.cpu().numpy(), y64, cond)
     check_mx4(q.cpu().numpy(), s.cpu().numpy(), y64, cond)
 
 
@@ -289,7 +291,8 @@ def test_inverse_transform_and_round_trip():
     yr = (rng.standard_normal((97, c.d)) * 3).astype(np.float32)
     xg = kq.inverse_transform(_gpu(torch.from_numpy(yr)), pd).cpu().numpy()
     y64 = yr.astype(np.float64)
-    check_transform(xg, o.inverse_transform(y64, c.params), o.abs_inverse_transform(y64, c.params))
+    check_transform_literal(xg, o.inverse_transform(y64, c.params),
+                            o.abs_inverse_transform(y64, c.params))
     yt = kq.transform(_gpu(c.x), pd)
     back = kq.inverse_transform(yt, pd).cpu().numpy()
     x64 = o.bf16_bits_to_float64(c.x_bits())

@@ -13,7 +13,7 @@ import torch
 
 import workloads as w
 from oracle import kq_oracle as o
-from tests.parity import TOL, check_mx4, check_transform
+from tests.parity import TOL, check_mx4, check_transform, check_transform_literal
 
 pytestmark = pytest.mark.gpu
 
@@ -38,6 +38,7 @@ def _check(W, params, q, s, f, bound=True):
     w64 = o.bf16_bits_to_float64(_bits(W))
     f64 = o.fold_weight(w64, params)
     cond = o.abs_fold_weight(w64, params)
+    check_transform_literal(f, f64, cond)
     worst = check_transform(f, f64, cond)
     st = check_mx4(q, s, f64, cond)
     if bound:

@@ -5,7 +5,7 @@ import pytest
 
 import workloads as w
 from oracle import kq_oracle as o
-from tests.parity import check_mx4, check_transform, relative_outside
+from tests.parity import check_mx4, check_transform, check_transform_literal, relative_outside
 
 
 @pytest.fixture(scope="module")
@@ -102,3 +102,22 @@ def test_relative_outside_counts_cancelling_entries():
     y64 = np.array([[1.0, 1e-9, -2.0]])
     y_gpu = y64 + np.array([[1e-7, 1e-7, 0.0]])
     assert relative_outside(y_gpu, y64) == 1
+
+
+def test_literal_transform_check():
+    """The literal reading passes values within 1e-5 of themselves and a
+    double-precision residue where the oracle's sum is exactly zero, and
+    fails a cancelling entry that only the componentwise band would pass."""
+    y64 = np.array([[1.0, -2.0, 0.0, 1e-3]])
+    cond = np.array([[3.0, 4.0, 5.0, 10.0]])
+    ok = y64 * (1 + 5e-6)
+    ok[0, 2] = 1e-16                        # residue of an exact cancellation
+    assert check_transform_literal(ok, y64, cond) <= 5e-6 * 1.0001
+    bad = y64.copy()
+    bad[0, 3] = 1e-3 * (1 + 1e-3)           # 1e-6 of the terms, 1e-3 of the value
+    assert check_transform(bad, y64, cond) < 1e-5
+    with pytest.raises(AssertionError):
+        check_transform_literal(bad, y64, cond)
+    # A float32 subnormal output is within one subnormal step of the value.
+    tiny = np.array([[5.1000693571781566e-43]])
+    assert check_transform_literal(np.float32(tiny).astype(np.float64), tiny, tiny * 1e6) == 0.0

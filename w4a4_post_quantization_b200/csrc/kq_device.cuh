@@ -232,17 +232,12 @@ __device__ __forceinline__ void kron_apply(f2 (&u)[16], const float* entry) {
 }
 
 // Fills one table entry from the (a, b, c) parameters of a block; the four
-// entries of each G_k (or of G_k^-1 = [[G11, -G01], [-G10, G00]], det 1) are
-// formed in double and rounded once to float.
-__device__ __forceinline__ void kron_entry(float* entry, const float* p, bool inverse) {
+// entries of each G_k are formed in double and rounded once to float.
+__device__ __forceinline__ void kron_entry(float* entry, const float* p) {
 #pragma unroll
   for (int k = 0; k < kFactors; ++k) {
     const double a = p[3 * k + 0], b = p[3 * k + 1], c = p[3 * k + 2];
-    double g00 = b, g01 = c, g10 = a * b, g11 = __fma_rn(a, c, recip_d(b));
-    if (inverse) {
-      const double t00 = g11, t01 = -g01, t10 = -g10, t11 = g00;
-      g00 = t00; g01 = t01; g10 = t10; g11 = t11;
-    }
+    const double g00 = b, g01 = c, g10 = a * b, g11 = __fma_rn(a, c, recip_d(b));
     const float f00 = (float)g00, f01 = (float)g01, f10 = (float)g10, f11 = (float)g11;
     float4* e = reinterpret_cast<float4*>(entry + 8 * k);
     e[0] = make_float4(f00, f00, f10, f10);

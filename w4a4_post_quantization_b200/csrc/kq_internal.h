@@ -35,6 +35,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // Device address of the library's device-side error word on device `dev`.
 int device_error_word(int dev, int** out);
 
+// The float32 outputs of the block transforms computed in double
+// (kq_exact.cu): kind 0 = x K, 1 = x K^-1, 2 = x K^-T; nf = 5 (32-element
+// blocks) or 4 (16-element blocks, two a 32-element unit); f32_in: float32
+// input (else bf16).  Shapes and pointers checked by the caller.
+int exact_transform(int kind, int nf, bool f32_in, const void* x, int64_t M, int64_t d,
+                    const float* params, float* y, cudaStream_t st);
+
 // Sets the dynamic shared-memory limit of one kernel once per device.
 template <auto kKernel>
 int allow_smem(int bytes, int dev) {

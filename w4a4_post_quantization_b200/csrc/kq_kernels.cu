@@ -61,7 +61,6 @@ struct LaunchArgs {
   int32_t nb;           // 32-blocks per row
   int32_t n_tiles;      // ceil(G / kTile)
   int32_t stages;       // TMA ring depth
-  int32_t inverse;      // table from G_k^-1 instead of G_k
   const float* aux;     // params [nb][5][3] (Kronecker) or inv_s [nb*32] (smooth)
   uint8_t* q;           // [G][16] packed codes
   uint8_t* scales;      // [G] scale bytes
@@ -75,7 +74,7 @@ template <int kXf>
 __device__ __forceinline__ void build_table(float* tab, const LaunchArgs& a, int j0, int jn,
                                             int t, int nt) {
   if (kXf == kXfKron) {
-    for (int j = t; j < jn; j += nt) kron_entry(tab + j * kTabStride, a.aux + (j0 + j) * 15, a.inverse);
+    for (int j = t; j < jn; j += nt) kron_entry(tab + j * kTabStride, a.aux + (j0 + j) * 15);
   } else if (kXf == kXfSmooth) {
     const float4* src = reinterpret_cast<const float4*>(a.aux + (int64_t)j0 * kBlock);
     float4* dst = reinterpret_cast<float4*>(tab);
@@ -529,10 +528,10 @@ __global__ void __launch_bounds__(Cfg::kThreads, Cfg::kMinBlocks)
 // ---------------------------------------------------------- direct kernel
 // Grid (row groups, column panels of kDirectThreads blocks); thread t of
 // panel p handles column block 256 p + t of rows blockIdx.x, +gridDim.x, ...
-// Input is bf16 (four 16-byte loads per block) or float32 (eight).
-template <int kXf, int kOut, bool kF32In>
+// (four 16-byte bf16 loads per block).
+template <int kXf, int kOut>
 __global__ void __launch_bounds__(kDirectThreads)
-    direct_kernel(const void* __restrict__ xin, int64_t M, const LaunchArgs a) {
+    direct_kernel(const uint16_t* __restrict__ xin, int64_t M, const LaunchArgs a) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   float* tab = reinterpret_cast<float*>(smem_raw);
   pdl_wait_then_trigger();     // programmatic dependent launch: no global access before
@@ -545,24 +544,14 @@ __global__ void __launch_bounds__(kDirectThreads)
   for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
     const int64_t g = r * a.nb + j0 + t;
     f2 u[16];
-    if (!kF32In) {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(xin) + g * kBlock);
+    const uint4* src = reinterpret_cast<const uint4*>(xin + g * kBlock);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 c = __ldg(src + q);
-        u[4 * q + 0] = bf16x2_to_f2(c.x);
-        u[4 * q + 1] = bf16x2_to_f2(c.y);
-        u[4 * q + 2] = bf16x2_to_f2(c.z);
-        u[4 * q + 3] = bf16x2_to_f2(c.w);
-      }
-    } else {
-      const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(xin) + g * kBlock);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 v = __ldcs(src + i);
-        u[2 * i] = pack2(v.x, v.y);
-        u[2 * i + 1] = pack2(v.z, v.w);
-      }
+    for (int q = 0; q < 4; ++q) {
+      const uint4 c = __ldg(src + q);
+      u[4 * q + 0] = bf16x2_to_f2(c.x);
+      u[4 * q + 1] = bf16x2_to_f2(c.y);
+      u[4 * q + 2] = bf16x2_to_f2(c.z);
+      u[4 * q + 3] = bf16x2_to_f2(c.w);
     }
     apply_xform<kXf>(u, tab, t);
     store_block<kOut>(u, a, g);
@@ -894,13 +883,13 @@ bool panel_fits(int64_t M, int nb, int sms) {
   }
 }
 
-template <int kXf, int kOut, bool kF32In>
-int launch_direct(const void* x, int64_t M, int64_t d, LaunchArgs a, cudaStream_t st,
+template <int kXf, int kOut>
+int launch_direct(const uint16_t* x, int64_t M, int64_t d, LaunchArgs a, cudaStream_t st,
                   const DeviceInfo& di, int dev) {
   const int nb = static_cast<int>(d / kBlock);
   const int panels = (nb + kDirectThreads - 1) / kDirectThreads;
   const int smem = table_floats(kXf, std::min(nb, kDirectThreads)) * 4;
-  int rc = allow_smem<direct_kernel<kXf, kOut, kF32In>>(std::max(smem, 1), dev);
+  int rc = allow_smem<direct_kernel<kXf, kOut>>(std::max(smem, 1), dev);
   if (rc != KQ_OK) return rc;
   a.nb = nb;
   a.G = M * nb;
@@ -908,7 +897,7 @@ int launch_direct(const void* x, int64_t M, int64_t d, LaunchArgs a, cudaStream_
   const int rows = static_cast<int>(std::min<int64_t>(M, std::min<int64_t>(want, 65535)));
   dim3 grid(rows, panels);
   {
-    cudaError_t le = launch_pdl(direct_kernel<kXf, kOut, kF32In>, grid, dim3(kDirectThreads), smem,
+    cudaError_t le = launch_pdl(direct_kernel<kXf, kOut>, grid, dim3(kDirectThreads), smem,
                                 st, x, M, a);
     if (le != cudaSuccess) return cuda_fail(le);
   }
@@ -929,7 +918,6 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
   a.q = q;
   a.scales = scales;
   a.y = y;
-  a.inverse = 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int64_t nb = d / kBlock;
   if constexpr (kron4(kXf) || kXf == kXfKronInvT) {
@@ -957,7 +945,7 @@ int run(const uint16_t* x, int64_t M, int64_t d, const float* aux, uint8_t* q, u
       return launch_panel<kXf, kOut>(x, M, d, aux, q, scales, y, st, *di, dev);
     }
     if (impl == KQ_IMPL_TMA) return launch_tma<kXf, kOut>(x, M, d, a, st, *di, dev);
-    if (impl == KQ_IMPL_DIRECT) return launch_direct<kXf, kOut, false>(x, M, d, a, st, *di, dev);
+    if (impl == KQ_IMPL_DIRECT) return launch_direct<kXf, kOut>(x, M, d, a, st, *di, dev);
     return KQ_ERR_INVALID;
   }
 }
@@ -1029,7 +1017,7 @@ extern "C" int kq_transform(const uint16_t* x, int64_t M, int64_t d, const float
   if (rc != KQ_OK || M == 0) return rc;
   if (!x || !params || !y || !aligned(x, 16) || !aligned(y, 16) || !aligned(params, 4))
     return KQ_ERR_INVALID;
-  return run<kXfKron, kOutF32>(x, M, d, params, nullptr, nullptr, y, KQ_IMPL_AUTO, stream);
+  return exact_transform(0, 5, false, x, M, d, params, y, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int kq_quantize16(const uint16_t* x, int64_t M, int64_t d, const float* params16,
@@ -1048,7 +1036,7 @@ extern "C" int kq_transform16(const uint16_t* x, int64_t M, int64_t d, const flo
   if (!x || !params16 || !y || !aligned(x, 16) || !aligned(y, 16) || !aligned(params16, 4) ||
       d / kBlock > 65535)
     return KQ_ERR_INVALID;
-  return run<kXfKron16, kOutF32>(x, M, d, params16, nullptr, nullptr, y, KQ_IMPL_PANEL, stream);
+  return exact_transform(0, 4, false, x, M, d, params16, y, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int kq_quantize16_tiled(const uint16_t* x, int64_t M, int64_t d,
@@ -1086,8 +1074,8 @@ extern "C" int kq_fold_weight16(const uint16_t* w, int64_t N, int64_t d, const f
   if (!w || !params16 || !w_folded || !aligned(w, 16) || !aligned(w_folded, 16) ||
       !aligned(params16, 4) || d / kBlock > 65535)
     return KQ_ERR_INVALID;
-  return run<kXfKron16InvT, kOutF32>(w, N, d, params16, nullptr, nullptr, w_folded,
-                                     KQ_IMPL_PANEL, stream);
+  return exact_transform(2, 4, false, w, N, d, params16, w_folded,
+                         static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int kq_quantize_weight(const uint16_t* w, int64_t N, int64_t d, const float* params,
@@ -1106,8 +1094,8 @@ extern "C" int kq_fold_weight(const uint16_t* w, int64_t N, int64_t d, const flo
   if (!w || !params || !w_folded || !aligned(w, 16) || !aligned(w_folded, 16) ||
       !aligned(params, 4) || d / kBlock > 65535)
     return KQ_ERR_INVALID;
-  return run<kXfKronInvT, kOutF32>(w, N, d, params, nullptr, nullptr, w_folded, KQ_IMPL_PANEL,
-                                   stream);
+  return exact_transform(2, 5, false, w, N, d, params, w_folded,
+                         static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int kq_quantize_tiled(const uint16_t* x, int64_t M, int64_t d, const float* params,
@@ -1131,16 +1119,7 @@ extern "C" int kq_inverse_transform(const float* y, int64_t M, int64_t d, const 
   if (rc != KQ_OK || M == 0) return rc;
   if (!y || !params || !x || !aligned(y, 16) || !aligned(x, 16) || !aligned(params, 4))
     return KQ_ERR_INVALID;
-  const DeviceInfo* di = nullptr;
-  int dev = 0;
-  rc = device_info(&di, &dev);
-  if (rc != KQ_OK) return rc;
-  LaunchArgs a{};
-  a.aux = params;
-  a.y = x;
-  a.inverse = 1;
-  return launch_direct<kXfKron, kOutF32, true>(y, M, d, a, static_cast<cudaStream_t>(stream), *di,
-                                               dev);
+  return exact_transform(1, 5, true, y, M, d, params, x, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int kq_dequantize(const uint8_t* q_packed, const uint8_t* scales, int64_t M, int64_t d,
