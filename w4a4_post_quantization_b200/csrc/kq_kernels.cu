@@ -1,13 +1,16 @@
 // Kernels of the KroQuant quantizer library and their launchers.
 //
-// Hot path (kq_quantize): one thread owns one 32-element block.  x is staged
-// into shared memory by TMA tile loads (64-byte swizzle, so that the
-// thread-per-block reads are bank-conflict free) through a ring of stages
-// guarded by mbarriers; a producer warp issues the loads and eight consumer
-// warps run the butterfly, the block maximum, the E8M0 scale and the E2M1
-// conversion, and store 16 bytes of codes and one scale byte per block.
-// CTAs are persistent (one per SM) and walk the flat list of blocks
-// (row-major, so block g is row g / nb, column block g % nb).
+// Hot path (kq_quantize): the panel kernel.  One thread owns one 32-element
+// block of a row at a time and keeps its column block, so its factors stay
+// in registers.  A CTA (one per SM, persistent) owns a column panel of W
+// blocks and walks the panel's row tiles; x is staged into shared memory by
+// 3-D TMA boxes (64-byte swizzle, so that the thread-per-block reads are
+// bank-conflict free) through a ring of stages guarded by mbarriers.  A
+// producer warp issues the loads; 12 to 16 consumer warps run the scaled
+// shear butterfly, the diagonal, the block maximum, the E8M0 scale and the
+// E2M1 conversion, and store 16 bytes of codes and one scale byte per block.
+// The flat-tile TMA kernel and the direct kernel below serve the shapes the
+// panel does not fit, and the measurements.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
