@@ -283,7 +283,9 @@ int kq_scales_to_tiled(const uint8_t* scales, int64_t rows, int64_t K, uint8_t* 
                        void* stream);
 
 /* x = y T^-1 in float32 with T^-1 = diag(G1^-1 (x) ... (x) G5^-1) (review,
- * axiom ledger: the inverse of a Kronecker product factorizes). */
+ * axiom ledger: the inverse of a Kronecker product factorizes), computed in
+ * double and rounded once as kq_transform is.  y: [M][d] float32, x: [M][d]
+ * float32, both 16-byte aligned; params as for kq_quantize. */
 int kq_inverse_transform(const float* y, int64_t M, int64_t d, const float* params,
                          float* x, void* stream);
 
