@@ -111,3 +111,27 @@ def test_abs_gradient_bounds_the_gradient():
     for inv in (False, True):
         assert (np.abs(c.transform_params_grad(x, g, p, inv)) <=
                 c.abs_transform_params_grad(x, g, p, inv) * (1 + 1e-12)).all()
+
+
+def test_calibration_loop_starts_at_three_output_losses_and_steps_by_adam():
+    """The loop's first recorded loss is L_out + lam_a L_A + lam_w L_W at the
+    Hadamard start, which the Eq. 10 weights make exactly 3 L_out; its first
+    step is bias-corrected Adam's, a move of lr g / (|g| + eps) against the
+    straight-through gradient, and its parameters come back in float32."""
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((16, 64))
+    x[:, 7] *= 30
+    w = rng.standard_normal((8, 64)) / 8
+    p0 = c.hadamard_params(2)
+    l_out, _, _ = c.losses(x, w, p0)
+    p1, hist, (lam_a, lam_w) = c.calibrate(x, w, steps=1, lr=1e-3)
+    assert len(hist) == 1 and math.isclose(hist[0], 3 * l_out, rel_tol=1e-12)
+    assert p1.dtype == np.float32 and p1.shape == p0.shape
+    _, _, g = c.loss_and_grad(x, w, p0, lam_a, lam_w)
+    step = p1.astype(np.float64) - p0.astype(np.float64)
+    np.testing.assert_allclose(step, -1e-3 * g / (np.abs(g) + c.ADAM_EPS), rtol=0, atol=1e-7)
+    # a second step continues from the first, with the moments carried over
+    p2, hist2, _ = c.calibrate(x, w, steps=2, lr=1e-3)
+    assert hist2[0] == hist[0] and np.array_equal(
+        c.calibrate(x, w, steps=1, lr=1e-3, params0=p0)[0], p1)
+    assert not np.array_equal(p2, p1)

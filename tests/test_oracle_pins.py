@@ -603,6 +603,28 @@ def test_fold_weight16_keeps_the_layer_output_eq1():
     np.testing.assert_allclose(lhs, x @ W.T, rtol=1e-10, atol=1e-10)
 
 
+def test_quantize_weight16_with_identity_or_orthonormal_factors():
+    """With G_k = I the 16-element fold is the identity, so the block-16
+    weight quantizer gives quantize16's bytes on the same bf16 matrix; with
+    an orthonormal block (K^-T = K) it quantizes the transformed rows."""
+    rng = np.random.default_rng(43)
+    W = rng.standard_normal((10, 64)).astype(np.float32)
+    W[:, 5] *= 40.0
+    Wb = (W.view(np.uint32) >> 16).astype(np.uint16)
+    p = np.zeros((4, 4, 3), dtype=np.float32)
+    p[:, :, 1] = 1.0
+    qw, sw = o.quantize_weight16(Wb, p)
+    qa, sa = o.quantize16(Wb, p)
+    assert sw.shape == (10, 4) and qw.shape == (10, 32)
+    assert np.array_equal(qw, qa) and np.array_equal(sw, sa)
+    s2 = 1 / math.sqrt(2)
+    p = np.tile(np.array([-1.0, s2, s2], dtype=np.float32), (4, 4, 1))
+    qw, sw = o.quantize_weight16(Wb, p)
+    qa, sa = o.quantize16(Wb, p)
+    assert np.array_equal(sw, sa)
+    assert (o.unpack_codes(qw) != o.unpack_codes(qa)).mean() < 0.01
+
+
 def test_block16_product_brute_force():
     """mxfp4_gemm with 16-element scale blocks against a triple loop over
     hand-decoded values."""
