@@ -139,12 +139,13 @@ def test_adaln_rejects_bad_arguments_and_no_wait_gave_up():
     assert kq.device_status() == 0
 
 
-def test_adaln_tiled_scales_feed_the_tiled_gemm():
+@pytest.mark.parametrize("name,di,T", [("pixart_sigma", 0, 128), ("flux_schnell", 1, 75)])
+def test_adaln_tiled_scales_feed_the_tiled_gemm(name, di, T):
     """kq_quantize_adaln_tiled writes the same codes and the tiled image of
     the row-major scales; the normalized layer's product through the tiled
-    GEMM equals the row-major one bit for bit."""
-    c = w.make_case("pixart_sigma", 0, 0, M=300)
-    T = 128
+    GEMM equals the row-major one bit for bit.  The wide case pairs a
+    thread's two rows and straddles samples (75 tokens a sample)."""
+    c = w.make_case(name, di, 0, M=300)
     shift, scale = w.draw_adaln(-(-c.M // T), c.d, c.seed)
     xd, sd, cd = c.x.to(DEV), shift.to(DEV), scale.to(DEV)
     pd = torch.from_numpy(c.params).to(DEV)

@@ -53,6 +53,12 @@ constexpr int kAdaMaxRows = 256;                  // TMA box limit on a group's 
 constexpr int kAdaMaxHalfRows = kAdaMaxRows / kAdaHalves;
 constexpr int kAdaSlots = kAdaWarps + kAdaMaxHalfRows;   // segment slots per half
 constexpr int kAdaSlotBufs = 4;
+// Rows of at least this many blocks (d >= 3072) take the paired apply:
+// one pass over the modulation table for a thread's two rows when they
+// belong to one sample.  Narrower rows keep the one-row apply, whose
+// register allocation does not spill (the paired form was measured 2-4 %
+// slower there and 1-3 % faster on wider rows).
+constexpr int kAdaPairMinBlocks = 96;
 
 struct AdaArgs {
   int64_t M;
@@ -283,7 +289,7 @@ __device__ __forceinline__ void adaln_issue(const AdaArgs& a, const CUtensorMap*
 // rows and a thread takes block j of rows rr and R + rr, so the two rows'
 // reductions run side by side and a group's latency is paid once per 64
 // elements of each thread.
-template <int kOut, int kForm>
+template <int kOut, int kForm, bool kPair>
 __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMap* xmap,
                                               uint8_t* stages, uint64_t* full, uint64_t* statbar,
                                               float4* slots, float4* modtab, int tid,
@@ -459,19 +465,92 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
         }
       }
     }
+    // Transform and encode one modulated row block.
+    auto emit = [&](int64_t row, f2 (&u)[16]) {
+      if (kForm == 1) {
+        plain_apply(u, pf);
+      } else {
+        shear_in_apply(u, si);
+      }
+      const int64_t gi = row * nb + j;
+      if (kOut == 0) {
+        const Mx4Block blk = mxfp4_block(u);
+        __stcs(reinterpret_cast<uint4*>(a.q + gi * 16), blk.codes);
+        if (a.scale_tiles_k == 0) {
+          a.scales[gi] = static_cast<uint8_t>(blk.scale);
+        } else {
+          // Tiled layout: 128-row x 4-scale tiles, row r = r0 + 32 r1 and
+          // scale i at byte 16 r0 + 4 r1 + i; the row's last block also
+          // zeroes the padding of its 4-scale column.
+          const int rl = static_cast<int>(row & 127);
+          const int64_t o = ((row >> 7) * a.scale_tiles_k + (j >> 2)) * 512 + 16 * (rl & 31) +
+                            4 * (rl >> 5) + (j & 3);
+          a.scales[o] = static_cast<uint8_t>(blk.scale);
+          if (j == nb - 1)
+            for (int t = (j & 3) + 1; t < 4; ++t) a.scales[o + t - (j & 3)] = 0;
+        }
+      } else {
+        float4* dst = reinterpret_cast<float4*>(a.y + gi * 32);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          float x0, x1, x2, x3;
+          unpack2(u[2 * t], x0, x1);
+          unpack2(u[2 * t + 1], x2, x3);
+          __stcs(dst + t, make_float4(x0, x1, x2, x3));
+        }
+      }
+    };
+    const int64_t row0 =
+        ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * (kAdaHalves * R) + rr;
+    if (!active || row0 >= a.M) continue;
+    if (row0 >= b_end) {                          // rows only grow: a new sample
+      const int64_t b = row0 / a.tokens;
+      b_end = (b + 1) * a.tokens;
+      load_modulation<kForm>(a, b, j, tid, modtab);
+    }
+    const int64_t row1 = row0 + R;
+    const float rstd0 = rsqrtf(__fmaf_rn(m2[0], inv_d, a.eps));
+    const f2 r20 = pack2(rstd0, rstd0), nm0 = pack2(-mean[0] * rstd0, -mean[0] * rstd0);
+    if (kPair && row1 < a.M && row1 < b_end) {
+      // Both rows in one sample: one pass over the modulation table for
+      // both (half the table reads; the second row's modulated values wait
+      // in registers while the first is transformed and encoded).
+      const float rstd1 = rsqrtf(__fmaf_rn(m2[1], inv_d, a.eps));
+      const f2 r21 = pack2(rstd1, rstd1), nm1 = pack2(-mean[1] * rstd1, -mean[1] * rstd1);
+      f2 u0[16], u1[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 al0 = modtab[(2 * q) * kAdaCons + tid];
+        const float4 al1 = modtab[(2 * q + 1) * kAdaCons + tid];
+        const float4 be0 = modtab[(8 + 2 * q) * kAdaCons + tid];
+        const float4 be1 = modtab[(8 + 2 * q + 1) * kAdaCons + tid];
+        const f2 A0 = pack2(al0.x, al0.y), A1 = pack2(al0.z, al0.w);
+        const f2 A2 = pack2(al1.x, al1.y), A3 = pack2(al1.z, al1.w);
+        const f2 B0 = pack2(be0.x, be0.y), B1 = pack2(be0.z, be0.w);
+        const f2 B2 = pack2(be1.x, be1.y), B3 = pack2(be1.z, be1.w);
+        u0[4 * q + 0] = fma2(fma2(bf16x2_to_f2(cc[0][q].x), r20, nm0), A0, B0);
+        u0[4 * q + 1] = fma2(fma2(bf16x2_to_f2(cc[0][q].y), r20, nm0), A1, B1);
+        u0[4 * q + 2] = fma2(fma2(bf16x2_to_f2(cc[0][q].z), r20, nm0), A2, B2);
+        u0[4 * q + 3] = fma2(fma2(bf16x2_to_f2(cc[0][q].w), r20, nm0), A3, B3);
+        u1[4 * q + 0] = fma2(fma2(bf16x2_to_f2(cc[1][q].x), r21, nm1), A0, B0);
+        u1[4 * q + 1] = fma2(fma2(bf16x2_to_f2(cc[1][q].y), r21, nm1), A1, B1);
+        u1[4 * q + 2] = fma2(fma2(bf16x2_to_f2(cc[1][q].z), r21, nm1), A2, B2);
+        u1[4 * q + 3] = fma2(fma2(bf16x2_to_f2(cc[1][q].w), r21, nm1), A3, B3);
+      }
+      emit(row0, u0);
+      emit(row1, u1);
+      continue;
+    }
 #pragma unroll
     for (int h = 0; h < kAdaHalves; ++h) {
-    const int64_t row =
-        ((int64_t)blockIdx.x + (int64_t)i * gridDim.x) * (kAdaHalves * R) + h * R + rr;
-    if (!active || row >= a.M) continue;
+    const int64_t row = row0 + (int64_t)h * R;
+    if (row >= a.M) continue;
     if (row >= b_end) {                           // rows only grow: a new sample
       const int64_t b = row / a.tokens;
       b_end = (b + 1) * a.tokens;
       load_modulation<kForm>(a, b, j, tid, modtab);
     }
-    // rsqrtf: within 2 ulp, far inside the 1e-5 band of the modulated value.
-    const float rstd = rsqrtf(__fmaf_rn(m2[h], inv_d, a.eps));
-    // h D = t alpha + beta with t = x rstd - mean rstd.
+    const float rstd = h == 0 ? rstd0 : rsqrtf(__fmaf_rn(m2[h], inv_d, a.eps));
     const f2 r2 = pack2(rstd, rstd), nmr2 = pack2(-mean[h] * rstd, -mean[h] * rstd);
     f2 u[16];
 #pragma unroll
@@ -489,38 +568,7 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
       u[4 * q + 3] = fma2(fma2(bf16x2_to_f2(cc[h][q].w), r2, nmr2), pack2(al1.z, al1.w),
                           pack2(be1.z, be1.w));
     }
-    if (kForm == 1) {
-      plain_apply(u, pf);
-    } else {
-      shear_in_apply(u, si);
-    }
-    const int64_t gi = row * nb + j;
-    if (kOut == 0) {
-      const Mx4Block blk = mxfp4_block(u);
-      __stcs(reinterpret_cast<uint4*>(a.q + gi * 16), blk.codes);
-      if (a.scale_tiles_k == 0) {
-        a.scales[gi] = static_cast<uint8_t>(blk.scale);
-      } else {
-        // Tiled layout: 128-row x 4-scale tiles, row r = r0 + 32 r1 and
-        // scale i at byte 16 r0 + 4 r1 + i; the row's last block also
-        // zeroes the padding of its 4-scale column.
-        const int rl = static_cast<int>(row & 127);
-        const int64_t o = ((row >> 7) * a.scale_tiles_k + (j >> 2)) * 512 + 16 * (rl & 31) +
-                          4 * (rl >> 5) + (j & 3);
-        a.scales[o] = static_cast<uint8_t>(blk.scale);
-        if (j == nb - 1)
-          for (int t = (j & 3) + 1; t < 4; ++t) a.scales[o + t - (j & 3)] = 0;
-      }
-    } else {
-      float4* dst = reinterpret_cast<float4*>(a.y + gi * 32);
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        float x0, x1, x2, x3;
-        unpack2(u[2 * t], x0, x1);
-        unpack2(u[2 * t + 1], x2, x3);
-        __stcs(dst + t, make_float4(x0, x1, x2, x3));
-      }
-    }
+    emit(row, u);
     }
   }
   if (!ok) {
@@ -531,7 +579,7 @@ __device__ __forceinline__ void adaln_consume(const AdaArgs& a, const CUtensorMa
   }
 }
 
-template <int kOut>
+template <int kOut, bool kPair>
 __global__ void __launch_bounds__(kAdaCons, 1)
     adaln_kernel(const __grid_constant__ CUtensorMap xmap, const AdaArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -620,13 +668,24 @@ __global__ void __launch_bounds__(kAdaCons, 1)
   if (plain) {
     if (active) load_plain(pf, prm);
     if (b_first >= 0) write_modulation<1>(prm, vs, vc, tid, modtab);
-    adaln_consume<kOut, 1>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf,
+    adaln_consume<kOut, 1, kPair>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf,
                            b_end_first);
   } else {
     if (b_first >= 0) write_modulation<0>(prm, vs, vc, tid, modtab);
-    adaln_consume<kOut, 0>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf,
+    adaln_consume<kOut, 0, kPair>(a, &xmap, stages, full, statbar, slots, modtab, tid, si, pf,
                            b_end_first);
   }
+}
+
+template <int kOut, bool kPair>
+int launch_adaln_kernel(const CUtensorMap& map, const AdaArgs& a, int grid, int smem, int dev,
+                        cudaStream_t st) {
+  int rc = allow_smem<adaln_kernel<kOut, kPair>>(smem, dev);
+  if (rc != KQ_OK) return rc;
+  cudaError_t e =
+      launch_pdl(adaln_kernel<kOut, kPair>, dim3(grid), dim3(kAdaCons), smem, st, map, a);
+  if (e != cudaSuccess) return record_cuda_error(e);
+  return KQ_OK;
 }
 
 // Launches the fused kernel; the shapes were checked by the caller.
@@ -689,16 +748,13 @@ int launch_adaln(const uint16_t* x, int64_t M, int64_t d, const uint16_t* shift,
   if (cr != CUDA_SUCCESS) return record_cuda_error(cudaErrorInvalidValue);
   const int grid = static_cast<int>(std::min<int64_t>(groups, di->sms));
   if (y) {
-    rc = allow_smem<adaln_kernel<1>>(smem, dev);
-    if (rc != KQ_OK) return rc;
-    cudaError_t e = launch_pdl(adaln_kernel<1>, dim3(grid), dim3(kAdaCons), smem, st, map, a);
-    if (e != cudaSuccess) return record_cuda_error(e);
+    rc = launch_adaln_kernel<1, false>(map, a, grid, smem, dev, st);
+  } else if (nb >= kAdaPairMinBlocks) {
+    rc = launch_adaln_kernel<0, true>(map, a, grid, smem, dev, st);
   } else {
-    rc = allow_smem<adaln_kernel<0>>(smem, dev);
-    if (rc != KQ_OK) return rc;
-    cudaError_t e = launch_pdl(adaln_kernel<0>, dim3(grid), dim3(kAdaCons), smem, st, map, a);
-    if (e != cudaSuccess) return record_cuda_error(e);
+    rc = launch_adaln_kernel<0, false>(map, a, grid, smem, dev, st);
   }
+  if (rc != KQ_OK) return rc;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return record_cuda_error(e);
   return KQ_OK;
