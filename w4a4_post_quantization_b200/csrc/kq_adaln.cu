@@ -32,6 +32,8 @@
 // channel, followed by the shear stages.  A thread keeps column block j for
 // the whole kernel, so it recomputes its block's alpha and beta only when its
 // rows enter a new sample, into a slice of shared memory that only it reads.
+// On wide rows a thread's two rows of a group share one pass over that slice
+// when they belong to the same sample.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
